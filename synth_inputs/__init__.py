@@ -1,0 +1,225 @@
+"""Seeded synthetic inputs for the batch-1 Llama decode step.
+
+This module is shared by the oracle tests, the CUDA-path tests and the bench.
+It only draws random numbers and lays them out; it holds none of the decode
+step's arithmetic (no norm, matvec, RoPE, attention or softmax).
+
+Recipe (the pages run random-init models of published shapes; no trained
+weights are needed or used):
+
+* linear and embedding weights: N(0, 0.02) drawn in fp32, rounded to bf16
+  (round-to-nearest-even, which is what ``torch.Tensor.to(torch.bfloat16)``
+  does);
+* RMSNorm gains: 1 + N(0, 0.01), rounded to bf16, so that a dropped gain
+  multiply cannot hide behind gains equal to one;
+* W8A16 weights: from the same N(0, 0.02) fp32 masters, one symmetric scale
+  per output row, ``s = fp16(max|w_row| / 127)`` and
+  ``q = clamp(round_half_even(w / s), -127, 127)`` (a row of zeros gets s = 1,
+  q = 0).  The decode step consumes q and s; neither side re-quantises;
+* prompt token ids: uniform in [0, vocab);
+* synthetic KV-cache fill for long contexts: N(0, 1) rounded to bf16.
+
+Every tensor is drawn from its own generator whose seed is derived from the
+base seed and the tensor's name, so the bytes do not depend on the order in
+which tensors are made.  The same call on the same device type gives the same
+bytes; CPU and CUDA generators give different (equally valid) bytes, so a test
+draws once and hands the identical bytes to both sides.
+"""
+from __future__ import annotations
+
+import dataclasses
+import hashlib
+from typing import Dict, List, Optional
+
+import torch
+
+__all__ = [
+    "ModelConfig",
+    "CONFIGS",
+    "get_config",
+    "make_model",
+    "make_prompt",
+    "make_kv_fill",
+    "model_bytes",
+]
+
+
+@dataclasses.dataclass(frozen=True)
+class ModelConfig:
+    name: str
+    hidden: int
+    n_layers: int
+    n_heads: int
+    n_kv_heads: int
+    head_dim: int
+    ffn: int
+    vocab: int
+    max_ctx: int
+    rms_eps: float = 1e-5
+    rope_theta: float = 1e4
+    tied: bool = False
+    quant: str = "bf16"  # "bf16" or "w8a16"
+
+    @property
+    def q_rows(self) -> int:
+        return self.n_heads * self.head_dim
+
+    @property
+    def kv_rows(self) -> int:
+        return self.n_kv_heads * self.head_dim
+
+    def with_(self, **kw) -> "ModelConfig":
+        return dataclasses.replace(self, **kw)
+
+
+# The five workloads: a tiny decoder, then random-init models shaped like
+# SmolLM2-135M, TinyLlama-1.1B, Llama-1B (W8A16) and Llama-7B (bf16 and W8A16).
+CONFIGS: Dict[str, ModelConfig] = {
+    "tiny": ModelConfig("tiny", 64, 2, 4, 2, 16, 172, 256, max_ctx=32),
+    "smol135": ModelConfig("smol135", 576, 30, 9, 3, 64, 1536, 49152,
+                           max_ctx=256, tied=True),
+    "tinyllama": ModelConfig("tinyllama", 2048, 22, 32, 4, 64, 5632, 32000,
+                             max_ctx=1088),
+    "llama1b_w8": ModelConfig("llama1b_w8", 2048, 16, 32, 8, 64, 8192, 128256,
+                              max_ctx=576, quant="w8a16"),
+    "llama7b": ModelConfig("llama7b", 4096, 32, 32, 32, 128, 11008, 32000,
+                           max_ctx=2112),
+    "llama7b_w8": ModelConfig("llama7b_w8", 4096, 32, 32, 32, 128, 11008,
+                              32000, max_ctx=2112, quant="w8a16"),
+}
+
+
+def get_config(name_or_cfg) -> ModelConfig:
+    if isinstance(name_or_cfg, ModelConfig):
+        return name_or_cfg
+    return CONFIGS[name_or_cfg]
+
+
+def _seed_for(seed: int, name: str) -> int:
+    h = hashlib.sha256(f"{seed}/{name}".encode()).digest()
+    return int.from_bytes(h[:8], "little") & ((1 << 63) - 1)
+
+
+def _gen(device, seed: int, name: str) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(_seed_for(seed, name))
+    return g
+
+
+def _normal(shape, std, device, seed, name) -> torch.Tensor:
+    g = _gen(device, seed, name)
+    return torch.randn(shape, generator=g, device=device,
+                       dtype=torch.float32).mul_(std)
+
+
+def _bf16_normal(shape, std, device, seed, name) -> torch.Tensor:
+    return _normal(shape, std, device, seed, name).to(torch.bfloat16)
+
+
+def _gain(n, device, seed, name) -> torch.Tensor:
+    return (_normal((n,), 0.01, device, seed, name) + 1.0).to(torch.bfloat16)
+
+
+def _int8_rows(shape, device, seed, name):
+    """Per-output-row symmetric int8 weights from N(0, 0.02) fp32 masters."""
+    w = _normal(shape, 0.02, device, seed, name)
+    amax = w.abs().amax(dim=1)
+    s = (amax / 127.0).to(torch.float16)
+    s = torch.where(amax == 0, torch.ones_like(s), s)
+    q = torch.round(w / s.to(torch.float32)[:, None]).clamp_(-127, 127)
+    q = torch.where((amax == 0)[:, None], torch.zeros_like(q), q)
+    del w
+    return q.to(torch.int8), s
+
+
+def make_model(cfg, seed: int = 0, device="cpu") -> Dict[str, object]:
+    """Random-init weights of ``cfg``'s shape.
+
+    Returns a dict with tensors on ``device``:
+      embed [vocab, hidden] bf16; final_norm [hidden] bf16;
+      lm_head [vocab, hidden] bf16 or int8 (None when tied);
+      lm_head_scale [vocab] fp16 (W8A16 and untied only, else None);
+      per-layer lists attn_norm, ffn_norm [hidden] bf16;
+      wq [nh*hd, hidden], wk/wv [nkv*hd, hidden], wo [hidden, nh*hd],
+      wgate/wup [ffn, hidden], wdown [hidden, ffn] (bf16, or int8), and for
+      W8A16 the fp16 row scales sq, sk, sv, so, sgate, sup, sdown.
+    All weights are row-major [out, in].
+    """
+    cfg = get_config(cfg)
+    h, L = cfg.hidden, cfg.n_layers
+    q8 = cfg.quant == "w8a16"
+    m: Dict[str, object] = {}
+    m["embed"] = _bf16_normal((cfg.vocab, h), 0.02, device, seed, "embed")
+    m["final_norm"] = _gain(h, device, seed, "final_norm")
+    m["lm_head"] = None
+    m["lm_head_scale"] = None
+    if not cfg.tied:
+        if q8:
+            m["lm_head"], m["lm_head_scale"] = _int8_rows(
+                (cfg.vocab, h), device, seed, "lm_head")
+        else:
+            m["lm_head"] = _bf16_normal((cfg.vocab, h), 0.02, device, seed,
+                                        "lm_head")
+    shapes = {
+        "wq": (cfg.q_rows, h),
+        "wk": (cfg.kv_rows, h),
+        "wv": (cfg.kv_rows, h),
+        "wo": (h, cfg.q_rows),
+        "wgate": (cfg.ffn, h),
+        "wup": (cfg.ffn, h),
+        "wdown": (h, cfg.ffn),
+    }
+    for key in ("attn_norm", "ffn_norm", *shapes):
+        m[key] = []
+    for key in shapes:
+        m["s" + key[1:]] = [] if q8 else None
+    for layer in range(L):
+        m["attn_norm"].append(_gain(h, device, seed, f"l{layer}.attn_norm"))
+        m["ffn_norm"].append(_gain(h, device, seed, f"l{layer}.ffn_norm"))
+        for key, shp in shapes.items():
+            name = f"l{layer}.{key}"
+            if q8:
+                q, s = _int8_rows(shp, device, seed, name)
+                m[key].append(q)
+                m["s" + key[1:]].append(s)
+            else:
+                m[key].append(_bf16_normal(shp, 0.02, device, seed, name))
+    return m
+
+
+def make_prompt(cfg, n: int, seed: int = 1, device="cpu") -> List[int]:
+    """``n`` uniform token ids in [0, vocab)."""
+    cfg = get_config(cfg)
+    g = _gen(device, seed, "prompt")
+    t = torch.randint(0, cfg.vocab, (n,), generator=g, device=device)
+    return [int(v) for v in t.tolist()]
+
+
+def make_kv_fill(cfg, ctx: int, seed: int = 2, device="cpu",
+                 layers: Optional[int] = None) -> torch.Tensor:
+    """Synthetic KV-cache rows 0..ctx-1: bf16 N(0,1), shape
+    [n_layers, 2, n_kv_heads, ctx, head_dim] (index 0 = K, 1 = V)."""
+    cfg = get_config(cfg)
+    L = cfg.n_layers if layers is None else layers
+    shape = (L, 2, cfg.n_kv_heads, ctx, cfg.head_dim)
+    return _bf16_normal(shape, 1.0, device, seed, "kvfill")
+
+
+def model_bytes(cfg) -> Dict[str, int]:
+    """Byte counts of the stored weights (for roofline bookkeeping)."""
+    cfg = get_config(cfg)
+    h, L = cfg.hidden, cfg.n_layers
+    wb = 1 if cfg.quant == "w8a16" else 2
+    per_layer_params = (cfg.q_rows * h + 2 * cfg.kv_rows * h + h * cfg.q_rows
+                        + 3 * cfg.ffn * h)
+    per_layer_rows = (cfg.q_rows + 2 * cfg.kv_rows + h + 2 * cfg.ffn + h)
+    linear = L * per_layer_params * wb
+    scales = L * per_layer_rows * 2 if wb == 1 else 0
+    head = 0 if cfg.tied else cfg.vocab * h * wb
+    head_scales = cfg.vocab * 2 if (wb == 1 and not cfg.tied) else 0
+    norms = (2 * L + 1) * h * 2
+    return {
+        "linear": linear, "scales": scales + head_scales, "head": head,
+        "norms": norms, "embed_row": h * 2,
+        "embed_table": cfg.vocab * h * 2,
+    }
