@@ -1,0 +1,603 @@
+// amk_host.cpp -- the C ABI of libamk (declared in include/amk.h): handle
+// lifetime, device memory, the per-token cooperative launch and error
+// reporting.
+//
+// "RightNow-AI/AutoMegaKernel" README, opening summary and "What is built and
+// verified": one launch per token, a KV cache carried across steps, and an
+// unsafe schedule rejected at validation instead of hanging the GPU
+// ("Deadlock-free by construction").
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "amk.h"
+#include "amk_internal.h"
+#include "amk_plan.h"
+
+using amk::ErrorWord;
+using amk::KParams;
+using amk::LayerPtrs;
+using amk::TaskDesc;
+
+extern "C" cudaError_t amk_kernel_configure(int smem_bytes);
+extern "C" cudaError_t amk_kernel_occupancy(int smem_bytes, int *blocks_per_sm);
+namespace amk {
+extern "C" cudaError_t amk_kernel_launch(const KParams *p, int n_ctas, int smem_bytes,
+                                         cudaStream_t stream);
+}
+
+namespace {
+thread_local char g_last_error[512] = "";
+}
+
+extern "C" int amk_set_error(int code, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+extern "C" const char *amk_last_error(void) { return g_last_error; }
+
+extern "C" const char *amk_version(void) { return "amk-b200 0.1 (sm_100a)"; }
+
+extern "C" const char *amk_strerror(int s)
+{
+    switch (s) {
+    case AMK_OK: return "ok";
+    case AMK_ERR_INVALID_ARG: return "invalid argument";
+    case AMK_ERR_UNSUPPORTED: return "unsupported shape";
+    case AMK_ERR_VALIDATION: return "schedule rejected by the validator";
+    case AMK_ERR_POS_RANGE: return "position or token out of range";
+    case AMK_ERR_LAUNCH: return "cooperative launch refused";
+    case AMK_ERR_TIMEOUT: return "device wait timed out";
+    case AMK_ERR_CUDA: return "CUDA runtime error";
+    case AMK_ERR_OOM: return "device allocation failed";
+    case AMK_ERR_POISONED: return "handle poisoned by an earlier timeout; call amk_reset_kv";
+    case AMK_ERR_NO_DEVICE: return "no CUDA device";
+    default: return "unknown status";
+    }
+}
+
+extern "C" int amk_default_options(amk_options *o)
+{
+    if (!o)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_default_options: NULL");
+    memset(o, 0, sizeof *o);
+    o->ring_stages = 6;
+    o->stage_bytes = 32768;
+    o->attn_splits = 0;
+    o->tasks_per_sm = 1;
+    o->n_sms = 0;
+    o->wait_timeout_us = 1000000;  // 1 s
+    o->debug_skip_signal_task = -1;
+    return AMK_OK;
+}
+
+// ---------------------------------------------------------------- host plans
+extern "C" int amk_plan_create(const amk_config *cfg, const amk_options *opt, int32_t n_sms,
+                               amk_plan **out, amk_validation_report *report)
+{
+    if (!cfg || !out)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_plan_create: NULL argument");
+    *out = nullptr;
+    amk_plan *P = new (std::nothrow) amk_plan();
+    if (!P)
+        return amk_set_error(AMK_ERR_OOM, "amk_plan_create: out of host memory");
+    int rc = amk_lower(cfg, opt, n_sms, P);
+    if (rc == AMK_OK) {
+        amk_graph g;
+        amk_plan_view(P, &g);
+        amk_validation_report local;
+        rc = amk_validate_graph(&g, report ? report : &local);
+        if (rc != AMK_OK)
+            amk_set_error(rc, "lowered schedule rejected: %s",
+                          (report ? report : &local)->message);
+    }
+    if (rc != AMK_OK) {
+        delete P;
+        return rc;
+    }
+    *out = P;
+    return AMK_OK;
+}
+
+extern "C" int amk_plan_graph(const amk_plan *p, amk_graph *out)
+{
+    if (!p || !out)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_plan_graph: NULL argument");
+    amk_plan_view(p, out);
+    return AMK_OK;
+}
+
+extern "C" int amk_plan_task_info(const amk_plan *p, int32_t *kind, int32_t *layer)
+{
+    if (!p)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_plan_task_info: NULL plan");
+    const size_t n = p->tasks.size();
+    if (kind)
+        memcpy(kind, p->kind.data(), n * sizeof(int32_t));
+    if (layer)
+        memcpy(layer, p->layer.data(), n * sizeof(int32_t));
+    return AMK_OK;
+}
+
+extern "C" void amk_plan_destroy(amk_plan *p) { delete p; }
+
+// ---------------------------------------------------------------- handles
+struct amk_handle {
+    amk_plan *plan = nullptr;
+    int device = 0;
+    cudaStream_t stream = nullptr;
+    std::vector<void *> dev_allocs;
+    TaskDesc *d_tasks = nullptr;
+    int32_t *d_qoff = nullptr;
+    uint32_t *d_ctr = nullptr;
+    ErrorWord *d_err = nullptr;
+    LayerPtrs *d_layers = nullptr;
+    float *d_qkv = nullptr, *d_part = nullptr, *d_xmid = nullptr, *d_xout = nullptr;
+    float *d_act = nullptr, *d_logits = nullptr;
+    unsigned long long *d_argkey = nullptr;
+    uint16_t *d_kv = nullptr;
+    size_t kv_bytes = 0, act_bytes = 0;
+    ErrorWord *h_err = nullptr;            // pinned
+    unsigned long long *h_key = nullptr;   // pinned
+    cudaEvent_t err_ev = nullptr;
+    bool err_pending = false;
+    KParams kp{};
+    uint32_t epoch = 0;
+    bool poisoned = false;
+    amk_error_info last_err{};
+};
+
+namespace {
+
+int cuda_fail(cudaError_t e, const char *what)
+{
+    return amk_set_error(e == cudaErrorMemoryAllocation ? AMK_ERR_OOM : AMK_ERR_CUDA, "%s: %s",
+                         what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return p && ((uintptr_t)p % 16) == 0; }
+
+template <typename T>
+int dalloc(amk_handle *H, T **out, size_t bytes)
+{
+    void *p = nullptr;
+    cudaError_t e = cudaMalloc(&p, bytes ? bytes : 16);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaMalloc");
+    H->dev_allocs.push_back(p);
+    *out = static_cast<T *>(p);
+    return AMK_OK;
+}
+
+void free_handle(amk_handle *H)
+{
+    if (!H)
+        return;
+    if (H->stream)
+        cudaStreamSynchronize(H->stream);
+    for (void *p : H->dev_allocs)
+        cudaFree(p);
+    if (H->h_err)
+        cudaFreeHost(H->h_err);
+    if (H->h_key)
+        cudaFreeHost(H->h_key);
+    if (H->err_ev)
+        cudaEventDestroy(H->err_ev);
+    delete H->plan;
+    delete H;
+}
+
+int check_weights(const amk_config *c, const amk_weights *w)
+{
+    if (!aligned16(w->embed) || !aligned16(w->final_norm))
+        return amk_set_error(AMK_ERR_INVALID_ARG, "embed/final_norm NULL or not 16-byte aligned");
+    if (!c->tied_embeddings) {
+        if (!aligned16(w->lm_head))
+            return amk_set_error(AMK_ERR_INVALID_ARG, "lm_head NULL or not 16-byte aligned");
+        if (c->quant == AMK_QUANT_W8A16 && !w->lm_head_scale)
+            return amk_set_error(AMK_ERR_INVALID_ARG, "lm_head_scale NULL for W8A16");
+    }
+    const void *const *mats[7] = {w->wq, w->wk, w->wv, w->wo, w->wgate, w->wup, w->wdown};
+    const void *const *scs[7] = {w->sq, w->sk, w->sv, w->so, w->sgate, w->sup, w->sdown};
+    if (!w->attn_norm || !w->ffn_norm)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "norm pointer arrays NULL");
+    for (int m = 0; m < 7; ++m) {
+        if (!mats[m])
+            return amk_set_error(AMK_ERR_INVALID_ARG, "weight pointer array %d NULL", m);
+        if (c->quant == AMK_QUANT_W8A16 && !scs[m])
+            return amk_set_error(AMK_ERR_INVALID_ARG, "scale pointer array %d NULL", m);
+    }
+    for (int l = 0; l < c->n_layers; ++l) {
+        if (!aligned16(w->attn_norm[l]) || !aligned16(w->ffn_norm[l]))
+            return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d norm NULL or misaligned", l);
+        for (int m = 0; m < 7; ++m) {
+            if (!aligned16(mats[m][l]))
+                return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d weight %d NULL or not "
+                                     "16-byte aligned", l, m);
+            if (c->quant == AMK_QUANT_W8A16 && !scs[m][l])
+                return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d scale %d NULL", l, m);
+        }
+    }
+    return AMK_OK;
+}
+
+int zero_state(amk_handle *H)
+{
+    const amk_plan *P = H->plan;
+    cudaError_t e;
+    e = cudaMemsetAsync(H->d_kv, 0, H->kv_bytes, H->stream);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(H->d_ctr, 0, sizeof(uint32_t) * (size_t)P->n_counters, H->stream);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(H->d_err, 0, sizeof(ErrorWord), H->stream);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(H->d_argkey, 0, 2 * sizeof(unsigned long long), H->stream);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(H->d_qkv, 0, H->act_bytes, H->stream);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "amk_reset_kv");
+    H->epoch = 0;
+    H->poisoned = false;
+    H->err_pending = false;
+    memset(&H->last_err, 0, sizeof H->last_err);
+    return AMK_OK;
+}
+
+// Maps a device error word to a status; poisons the handle on failure.
+int absorb_error(amk_handle *H, const ErrorWord &e)
+{
+    if (e.code == 0)
+        return AMK_OK;
+    H->poisoned = true;
+    H->last_err.code = (int32_t)e.code;
+    H->last_err.task = e.task;
+    H->last_err.counter = e.counter;
+    H->last_err.sm = e.sm;
+    H->last_err.seen = e.seen;
+    H->last_err.target = e.target;
+    if (e.code == 3)
+        return amk_set_error(AMK_ERR_POS_RANGE, "device token out of range (%u)", e.seen);
+    return amk_set_error(AMK_ERR_TIMEOUT, "device wait timed out (code %u, task %d, counter "
+                         "%d, sm %d, seen %u, needed %u)", e.code, e.task, e.counter, e.sm,
+                         e.seen, e.target);
+}
+
+}  // namespace
+
+extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk_options *opt,
+                          void *cuda_stream, amk_handle **out)
+{
+    if (!cfg || !w || !out)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_create: NULL argument");
+    *out = nullptr;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+        cudaGetLastError();
+        return amk_set_error(AMK_ERR_NO_DEVICE, "amk_create: no CUDA device");
+    }
+    int rc = check_weights(cfg, w);
+    if (rc != AMK_OK)
+        return rc;
+    amk_handle *H = new (std::nothrow) amk_handle();
+    if (!H)
+        return amk_set_error(AMK_ERR_OOM, "amk_create: out of host memory");
+    cudaGetDevice(&H->device);
+    H->stream = static_cast<cudaStream_t>(cuda_stream);
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, H->device);
+    int n_sms = (opt && opt->n_sms > 0) ? opt->n_sms : sms;
+    if (n_sms > sms) {
+        delete H;
+        return amk_set_error(AMK_ERR_INVALID_ARG, "n_sms %d > %d SMs on the device", n_sms, sms);
+    }
+    amk_validation_report rep;
+    rc = amk_plan_create(cfg, opt, n_sms, &H->plan, &rep);
+    if (rc != AMK_OK) {
+        delete H;
+        return rc;
+    }
+    const amk_plan *P = H->plan;
+    cudaError_t e = amk_kernel_configure(P->smem_bytes);
+    if (e != cudaSuccess) {
+        free_handle(H);
+        return cuda_fail(e, "cudaFuncSetAttribute");
+    }
+    int per_sm = 0;
+    e = amk_kernel_occupancy(P->smem_bytes, &per_sm);
+    if (e != cudaSuccess || per_sm < 1) {
+        free_handle(H);
+        return amk_set_error(AMK_ERR_LAUNCH, "kernel does not fit one SM (smem %d B)",
+                             P->smem_bytes);
+    }
+    const amk_config &c = P->cfg;
+    const int L = c.n_layers, nkv = c.n_kv_heads, hd = c.head_dim;
+    const size_t part_floats = (size_t)nkv * P->opt.attn_splits * P->group * (hd + 2);
+    const size_t qkv_f = (size_t)L * P->qkv_rows, part_f = (size_t)L * part_floats;
+    const size_t h_f = (size_t)L * c.hidden, act_f = (size_t)L * c.ffn;
+    H->kv_bytes = (size_t)L * 2 * nkv * c.max_ctx * hd * sizeof(uint16_t);
+    // activations in one block: qkv | part | xmid | xout | act
+    H->act_bytes = (qkv_f + part_f + 2 * h_f + act_f) * sizeof(float);
+    float *act_block = nullptr;
+    if ((rc = dalloc(H, &H->d_tasks, sizeof(TaskDesc) * P->tasks.size())) ||
+        (rc = dalloc(H, &H->d_qoff, sizeof(int32_t) * P->queue_off.size())) ||
+        (rc = dalloc(H, &H->d_ctr, sizeof(uint32_t) * (size_t)P->n_counters)) ||
+        (rc = dalloc(H, &H->d_err, sizeof(ErrorWord))) ||
+        (rc = dalloc(H, &H->d_layers, sizeof(LayerPtrs) * (size_t)L)) ||
+        (rc = dalloc(H, &act_block, H->act_bytes)) ||
+        (rc = dalloc(H, &H->d_logits, sizeof(float) * (size_t)c.vocab)) ||
+        (rc = dalloc(H, &H->d_argkey, 2 * sizeof(unsigned long long))) ||
+        (rc = dalloc(H, &H->d_kv, H->kv_bytes))) {
+        free_handle(H);
+        return rc;
+    }
+    H->d_qkv = act_block;
+    H->d_part = H->d_qkv + qkv_f;
+    H->d_xmid = H->d_part + part_f;
+    H->d_xout = H->d_xmid + h_f;
+    H->d_act = H->d_xout + h_f;
+    if ((e = cudaMallocHost(&H->h_err, sizeof(ErrorWord))) != cudaSuccess ||
+        (e = cudaMallocHost(&H->h_key, 2 * sizeof(unsigned long long))) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&H->err_ev, cudaEventDisableTiming)) != cudaSuccess) {
+        free_handle(H);
+        return cuda_fail(e, "host buffers");
+    }
+    std::vector<LayerPtrs> lp(L);
+    const void *const *mats[7] = {w->wq, w->wk, w->wv, w->wo, w->wgate, w->wup, w->wdown};
+    const void *const *scs[7] = {w->sq, w->sk, w->sv, w->so, w->sgate, w->sup, w->sdown};
+    const bool q8 = c.quant == AMK_QUANT_W8A16;
+    for (int l = 0; l < L; ++l) {
+        for (int m = 0; m < 7; ++m) {
+            lp[l].w[m] = mats[m][l];
+            lp[l].s[m] = q8 ? static_cast<const uint16_t *>(scs[m][l]) : nullptr;
+        }
+        lp[l].attn_norm = static_cast<const uint16_t *>(w->attn_norm[l]);
+        lp[l].ffn_norm = static_cast<const uint16_t *>(w->ffn_norm[l]);
+    }
+    if ((e = cudaMemcpyAsync(H->d_tasks, P->tasks.data(), sizeof(TaskDesc) * P->tasks.size(),
+                             cudaMemcpyHostToDevice, H->stream)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(H->d_qoff, P->queue_off.data(),
+                             sizeof(int32_t) * P->queue_off.size(), cudaMemcpyHostToDevice,
+                             H->stream)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(H->d_layers, lp.data(), sizeof(LayerPtrs) * lp.size(),
+                             cudaMemcpyHostToDevice, H->stream)) != cudaSuccess) {
+        free_handle(H);
+        return cuda_fail(e, "upload schedule");
+    }
+    if ((rc = zero_state(H)) != AMK_OK) {
+        free_handle(H);
+        return rc;
+    }
+    if ((e = cudaStreamSynchronize(H->stream)) != cudaSuccess) {
+        free_handle(H);
+        return cuda_fail(e, "amk_create");
+    }
+    KParams &k = H->kp;
+    k.tasks = H->d_tasks;
+    k.queue_off = H->d_qoff;
+    k.counters = H->d_ctr;
+    k.err = H->d_err;
+    k.layers = H->d_layers;
+    k.embed = static_cast<const uint16_t *>(w->embed);
+    k.final_norm = static_cast<const uint16_t *>(w->final_norm);
+    k.lm_head = static_cast<const uint16_t *>(c.tied_embeddings ? w->embed : w->lm_head);
+    k.lm_head_scale = (q8 && !c.tied_embeddings) ? static_cast<const uint16_t *>(w->lm_head_scale)
+                                                  : nullptr;
+    k.qkv = H->d_qkv;
+    k.part = H->d_part;
+    k.xmid = H->d_xmid;
+    k.xout = H->d_xout;
+    k.act = H->d_act;
+    k.logits = H->d_logits;
+    k.argkey = H->d_argkey;
+    k.kv = H->d_kv;
+    k.hidden = c.hidden;
+    k.n_layers = L;
+    k.n_heads = c.n_heads;
+    k.n_kv_heads = nkv;
+    k.head_dim = hd;
+    k.ffn = c.ffn;
+    k.vocab = c.vocab;
+    k.max_ctx = c.max_ctx;
+    k.qkv_rows = P->qkv_rows;
+    k.group = P->group;
+    k.attn_splits = P->opt.attn_splits;
+    k.quant = q8 ? 1 : 0;
+    k.tied = c.tied_embeddings ? 1 : 0;
+    k.rms_eps = c.rms_eps;
+    k.rope_theta = c.rope_theta;
+    k.ring_stages = P->opt.ring_stages;
+    k.stage_bytes = P->opt.stage_bytes;
+    k.vec_floats = P->vec_floats;
+    k.att_lph = P->att_lph;
+    k.att_hpb = P->att_hpb;
+    k.att_e = P->att_e;
+    k.timeout_ns = (uint64_t)P->opt.wait_timeout_us * 1000ull;
+    k.skip_signal_task = P->opt.debug_skip_signal_task;
+    *out = H;
+    return AMK_OK;
+}
+
+extern "C" void amk_destroy(amk_handle *h) { free_handle(h); }
+
+extern "C" int amk_reset_kv(amk_handle *h)
+{
+    if (!h)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_reset_kv: NULL handle");
+    return zero_state(h);
+}
+
+namespace {
+
+// Non-blocking look at the error word copied after an earlier step.
+int poll_pending_error(amk_handle *H)
+{
+    if (!H->err_pending)
+        return AMK_OK;
+    if (cudaEventQuery(H->err_ev) != cudaSuccess) {
+        cudaGetLastError();  // clear cudaErrorNotReady
+        return AMK_OK;
+    }
+    H->err_pending = false;
+    return absorb_error(H, *H->h_err);
+}
+
+int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev)
+{
+    if (!H)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "NULL handle");
+    int rc = poll_pending_error(H);
+    if (rc != AMK_OK)
+        return rc;
+    if (H->poisoned)
+        return amk_set_error(AMK_ERR_POISONED, "handle poisoned; call amk_reset_kv");
+    const amk_config &c = H->plan->cfg;
+    if (pos < 0 || pos >= c.max_ctx)
+        return amk_set_error(AMK_ERR_POS_RANGE, "pos %d outside [0, %d)", pos, c.max_ctx);
+    if (token_id >= c.vocab || token_id < -1)
+        return amk_set_error(AMK_ERR_POS_RANGE, "token %d outside [0, %d)", token_id, c.vocab);
+    if (token_id == -1 && H->epoch == 0)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "token -1 needs a previous step");
+    if (logits_dev && ((uintptr_t)logits_dev % 4))
+        return amk_set_error(AMK_ERR_INVALID_ARG, "logits_dev misaligned");
+    KParams k = H->kp;
+    k.pos = pos;
+    k.token = token_id;
+    k.epoch = H->epoch;
+    k.parity = (int32_t)(H->epoch & 1u);
+    if (logits_dev)
+        k.logits = logits_dev;
+    cudaError_t e = amk::amk_kernel_launch(&k, H->plan->n_sms, H->plan->smem_bytes, H->stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return amk_set_error(e == cudaErrorCooperativeLaunchTooLarge ? AMK_ERR_LAUNCH
+                                                                      : AMK_ERR_CUDA,
+                             "cooperative launch: %s", cudaGetErrorString(e));
+    }
+    H->epoch += 1;
+    e = cudaMemcpyAsync(H->h_err, H->d_err, sizeof(ErrorWord), cudaMemcpyDeviceToHost,
+                        H->stream);
+    if (e == cudaSuccess)
+        e = cudaEventRecord(H->err_ev, H->stream);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "error word copy");
+    H->err_pending = true;
+    return AMK_OK;
+}
+
+int finish_sync(amk_handle *H, int32_t *argmax_host)
+{
+    const int parity = (int)((H->epoch - 1) & 1u);
+    cudaError_t e = cudaSuccess;
+    if (argmax_host)
+        e = cudaMemcpyAsync(H->h_key, H->d_argkey + parity, sizeof(unsigned long long),
+                            cudaMemcpyDeviceToHost, H->stream);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(H->stream);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "decode step");
+    H->err_pending = false;
+    int rc = absorb_error(H, *H->h_err);
+    if (rc != AMK_OK)
+        return rc;
+    if (argmax_host)
+        *argmax_host = (int32_t)(0xFFFFFFFFu - (uint32_t)(*H->h_key & 0xFFFFFFFFull));
+    return AMK_OK;
+}
+
+}  // namespace
+
+extern "C" int amk_decode_step(amk_handle *h, int32_t token_id, int32_t pos, float *logits_dev,
+                               int32_t *argmax_host)
+{
+    int rc = launch_step(h, token_id, pos, logits_dev);
+    if (rc != AMK_OK || !argmax_host)
+        return rc;
+    return finish_sync(h, argmax_host);
+}
+
+extern "C" int amk_decode_step_host(amk_handle *h, int32_t token_id, int32_t pos,
+                                    float *logits_host, int32_t *argmax_host)
+{
+    int rc = launch_step(h, token_id, pos, nullptr);
+    if (rc != AMK_OK)
+        return rc;
+    if (logits_host) {
+        cudaError_t e = cudaMemcpyAsync(logits_host, h->d_logits,
+                                        sizeof(float) * (size_t)h->plan->cfg.vocab,
+                                        cudaMemcpyDeviceToHost, h->stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "logits copy");
+    }
+    return finish_sync(h, argmax_host);
+}
+
+extern "C" int amk_get_kv(amk_handle *h, int32_t layer, void **k_dev, void **v_dev)
+{
+    if (!h || layer < 0 || layer >= h->plan->cfg.n_layers)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_get_kv: bad handle or layer");
+    const amk_config &c = h->plan->cfg;
+    const size_t blk = (size_t)c.n_kv_heads * c.max_ctx * c.head_dim;
+    if (k_dev)
+        *k_dev = h->d_kv + ((size_t)layer * 2 + 0) * blk;
+    if (v_dev)
+        *v_dev = h->d_kv + ((size_t)layer * 2 + 1) * blk;
+    return AMK_OK;
+}
+
+extern "C" int amk_get_logits(amk_handle *h, float **logits_dev)
+{
+    if (!h || !logits_dev)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_get_logits: NULL argument");
+    *logits_dev = h->d_logits;
+    return AMK_OK;
+}
+
+extern "C" int amk_get_stats(amk_handle *h, amk_plan_stats *o)
+{
+    if (!h || !o)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_get_stats: NULL argument");
+    const amk_plan *P = h->plan;
+    memset(o, 0, sizeof *o);
+    o->n_tasks = (int32_t)P->tasks.size();
+    o->n_counters = P->n_counters;
+    o->n_sms = P->n_sms;
+    o->ring_stages = P->opt.ring_stages;
+    o->stage_bytes = P->opt.stage_bytes;
+    o->attn_splits = P->opt.attn_splits;
+    o->smem_bytes = P->smem_bytes;
+    o->threads_per_cta = amk::kThreads;
+    o->weight_bytes = P->weight_bytes;
+    o->kv_row_bytes = P->kv_row_bytes;
+    o->epoch = h->epoch;
+    return AMK_OK;
+}
+
+extern "C" int amk_get_workspace(amk_handle *h, amk_workspace *out)
+{
+    if (!h || !out)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_get_workspace: NULL argument");
+    out->qkv = h->d_qkv;
+    out->xmid = h->d_xmid;
+    out->xout = h->d_xout;
+    out->act = h->d_act;
+    out->qkv_rows = h->plan->qkv_rows;
+    return AMK_OK;
+}
+
+extern "C" int amk_get_error_info(amk_handle *h, amk_error_info *out)
+{
+    if (!h || !out)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_get_error_info: NULL argument");
+    *out = h->last_err;
+    return AMK_OK;
+}

@@ -1,0 +1,106 @@
+// amk_internal.h -- structures shared by the host lowering/launcher and the
+// sm_100a megakernel.  Plain PODs: the host writes them once at create time
+// and the kernel reads them.
+#ifndef AMK_INTERNAL_H
+#define AMK_INTERNAL_H
+
+#include <stdint.h>
+
+#include "amk.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+// Records a thread-local error message and returns `code`.
+int amk_set_error(int code, const char *fmt, ...);
+#ifdef __cplusplus
+}
+#endif
+
+namespace amk {
+
+// Persistent CTA shape: 8 consumer warps (compute) + 1 producer warp (TMA).
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kThreads = kConsumerThreads + 32;
+constexpr int kMaxTaskRows = 256;   // output rows of one GEMV task (red buffer)
+constexpr int kMaxStages = 16;
+
+// Task kinds (the instruction set: GEMV row tiles with fused prologues and
+// epilogues, and the split-K attention tile).
+enum TaskKind : uint8_t {
+    TK_QKV = 1,     // rows of Wq|Wk|Wv (mat 0/1/2), RMSNorm prologue, raw q/k/v out
+    TK_ATTN = 2,    // (kv head g, split c): RoPE, KV append (c == 0), partial softmax
+    TK_OPROJ = 3,   // rows of Wo, split-K combine prologue, residual epilogue
+    TK_GATEUP = 4,  // rows of Wgate and Wup, RMSNorm prologue, SwiGLU epilogue
+    TK_DOWN = 5,    // rows of Wdown, residual epilogue
+    TK_LMHEAD = 6,  // rows of the LM head, final RMSNorm prologue, argmax epilogue
+};
+
+enum TaskFlags : uint8_t {
+    TF_RESET_ARGKEY = 1,  // this task clears the next step's argmax key
+};
+
+struct TaskDesc {           // 32 bytes
+    uint8_t kind, mat, flags, pad;
+    int32_t layer;
+    int32_t wait_ctr;       // -1: no wait
+    uint32_t wait_count;    // threshold t within one epoch
+    uint32_t wait_total;    // producers of wait_ctr (signals per epoch)
+    int32_t signal_ctr;     // -1: no signal
+    int32_t r0, r1;         // GEMV: output rows [r0, r1); ATTN: r0 = g, r1 = c
+};
+static_assert(sizeof(TaskDesc) == 32, "TaskDesc is 32 bytes");
+
+// Per-layer weight pointers (device copies of the caller's pointers).
+struct LayerPtrs {
+    const void *w[7];          // 0 q, 1 k, 2 v, 3 o, 4 gate, 5 up, 6 down
+    const uint16_t *s[7];      // fp16 row scales (W8A16) or null
+    const uint16_t *attn_norm, *ffn_norm;
+};
+enum { W_Q = 0, W_K, W_V, W_O, W_GATE, W_UP, W_DOWN };
+
+struct ErrorWord {
+    uint32_t code;      // 0 = ok, 1 = counter wait timeout, 2 = ring wait timeout
+    int32_t task, counter, sm;
+    uint32_t seen, target;
+    uint32_t pad[2];
+};
+
+struct KParams {
+    // schedule
+    const TaskDesc *tasks;     // grouped by SM, in queue order
+    const int32_t *queue_off;  // [n_sms + 1]
+    uint32_t *counters;
+    ErrorWord *err;
+    // weights
+    const LayerPtrs *layers;
+    const uint16_t *embed, *final_norm, *lm_head, *lm_head_scale;
+    // state and activations (fp32 unless noted)
+    float *qkv;       // [L][qkv_rows]: q | k | v, before RoPE
+    float *part;      // [L][nkv][C][G][hd + 2]: split-K partials (m, l, o[hd])
+    float *xmid;      // [L][h]: residual after attention
+    float *xout;      // [L][h]: residual after the FFN
+    float *act;       // [L][ffn]: SwiGLU activations
+    float *logits;    // [vocab]
+    unsigned long long *argkey;  // [2] packed (ordered logit << 32 | ~index)
+    uint16_t *kv;     // bf16 [L][2][nkv][max_ctx][hd]
+    // shapes
+    int32_t hidden, n_layers, n_heads, n_kv_heads, head_dim, ffn, vocab, max_ctx;
+    int32_t qkv_rows, group, attn_splits, quant, tied;
+    float rms_eps, rope_theta;
+    // ring
+    int32_t ring_stages, stage_bytes, vec_floats;
+    // attention lane layout
+    int32_t att_lph, att_hpb, att_e;  // lanes per head, heads per batch, elems per lane
+    // step
+    int32_t pos, token;         // token < 0: previous step's argmax
+    uint32_t epoch;             // steps since reset (counter targets)
+    int32_t parity;             // epoch & 1
+    uint64_t timeout_ns;
+    int32_t skip_signal_task;   // test hook, -1 = off
+};
+
+}  // namespace amk
+
+#endif

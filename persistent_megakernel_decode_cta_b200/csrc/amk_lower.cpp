@@ -1,0 +1,425 @@
+// amk_lower.cpp -- lowering a Llama-family decoder shape to the per-SM task
+// DAG of one decode step, plus the graph the static validator checks.
+//
+// paperfeed "RightNow-AI/AutoMegaKernel", "How it works", layer 2: model ->
+// graph IR -> tiled task DAG -> instruction stream; the schedule knobs are
+// tiling, SM assignment and pipelining depth ("RightNow-AI/AutoMegaKernel"
+// README, "Two autoresearch loops").  The lowering is deterministic: the same
+// shape and knobs always give the same DAG.
+//
+// Levels of one layer (each a set of independent tasks; a level waits for the
+// full count of the previous level's counter):
+//   QKV    row tiles of Wq, Wk, Wv; RMSNorm prologue
+//   ATTN   (KV head, position chunk) split-K tiles; RoPE, KV append, partials
+//   OPROJ  row tiles of Wo; split-K combine prologue, residual epilogue
+//   GATEUP row tiles of Wgate/Wup; RMSNorm prologue, SwiGLU epilogue
+//   DOWN   row tiles of Wdown; residual epilogue
+// then LMHEAD row tiles with a final-RMSNorm prologue and an argmax epilogue.
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <numeric>
+#include <vector>
+
+#include "amk.h"
+#include "amk_internal.h"
+#include "amk_plan.h"
+
+extern "C" int amk_kernel_smem_bytes(int ring_stages, int stage_bytes, int vec_floats);
+
+namespace {
+
+using amk::TaskDesc;
+
+constexpr int kMaxSmem = 232448;  // 227 KB opt-in shared memory per CTA on sm_100
+constexpr int kMaxK = amk::kConsumerThreads * 48;  // activations a lane keeps in registers
+
+int gran_rows(int64_t row_bytes)
+{
+    int g = 16;
+    while (row_bytes % g)
+        g >>= 1;
+    return 16 / g;  // rows whose bytes are a multiple of 16
+}
+
+// Split [0, rows) into about n tiles whose starts are multiples of gran.
+std::vector<std::pair<int, int>> tiles(int rows, int n, int gran)
+{
+    std::vector<std::pair<int, int>> out;
+    n = std::max(1, std::min(n, (rows + gran - 1) / gran));
+    int prev = 0;
+    for (int i = 1; i <= n; ++i) {
+        int b = (int)((int64_t)rows * i / n);
+        b -= b % gran;
+        if (i == n)
+            b = rows;
+        if (b > prev) {
+            out.push_back({prev, b});
+            prev = b;
+        }
+    }
+    return out;
+}
+
+struct Logical {
+    TaskDesc d;
+    int64_t cost;  // bytes streamed
+};
+
+}  // namespace
+
+int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_plan *P)
+{
+    amk_options opt;
+    amk_default_options(&opt);
+    if (opt_in) {
+        if (opt_in->ring_stages > 0) opt.ring_stages = opt_in->ring_stages;
+        if (opt_in->stage_bytes > 0) opt.stage_bytes = opt_in->stage_bytes;
+        if (opt_in->attn_splits > 0) opt.attn_splits = opt_in->attn_splits;
+        if (opt_in->tasks_per_sm > 0) opt.tasks_per_sm = opt_in->tasks_per_sm;
+        if (opt_in->wait_timeout_us > 0) opt.wait_timeout_us = opt_in->wait_timeout_us;
+        opt.debug_skip_signal_task = opt_in->debug_skip_signal_task;
+        opt.n_sms = opt_in->n_sms;
+    }
+    const amk_config &c = *cfg;
+    const int h = c.hidden, L = c.n_layers, nh = c.n_heads, nkv = c.n_kv_heads;
+    const int hd = c.head_dim, F = c.ffn, V = c.vocab;
+    if (h <= 0 || L <= 0 || nh <= 0 || nkv <= 0 || hd <= 0 || F <= 0 || V <= 0 ||
+        c.max_ctx <= 0 || n_sms <= 0)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "lowering: non-positive shape or SM count");
+    if (c.quant != AMK_QUANT_BF16 && c.quant != AMK_QUANT_W8A16)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "lowering: unknown quant mode %d", c.quant);
+    if (!(c.rms_eps >= 0.f) || !(c.rope_theta > 0.f))
+        return amk_set_error(AMK_ERR_INVALID_ARG, "lowering: bad rms_eps or rope_theta");
+    if (nh % nkv)
+        return amk_set_error(AMK_ERR_UNSUPPORTED, "n_heads %% n_kv_heads != 0");
+    if (hd % 8)
+        return amk_set_error(AMK_ERR_UNSUPPORTED, "head_dim must be a multiple of 8 "
+                             "(16-byte KV rows for bulk copies)");
+    if (opt.ring_stages < 2 || opt.ring_stages > amk::kMaxStages || opt.stage_bytes < 1024 ||
+        opt.stage_bytes % 1024)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "ring_stages in [2,%d], stage_bytes a "
+                             "multiple of 1024", amk::kMaxStages);
+    const int G = nh / nkv;
+    // attention lane layout: lph lanes per head, E elements per lane
+    int lph = 32;
+    while (lph > 1 && (lph * G > 32 || hd % lph))
+        lph >>= 1;
+    if (G > 32 || lph * G > 32 || hd % lph || hd / lph > 32)
+        return amk_set_error(AMK_ERR_UNSUPPORTED, "attention layout: group %d x head_dim %d "
+                             "does not fit one warp", G, hd);
+    const int esz = c.quant == AMK_QUANT_W8A16 ? 1 : 2;
+    const int head_esz = (c.tied_embeddings || c.quant != AMK_QUANT_W8A16) ? 2 : 1;
+    struct Mat { int rows, K, esz; const char *name; };
+    const Mat mats[] = {{nh * hd, h, esz, "wq"}, {nkv * hd, h, esz, "wk"},
+                        {nkv * hd, h, esz, "wv"}, {h, nh * hd, esz, "wo"},
+                        {F, h, esz, "wgate"},     {F, h, esz, "wup"},
+                        {h, F, esz, "wdown"},     {V, h, head_esz, "lm_head"}};
+    for (const Mat &m : mats) {
+        const int64_t rb = (int64_t)m.K * m.esz;
+        if (m.K > kMaxK)
+            return amk_set_error(AMK_ERR_UNSUPPORTED, "%s: inner dimension %d > %d", m.name,
+                                 m.K, kMaxK);
+        if (rb % 4)
+            return amk_set_error(AMK_ERR_UNSUPPORTED, "%s: row of %lld bytes is not a "
+                                 "multiple of 4", m.name, (long long)rb);
+        if (((int64_t)m.rows * rb) % 16)
+            return amk_set_error(AMK_ERR_UNSUPPORTED, "%s: %lld bytes is not a multiple of "
+                                 "16", m.name, (long long)(m.rows * rb));
+        if ((int64_t)gran_rows(rb) * rb > opt.stage_bytes)
+            return amk_set_error(AMK_ERR_UNSUPPORTED, "%s: a row of %lld bytes does not fit a "
+                                 "%d-byte ring stage", m.name, (long long)rb, opt.stage_bytes);
+    }
+    if (4 * hd > opt.stage_bytes)
+        return amk_set_error(AMK_ERR_UNSUPPORTED, "head_dim too large for the ring stage");
+
+    int C = opt.attn_splits;
+    if (C <= 0) {
+        const int by_sms = (n_sms + nkv - 1) / nkv;
+        const int by_combine = std::max(1, 65536 / (nh * (hd + 2) * 4));
+        C = std::max(1, std::min(by_sms, by_combine));
+    }
+    C = std::min(C, c.max_ctx);
+    int vec = std::max({h, F, nh * hd + nh * C,
+                        G * hd + 2 * hd + amk::kConsumerWarps * G * (hd + 2)});
+    vec = (vec + 3) & ~3;
+    int stages = opt.ring_stages;
+    while (stages > 2 && amk_kernel_smem_bytes(stages, opt.stage_bytes, vec) > kMaxSmem)
+        --stages;
+    const int smem = amk_kernel_smem_bytes(stages, opt.stage_bytes, vec);
+    if (smem > kMaxSmem)
+        return amk_set_error(AMK_ERR_UNSUPPORTED, "shared memory %d bytes > %d", smem, kMaxSmem);
+
+    P->cfg = c;
+    P->opt = opt;
+    P->opt.ring_stages = stages;
+    P->opt.attn_splits = C;
+    P->n_sms = n_sms;
+    P->group = G;
+    P->qkv_rows = nh * hd + 2 * nkv * hd;
+    P->vec_floats = vec;
+    P->smem_bytes = smem;
+    P->att_lph = lph;
+    P->att_hpb = 32 / lph;
+    P->att_e = hd / lph;
+
+    // ---- logical tasks per level ---------------------------------------------
+    enum { LV_QKV, LV_ATTN, LV_OPROJ, LV_GATEUP, LV_DOWN, LV_N };
+    auto ctr_of = [&](int layer, int lv) { return layer * LV_N + lv; };
+    const int n_ctr = L * LV_N;
+    std::vector<std::vector<Logical>> levels;
+    auto mk = [](uint8_t kind, int layer, int r0, int r1, uint8_t mat = 0) {
+        TaskDesc d{};
+        d.kind = kind;
+        d.mat = mat;
+        d.layer = layer;
+        d.wait_ctr = -1;
+        d.signal_ctr = -1;
+        d.r0 = r0;
+        d.r1 = r1;
+        return d;
+    };
+    const int tps = std::max(1, opt.tasks_per_sm);
+    auto gemv_level = [&](uint8_t kind, int layer, int rows, int K, int e, int target,
+                          int max_rows, uint8_t mat, std::vector<Logical> &out) {
+        const int64_t rb = (int64_t)K * e;
+        int n = std::max(target, (rows + max_rows - 1) / max_rows);
+        std::vector<std::pair<int, int>> tl;
+        for (;; ++n) {  // granule rounding may grow a tile past max_rows
+            tl = tiles(rows, n, gran_rows(rb));
+            bool fits = true;
+            for (auto t : tl)
+                fits &= t.second - t.first <= max_rows;
+            if (fits)
+                break;
+        }
+        for (auto t : tl)
+            out.push_back({mk(kind, layer, t.first, t.second, mat),
+                           (int64_t)(t.second - t.first) * rb});
+    };
+    for (int l = 0; l < L; ++l) {
+        // QKV: tiles shared among the three matrices in proportion to rows
+        std::vector<Logical> qkv;
+        const int rows3[3] = {nh * hd, nkv * hd, nkv * hd};
+        const int total = P->qkv_rows;
+        const int target = n_sms * tps;
+        int given = 0;
+        for (int m = 0; m < 3; ++m) {
+            int nt = m < 2 ? std::max(1, (int)((int64_t)target * rows3[m] / total))
+                           : std::max(1, target - given);
+            given += nt;
+            gemv_level(amk::TK_QKV, l, rows3[m], h, esz, nt, amk::kMaxTaskRows, (uint8_t)m, qkv);
+        }
+        levels.push_back(std::move(qkv));
+        std::vector<Logical> att;
+        for (int g = 0; g < nkv; ++g)
+            for (int ci = 0; ci < C; ++ci)
+                att.push_back({mk(amk::TK_ATTN, l, g, ci), 0});
+        levels.push_back(std::move(att));
+        std::vector<Logical> o, gu, dn;
+        gemv_level(amk::TK_OPROJ, l, h, nh * hd, esz, target, amk::kMaxTaskRows, 0, o);
+        levels.push_back(std::move(o));
+        gemv_level(amk::TK_GATEUP, l, F, h, esz, target, amk::kMaxTaskRows / 2, 0, gu);
+        for (auto &t : gu)
+            t.cost *= 2;
+        levels.push_back(std::move(gu));
+        gemv_level(amk::TK_DOWN, l, h, F, esz, target, amk::kMaxTaskRows, 0, dn);
+        levels.push_back(std::move(dn));
+    }
+    {
+        std::vector<Logical> lm;
+        gemv_level(amk::TK_LMHEAD, L - 1, V, h, head_esz, n_sms * tps, amk::kMaxTaskRows, 0, lm);
+        lm[0].d.flags |= amk::TF_RESET_ARGKEY;
+        levels.push_back(std::move(lm));
+    }
+    // waits / signals: level i of layer l signals ctr(l, i); waits on the
+    // previous level's counter at full count (QKV of layer l > 0 waits on
+    // DOWN of layer l-1; LMHEAD waits on DOWN of the last layer)
+    std::vector<uint32_t> total(n_ctr, 0);
+    for (size_t li = 0; li + 1 < levels.size(); ++li) {
+        const int layer = (int)li / LV_N, lv = (int)li % LV_N;
+        for (auto &t : levels[li])
+            t.d.signal_ctr = ctr_of(layer, lv);
+        total[ctr_of(layer, lv)] = (uint32_t)levels[li].size();
+    }
+    for (size_t li = 1; li < levels.size(); ++li) {
+        const int prev = (int)li - 1;
+        const int pc = ctr_of(prev / LV_N, prev % LV_N);
+        for (auto &t : levels[li]) {
+            t.d.wait_ctr = pc;
+            t.d.wait_count = total[pc];
+            t.d.wait_total = total[pc];
+        }
+    }
+
+    // ---- SM assignment: per level, heaviest task to the least-loaded SM --------
+    std::vector<std::vector<TaskDesc>> queues(n_sms);
+    std::vector<int64_t> cum(n_sms, 0);
+    for (auto &lv : levels) {
+        std::vector<int> idx(lv.size());
+        std::iota(idx.begin(), idx.end(), 0);
+        std::stable_sort(idx.begin(), idx.end(),
+                         [&](int a, int b) { return lv[a].cost > lv[b].cost; });
+        std::vector<int64_t> load(n_sms, 0);
+        std::vector<std::vector<int>> mine(n_sms);
+        for (int i : idx) {
+            int best = 0;
+            for (int s = 1; s < n_sms; ++s)
+                if (load[s] < load[best] || (load[s] == load[best] && cum[s] < cum[best]))
+                    best = s;
+            load[best] += std::max<int64_t>(lv[i].cost, 1);
+            cum[best] += lv[i].cost;
+            mine[best].push_back(i);
+        }
+        for (int s = 0; s < n_sms; ++s) {
+            std::sort(mine[s].begin(), mine[s].end());
+            for (int i : mine[s])
+                queues[s].push_back(lv[i].d);
+        }
+    }
+    P->tasks.clear();
+    P->queue_off.assign(n_sms + 1, 0);
+    for (int s = 0; s < n_sms; ++s) {
+        P->queue_off[s] = (int32_t)P->tasks.size();
+        for (auto &d : queues[s])
+            P->tasks.push_back(d);
+    }
+    P->queue_off[n_sms] = (int32_t)P->tasks.size();
+    P->n_counters = n_ctr;
+
+    // ---- the validator's graph ----------------------------------------------
+    const int T = (int)P->tasks.size();
+    auto B_QKV = [](int l) { return 6 * l + 0; };
+    auto B_PART = [](int l) { return 6 * l + 1; };
+    auto B_XMID = [](int l) { return 6 * l + 2; };
+    auto B_XOUT = [](int l) { return 6 * l + 3; };
+    auto B_ACT = [](int l) { return 6 * l + 4; };
+    auto B_KVNEW = [](int l) { return 6 * l + 5; };
+    const int B_LOGITS = 6 * L, B_KEY = 6 * L + 1, B_KEYNEXT = 6 * L + 2;
+    P->gbufs.assign(6 * L + 3, amk_graph_buffer{0, 0, -1});
+    const int64_t part_sz = (int64_t)nkv * C * G * (hd + 2);
+    for (int l = 0; l < L; ++l) {
+        P->gbufs[B_QKV(l)].size = P->qkv_rows;
+        P->gbufs[B_PART(l)].size = part_sz;
+        P->gbufs[B_XMID(l)].size = h;
+        P->gbufs[B_XOUT(l)].size = h;
+        P->gbufs[B_ACT(l)].size = F;
+        P->gbufs[B_KVNEW(l)].size = (int64_t)nkv * 2 * hd;
+    }
+    P->gbufs[B_LOGITS] = {V, AMK_BUF_OUTPUT, -1};
+    P->gbufs[B_KEY] = {1, AMK_BUF_OUTPUT, B_KEYNEXT};
+    P->gbufs[B_KEYNEXT] = {1, 0, -1};
+    P->gtasks.assign(T, amk_graph_task{});
+    P->gwaits.clear();
+    P->gsignals.clear();
+    P->gacc.clear();
+    P->kind.assign(T, 0);
+    P->layer.assign(T, 0);
+    auto acc = [&](int buf, int kind, int64_t b, int64_t e) {
+        P->gacc.push_back(amk_graph_access{buf, kind, b, e});
+    };
+    for (int s = 0; s < n_sms; ++s) {
+        for (int t = P->queue_off[s]; t < P->queue_off[s + 1]; ++t) {
+            const TaskDesc &d = P->tasks[t];
+            amk_graph_task &gt = P->gtasks[t];
+            gt.sm = s;
+            gt.wait_begin = (int32_t)P->gwaits.size();
+            if (d.wait_ctr >= 0)
+                P->gwaits.push_back({d.wait_ctr, (int32_t)d.wait_count});
+            gt.wait_count = (int32_t)P->gwaits.size() - gt.wait_begin;
+            gt.signal_begin = (int32_t)P->gsignals.size();
+            if (d.signal_ctr >= 0)
+                P->gsignals.push_back(d.signal_ctr);
+            gt.signal_count = (int32_t)P->gsignals.size() - gt.signal_begin;
+            gt.access_begin = (int32_t)P->gacc.size();
+            const int l = d.layer;
+            // what the kernel's task of this kind reads and writes
+            switch (d.kind) {
+            case amk::TK_QKV: {
+                const int off = d.mat == 0 ? 0 : d.mat == 1 ? nh * hd : (nh + nkv) * hd;
+                if (l > 0)
+                    acc(B_XOUT(l - 1), AMK_ACC_READ, 0, h);
+                else
+                    acc(B_KEYNEXT, AMK_ACC_READ_PREV, 0, 1);
+                acc(B_QKV(l), AMK_ACC_WRITE, off + d.r0, off + d.r1);
+                break;
+            }
+            case amk::TK_ATTN: {
+                const int g = d.r0, ci = d.r1;
+                acc(B_QKV(l), AMK_ACC_READ, (int64_t)g * G * hd, (int64_t)(g + 1) * G * hd);
+                acc(B_QKV(l), AMK_ACC_READ, (int64_t)nh * hd + g * hd,
+                    (int64_t)nh * hd + (g + 1) * hd);
+                acc(B_QKV(l), AMK_ACC_READ, (int64_t)(nh + nkv) * hd + g * hd,
+                    (int64_t)(nh + nkv) * hd + (g + 1) * hd);
+                const int64_t slot = ((int64_t)g * C + ci) * G * (hd + 2);
+                acc(B_PART(l), AMK_ACC_WRITE, slot, slot + (int64_t)G * (hd + 2));
+                if (ci == 0)
+                    acc(B_KVNEW(l), AMK_ACC_WRITE, (int64_t)g * 2 * hd, (int64_t)(g + 1) * 2 * hd);
+                break;
+            }
+            case amk::TK_OPROJ:
+                acc(B_PART(l), AMK_ACC_READ, 0, part_sz);
+                if (l > 0)
+                    acc(B_XOUT(l - 1), AMK_ACC_READ, d.r0, d.r1);
+                else
+                    acc(B_KEYNEXT, AMK_ACC_READ_PREV, 0, 1);
+                acc(B_XMID(l), AMK_ACC_WRITE, d.r0, d.r1);
+                break;
+            case amk::TK_GATEUP:
+                acc(B_XMID(l), AMK_ACC_READ, 0, h);
+                acc(B_ACT(l), AMK_ACC_WRITE, d.r0, d.r1);
+                break;
+            case amk::TK_DOWN:
+                acc(B_ACT(l), AMK_ACC_READ, 0, F);
+                acc(B_XMID(l), AMK_ACC_READ, d.r0, d.r1);
+                acc(B_XOUT(l), AMK_ACC_WRITE, d.r0, d.r1);
+                break;
+            case amk::TK_LMHEAD:
+                acc(B_XOUT(L - 1), AMK_ACC_READ, 0, h);
+                acc(B_LOGITS, AMK_ACC_WRITE, d.r0, d.r1);
+                acc(B_KEY, AMK_ACC_ACCUM, 0, 1);
+                if (d.flags & amk::TF_RESET_ARGKEY)
+                    acc(B_KEYNEXT, AMK_ACC_RESET, 0, 1);
+                break;
+            }
+            gt.access_count = (int32_t)P->gacc.size() - gt.access_begin;
+            P->kind[t] = d.kind;
+            P->layer[t] = d.layer;
+        }
+    }
+    P->gqueue.resize(T);
+    std::iota(P->gqueue.begin(), P->gqueue.end(), 0);
+
+    // ---- bytes streamed per step -------------------------------------------
+    int64_t wb = 0;
+    for (const Mat &m : mats) {
+        const int64_t bytes = (int64_t)m.rows * m.K * m.esz;
+        const bool is_head = !strcmp(m.name, "lm_head");
+        wb += is_head ? bytes : bytes * L;
+        if (m.esz == 1)
+            wb += (int64_t)m.rows * 2 * (is_head ? 1 : L);
+    }
+    wb += (int64_t)(2 * L + 1) * h * 2 + (int64_t)h * 2;  // norm gains + embedding row
+    P->weight_bytes = wb;
+    P->kv_row_bytes = (int64_t)L * 2 * nkv * hd * 2;
+    return AMK_OK;
+}
+
+void amk_plan_view(const amk_plan *P, amk_graph *g)
+{
+    memset(g, 0, sizeof *g);
+    g->n_tasks = (int32_t)P->tasks.size();
+    g->n_counters = P->n_counters;
+    g->n_buffers = (int32_t)P->gbufs.size();
+    g->n_sms = P->n_sms;
+    g->n_waits = (int32_t)P->gwaits.size();
+    g->n_signals = (int32_t)P->gsignals.size();
+    g->n_accesses = (int32_t)P->gacc.size();
+    g->tasks = P->gtasks.data();
+    g->waits = P->gwaits.data();
+    g->signals = P->gsignals.data();
+    g->accesses = P->gacc.data();
+    g->buffers = P->gbufs.data();
+    g->queue_offsets = P->queue_off.data();
+    g->queue_tasks = P->gqueue.data();
+}

@@ -1,0 +1,36 @@
+// amk_plan.h -- the lowered schedule of one decode step (host side).
+#ifndef AMK_PLAN_H
+#define AMK_PLAN_H
+
+#include <cstdint>
+#include <vector>
+
+#include "amk.h"
+#include "amk_internal.h"
+
+struct amk_plan {
+    amk_config cfg;
+    amk_options opt;       // effective knobs (ring_stages, attn_splits resolved)
+    int n_sms = 0;
+    int group = 0, qkv_rows = 0, vec_floats = 0, smem_bytes = 0;
+    int att_lph = 0, att_hpb = 0, att_e = 0;
+    std::vector<amk::TaskDesc> tasks;  // grouped by SM, queue order
+    std::vector<int32_t> queue_off;    // [n_sms + 1]
+    int n_counters = 0;
+    // the validator's view
+    std::vector<amk_graph_task> gtasks;
+    std::vector<amk_graph_wait> gwaits;
+    std::vector<int32_t> gsignals;
+    std::vector<amk_graph_access> gacc;
+    std::vector<amk_graph_buffer> gbufs;
+    std::vector<int32_t> gqueue;
+    std::vector<int32_t> kind, layer;
+    int64_t weight_bytes = 0, kv_row_bytes = 0;
+};
+
+// Lowers cfg for n_sms persistent CTAs into *P (no validation).
+int amk_lower(const amk_config *cfg, const amk_options *opt, int n_sms, amk_plan *P);
+// A non-owning amk_graph view of P's graph arrays.
+void amk_plan_view(const amk_plan *P, amk_graph *g);
+
+#endif

@@ -1,0 +1,86 @@
+"""Shared helpers for the GPU parity tests: build the same seeded model for the
+CUDA path and the fp64 oracle, and compare them.
+
+Tolerances are the ones the workload states for this path: max |logit
+difference| <= 1e-2 * max |logit| for bf16 weights and 2e-2 * max |logit| for
+W8A16; greedy tokens must match wherever the oracle's top-2 margin exceeds
+that bound (elsewhere both candidates are correct).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as orc
+import persistent_megakernel_decode_cta_b200 as amk
+import synth_inputs as si
+
+
+def tol_frac(cfg) -> float:
+    return 2e-2 if cfg.quant == "w8a16" else 1e-2
+
+
+class Pair:
+    """A Decoder and an OracleModel over identical weight bytes."""
+
+    def __init__(self, cfg, seed=0, options=None, weights=None):
+        self.cfg = cfg
+        self.w = weights if weights is not None else si.make_model(cfg, seed=seed, device="cuda")
+        torch.cuda.synchronize()
+        self.dec = amk.Decoder(cfg, self.w, options)
+        self.orc = orc.OracleModel(cfg, self.w)
+        self.logits = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+
+    def fill_kv(self, ctx: int, seed: int = 2):
+        kv = si.make_kv_fill(self.cfg, ctx, seed=seed, device="cuda")
+        for l in range(self.cfg.n_layers):
+            k, v = self.dec.kv(l)
+            k[:, :ctx, :].copy_(kv[l, 0])
+            v[:, :ctx, :].copy_(kv[l, 1])
+        torch.cuda.synchronize()
+        self.orc.fill_kv(kv)
+
+    def step(self, token: int, pos: int):
+        """Runs both sides; returns (gpu logits, gpu argmax, oracle logits,
+        oracle argmax)."""
+        am = self.dec.step(token, pos, logits=self.logits)
+        g = self.logits.double().cpu().numpy()
+        ref, ref_am, _ = self.orc.step(token, pos)
+        return g, am, ref, ref_am
+
+
+def compare(cfg, g, am, ref, ref_am, what=""):
+    """Asserts the parity bound; returns (max abs diff / max |logit|, margin ok)."""
+    assert np.isfinite(g).all(), f"{what}: non-finite GPU logits"
+    scale = np.abs(ref).max()
+    err = np.abs(g - ref).max()
+    tol = tol_frac(cfg) * scale
+    assert err <= tol, f"{what}: max|dlogit| {err:.4g} > {tol:.4g} (max|logit| {scale:.4g})"
+    top2 = np.sort(ref)[-2:]
+    margin = top2[1] - top2[0]
+    if margin > tol:
+        assert am == ref_am, f"{what}: token {am} != oracle {ref_am} (margin {margin:.4g})"
+    else:
+        # several answers are correct; the GPU's must be one of the near-ties
+        assert ref[am] >= ref.max() - tol, f"{what}: token {am} not within tolerance of max"
+    return err / scale, margin > tol
+
+
+def greedy_teacher_forced(pair: Pair, prompt, n_new: int, start_pos: int = 0):
+    """Feeds the prompt, then n_new greedy steps; the oracle's token is fed to
+    both sides so the sequences stay aligned.  Returns the worst relative
+    error and the number of exact-token checks."""
+    cfg = pair.cfg
+    worst, checked = 0.0, 0
+    pos = start_pos
+    tok = None
+    for i, t in enumerate(list(prompt) + [None] * n_new):
+        if t is None:
+            t = tok
+        g, am, ref, ref_am = pair.step(t, pos)
+        e, exact = compare(cfg, g, am, ref, ref_am, what=f"pos {pos}")
+        worst = max(worst, e)
+        checked += exact
+        tok = ref_am
+        pos += 1
+    return worst, checked

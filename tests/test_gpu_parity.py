@@ -1,0 +1,152 @@
+"""GPU parity: the megakernel (called through the C ABI) against the fp64
+oracle on identical seeded weights, element by element on the logits, and
+on greedy tokens wherever the oracle's top-2 margin exceeds the bound.
+
+Workloads: the tiny decoder (8 greedy steps from a 4-token prompt) and
+random-init models shaped like SmolLM2-135M, TinyLlama-1.1B, Llama-1B
+(W8A16) and Llama-7B (bf16 and W8A16), at KV context 0 and the long contexts
+of those workloads (long caches filled with seeded N(0,1) bf16 rows).
+"""
+import numpy as np
+import pytest
+import torch
+
+import persistent_megakernel_decode_cta_b200 as amk
+from persistent_megakernel_decode_cta_b200 import build
+import synth_inputs as si
+from parity_helpers import Pair, compare, greedy_teacher_forced
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built(cuda_ok):
+    build.build()
+
+
+@pytest.mark.parametrize("variant", ["bf16", "tied", "w8a16"])
+@pytest.mark.parametrize("n_sms", [0, 3])
+def test_tiny_greedy(variant, n_sms):
+    cfg = si.get_config("tiny")
+    if variant == "tied":
+        cfg = cfg.with_(tied=True, name="tiny_tied")
+    elif variant == "w8a16":
+        cfg = cfg.with_(quant="w8a16", name="tiny_w8")
+    opts = amk.default_options(n_sms=n_sms) if n_sms else None
+    pair = Pair(cfg, options=opts)
+    prompt = si.make_prompt(cfg, 4)
+    worst, checked = greedy_teacher_forced(pair, prompt, 8)
+    assert checked >= 6
+    # the KV rows the kernel appended equal the oracle's (bf16 of nearly equal
+    # fp32/fp64 values: within one bf16 ulp)
+    for l in range(cfg.n_layers):
+        k, v = pair.dec.kv(l)
+        gk = k[:, :12].float().cpu().numpy()
+        from oracle.brute import bf16_bits_to_f64
+        rk = bf16_bits_to_f64(pair.orc.kv[l, 0, :, :12])
+        assert np.allclose(gk, rk, rtol=2 ** -7, atol=1e-6)
+
+
+def test_tiny_device_token_chaining():
+    """token_id = -1 feeds the previous step's device argmax (no host copy):
+    the chained run must give exactly the tokens of a run whose tokens are
+    read back and fed from the host (the kernel is deterministic)."""
+    cfg = si.get_config("tiny")
+    pair = Pair(cfg)
+    prompt = si.make_prompt(cfg, 4)
+    explicit = []
+    tok = None
+    for pos in range(12):
+        tok = pair.dec.step(prompt[pos] if pos < 4 else tok, pos)
+        if pos >= 3:
+            explicit.append(tok)
+    pair.dec.reset()
+    for pos in range(4):
+        first = pair.dec.step(prompt[pos], pos)
+    chained = [first]
+    for pos in range(4, 12):
+        if pos < 11:
+            pair.dec.step(-1, pos, want_argmax=False)
+        else:
+            chained.append(pair.dec.step(-1, pos))
+    assert chained == [explicit[0], explicit[-1]]
+
+
+def test_host_path_matches_device_path():
+    cfg = si.get_config("tiny")
+    pair = Pair(cfg)
+    host = np.zeros(cfg.vocab, dtype=np.float32)
+    a = pair.dec.step_host(5, 0, host)
+    pair.dec.reset()
+    b = pair.dec.step(5, 0, logits=pair.logits)
+    assert a == b
+    assert np.array_equal(host, pair.logits.cpu().numpy())
+
+
+@pytest.mark.parametrize("name,ctxs", [
+    ("smol135", [0, 128]),
+    ("tinyllama", [0, 256, 1024]),
+    ("llama1b_w8", [0, 512]),
+    ("llama7b", [0, 2048]),
+    ("llama7b_w8", [0, 2048]),
+])
+def test_full_size_single_steps(name, ctxs):
+    cfg = si.get_config(name)
+    pair = Pair(cfg)
+    for ctx in ctxs:
+        pair.dec.reset()
+        pair.orc.reset()
+        if ctx:
+            pair.fill_kv(ctx)
+        tok = si.make_prompt(cfg, 1, seed=10 + ctx)[0]
+        g, am, ref, ref_am = pair.step(tok, ctx)
+        compare(cfg, g, am, ref, ref_am, what=f"{name} ctx {ctx}")
+    del pair
+    torch.cuda.empty_cache()
+
+
+def test_smol_greedy_32_steps():
+    cfg = si.get_config("smol135")
+    pair = Pair(cfg)
+    worst, checked = greedy_teacher_forced(pair, si.make_prompt(cfg, 1), 31)
+    assert checked >= 16
+
+
+def test_bad_arguments():
+    cfg = si.get_config("tiny")
+    pair = Pair(cfg)
+    with pytest.raises(amk.AmkError) as e:
+        pair.dec.step(0, cfg.max_ctx)
+    assert e.value.name == "AMK_ERR_POS_RANGE"
+    with pytest.raises(amk.AmkError) as e:
+        pair.dec.step(cfg.vocab, 0)
+    assert e.value.name == "AMK_ERR_POS_RANGE"
+    with pytest.raises(amk.AmkError) as e:
+        pair.dec.step(-1, 0)
+    assert e.value.name == "AMK_ERR_INVALID_ARG"
+
+
+def test_wait_timeout_is_reported_and_recoverable():
+    """Fault injection on the host: one task never signals its counter, so a
+    downstream wait runs out after its (short) limit; the kernel returns, the
+    call reports AMK_ERR_TIMEOUT, the handle is poisoned until reset, and after
+    a reset a normal handle decodes correctly again."""
+    cfg = si.get_config("tiny")
+    plan = amk.Plan(cfg, 4)
+    kinds, _ = plan.task_info()
+    victim = kinds.index(1)  # a QKV task
+    opts = amk.default_options(n_sms=4, wait_timeout_us=20000, debug_skip_signal_task=victim)
+    pair = Pair(cfg, options=opts)
+    with pytest.raises(amk.AmkError) as e:
+        pair.dec.step(3, 0)
+    assert e.value.name == "AMK_ERR_TIMEOUT"
+    info = pair.dec.error_info()
+    assert info.code == 1 and info.counter >= 0
+    with pytest.raises(amk.AmkError) as e:
+        pair.dec.step(3, 0)
+    assert e.value.name == "AMK_ERR_POISONED"
+    pair.dec.reset()
+    # the device context is still usable: a fresh handle on the same weights works
+    good = Pair(cfg, weights=pair.w, options=amk.default_options(n_sms=4))
+    g, am, ref, ref_am = good.step(3, 0)
+    compare(cfg, g, am, ref, ref_am, "after timeout")

@@ -1,0 +1,104 @@
+"""Host lowering: every workload lowers to a schedule the validator accepts,
+its tiles cover each weight matrix exactly once, and a small real lowering
+also passes the brute-force interleaving checker.
+
+paperfeed "RightNow-AI/AutoMegaKernel", "How it works": model -> tiled task
+DAG; x-techcon AutoMegaKernel article, section 1: all real lowerings accepted.
+"""
+import pytest
+
+import persistent_megakernel_decode_cta_b200 as amk
+from persistent_megakernel_decode_cta_b200 import abi, build
+import synth_inputs as si
+from oracle import interleave as bf
+
+KIND = {1: "QKV", 2: "ATTN", 3: "OPROJ", 4: "GATEUP", 5: "DOWN", 6: "LMHEAD"}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+
+
+def _writes(g, buf):
+    out = []
+    for t, task in enumerate(g["tasks"]):
+        for (b, k, lo, hi) in task["accesses"]:
+            if b == buf and k == abi.ACC_WRITE:
+                out.append((lo, hi, t))
+    return sorted(out)
+
+
+def _partition(ranges, size):
+    pos = 0
+    for lo, hi, _ in ranges:
+        assert lo == pos, (lo, pos)
+        pos = hi
+    assert pos == size
+
+
+@pytest.mark.parametrize("name", list(si.CONFIGS))
+@pytest.mark.parametrize("n_sms", [148, 7])
+def test_real_lowerings_accepted_and_cover(name, n_sms):
+    cfg = si.get_config(name)
+    plan = amk.Plan(cfg, n_sms)
+    g = plan.graph()
+    kinds, layers = plan.task_info()
+    L, h, F = cfg.n_layers, cfg.hidden, cfg.ffn
+    # buffers: 6 per layer (qkv, part, xmid, xout, act, kvnew) + logits, key, key_next
+    assert len(g["buffers"]) == 6 * L + 3
+    for l in range(L):
+        _partition(_writes(g, 6 * l + 0), cfg.q_rows + 2 * cfg.kv_rows)   # QKV rows
+        _partition(_writes(g, 6 * l + 2), h)                               # O rows
+        _partition(_writes(g, 6 * l + 3), h)                               # down rows
+        _partition(_writes(g, 6 * l + 4), F)                               # gate/up rows
+    _partition(_writes(g, 6 * L), cfg.vocab)                               # LM head rows
+    # every SM runs its tasks level by level
+    for q in g["queues"]:
+        seq = [(layers[t], ["QKV", "ATTN", "OPROJ", "GATEUP", "DOWN", "LMHEAD"].index(
+            KIND[kinds[t]])) for t in q]
+        assert seq == sorted(seq)
+    n_att = sum(1 for k in kinds if KIND[k] == "ATTN")
+    assert n_att % (L * cfg.n_kv_heads) == 0
+    # the library's validator accepts the plan (it ran inside amk_plan_create
+    # too); run it again on the exported graph
+    ok, rule, msg = amk.validate_graph(g)
+    assert ok, (rule, msg)
+
+
+def test_small_real_lowering_passes_brute_force():
+    cfg = si.get_config("tiny").with_(n_layers=1, name="tiny1")
+    opts = amk.default_options(attn_splits=1)
+    g = amk.Plan(cfg, 2, opts).graph()
+    assert len(g["tasks"]) <= 14
+    assert bf.check(g) == (True, "ok")
+
+
+def test_balanced_tiles_on_148_sms():
+    cfg = si.get_config("tinyllama")
+    plan = amk.Plan(cfg, 148)
+    g = plan.graph()
+    kinds, layers = plan.task_info()
+    per_sm_gateup = [sum(1 for t in q if kinds[t] == 4 and layers[t] == 0) for q in g["queues"]]
+    assert max(per_sm_gateup) == 1 and min(per_sm_gateup) == 1
+
+
+@pytest.mark.parametrize("edit,status", [
+    (dict(head_dim=12), "AMK_ERR_UNSUPPORTED"),          # KV rows not 16-byte multiples
+    (dict(n_kv_heads=3), "AMK_ERR_UNSUPPORTED"),         # 4 heads not divisible by 3
+    (dict(ffn=12290), "AMK_ERR_UNSUPPORTED"),            # down K above the register slice
+    (dict(hidden=0), "AMK_ERR_INVALID_ARG"),
+    (dict(ffn=171), "AMK_ERR_UNSUPPORTED"),              # odd bf16 K: row not 4-byte aligned
+])
+def test_unsupported_shapes_rejected(edit, status):
+    cfg = si.get_config("tiny").with_(**edit)
+    with pytest.raises(amk.AmkError) as e:
+        amk.Plan(cfg, 4)
+    assert e.value.name == status
+
+
+def test_bad_options_rejected():
+    cfg = si.get_config("tiny")
+    with pytest.raises(amk.AmkError) as e:
+        amk.Plan(cfg, 4, amk.default_options(stage_bytes=1000))
+    assert e.value.name == "AMK_ERR_INVALID_ARG"
