@@ -1,0 +1,412 @@
+"""Batch-1 decode benchmark: µs/token and achieved HBM GB/s of the persistent
+decode megakernel on B200, next to the fp64 CPU oracle.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl ours|reference]
+
+One "step" = one decode step of the whole forward pass (one cooperative
+launch), greedy, token chained on the device.  The default workload is the
+Llama-7B-shaped bf16 decoder decoding at KV context 2048 (13.2 GB of weights
++ 1.07 GB of KV read per token: larger than L2, so no flush is needed).
+Every step decodes at position = context (the row is rewritten each step).
+
+The timing is printed only beside a PASS parity verdict from the same run
+(the first step's logits against the oracle), after the honesty rule of
+"RightNow-AI/AutoMegaKernel" README, "Honesty rules": no latency without a
+paired correctness verdict.
+
+Multi-GPU: batch-1 decode does not shard; N GPUs run N independent replicas
+(one rank per GPU, no data-path collective).  value = whole-job time per
+token = max-over-ranks elapsed / (N * K).
+
+--impl reference times the fp64 oracle (the only reference implementation
+this path has) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth_inputs as si  # noqa: E402
+
+METRIC = "batch-1 decode us/token"
+UNIT = "us/token"
+
+# name -> (model config, KV context)
+WORKLOADS = {
+    "llama7b-ctx2048": ("llama7b", 2048),
+    "llama7b-ctx0": ("llama7b", 0),
+    "llama7b_w8-ctx2048": ("llama7b_w8", 2048),
+    "llama7b_w8-ctx0": ("llama7b_w8", 0),
+    "tinyllama-ctx0": ("tinyllama", 0),
+    "tinyllama-ctx1024": ("tinyllama", 1024),
+    "llama1b_w8-ctx0": ("llama1b_w8", 0),
+    "llama1b_w8-ctx512": ("llama1b_w8", 512),
+    "smol135-ctx0": ("smol135", 0),
+    "smol135-ctx128": ("smol135", 128),
+    "tiny-ctx4": ("tiny", 4),
+}
+DEFAULT_WORKLOAD = "llama7b-ctx2048"
+KERNEL_SOURCES = ["persistent_megakernel_decode_cta_b200/csrc/amk_kernel.cu",
+                  "persistent_megakernel_decode_cta_b200/csrc/amk_internal.h"]
+
+
+def algorithmic_bytes(cfg, ctx: int) -> int:
+    """Bytes one decode step must move: every weight byte once (int8 scales,
+    norm gains and one embedding row included), the KV rows 0..ctx-1 of every
+    layer, the new K/V row, and the logits."""
+    b = si.model_bytes(cfg)
+    kv_row = 2 * cfg.n_layers * cfg.n_kv_heads * cfg.head_dim * 2
+    return (b["linear"] + b["scales"] + b["head"] + b["norms"] + b["embed_row"]
+            + kv_row * ctx + kv_row + cfg.vocab * 4)
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(workload: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
+    on this workload with the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(path))
+    except (OSError, ValueError):
+        return None
+    e = d.get(workload)
+    if not e or e.get("kernel_hash") != kernel_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def measured_peak():
+    try:
+        d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            try:
+                gid = "GPU-" + str(torch.cuda.get_device_properties(self.gpu).uuid)
+            except Exception:
+                gid = str(self.gpu)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gid}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        rows = []
+        for ln in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5], f[6], f[7], f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            for n, v in zip(names, r[2:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value: float) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_steps(cfg, weights, ctx, kv_fill, budget_s: float, max_steps: int):
+    """Times full fp64 oracle decode steps at position ctx (as many as fit the
+    budget, at least one).  Returns (us per token, steps, threads, logits of
+    the first step)."""
+    import oracle
+    m = oracle.OracleModel(cfg, weights)
+    threads = oracle.set_threads(0)
+    if kv_fill is not None:
+        m.fill_kv(kv_fill)
+    tok = si.make_prompt(cfg, 1, seed=10 + ctx)[0]
+    times, first = [], None
+    t_all = time.perf_counter()
+    while len(times) < max_steps:
+        t0 = time.perf_counter()
+        logits, am, _ = m.step(tok, ctx)
+        times.append(time.perf_counter() - t0)
+        if first is None:
+            first = logits
+        tok = am
+        if time.perf_counter() - t_all > budget_s:
+            break
+    return statistics.median(times) * 1e6, len(times), threads, first
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup(args.gpus)
+    if rank != 0:
+        return
+    name = args.workload
+    mname, ctx = WORKLOADS[name]
+    cfg = si.get_config(mname)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w = si.make_model(cfg, seed=0, device=dev)
+    kv = si.make_kv_fill(cfg, ctx, device=dev) if ctx else None
+    budget = float(os.environ.get("AMK_REF_BUDGET_S", "120"))
+    us, n, threads, _ = oracle_steps(cfg, w, ctx, kv, budget, args.steps + args.warmup)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(name, cfg, ctx),
+        "cpu_baseline": {"value": us, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{n} full fp64 decode steps of {name} (of "
+                                   f"{args.steps + args.warmup} requested; {budget:.0f} s cap)"},
+        "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(name, cfg, ctx):
+    return {"workload": f"{name}: random-init {cfg.name}-shaped decoder, batch 1, "
+                        f"greedy decode at KV context {ctx}",
+            "hidden": cfg.hidden, "layers": cfg.n_layers, "heads": cfg.n_heads,
+            "kv_heads": cfg.n_kv_heads, "head_dim": cfg.head_dim, "ffn": cfg.ffn,
+            "vocab": cfg.vocab, "kv_context": ctx, "weights": cfg.quant,
+            "tied_embeddings": cfg.tied, "global_batch": 1,
+            "l2": "inputs larger than L2 (weights streamed every step)"
+            if si.model_bytes(cfg)["linear"] > 126e6 else "weights fit in L2"}
+
+
+def run_ours(args):
+    import persistent_megakernel_decode_cta_b200 as amk
+    from persistent_megakernel_decode_cta_b200 import build as amk_build
+    world, rank, local = dist_setup(args.gpus)
+    if rank == 0:
+        amk_build.build()
+    barrier(world)
+    name = args.workload
+    mname, ctx = WORKLOADS[name]
+    cfg = si.get_config(mname)
+    if ctx + 2 > cfg.max_ctx:
+        raise SystemExit("context too large for the config")
+    w = si.make_model(cfg, seed=0, device="cuda")
+    kv = si.make_kv_fill(cfg, ctx, device="cuda") if ctx else None
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    opts = amk.default_options()
+    with torch.cuda.stream(stream):
+        dec = amk.Decoder(cfg, w, opts, stream=stream.cuda_stream)
+
+    def fill():
+        if kv is None:
+            return
+        for l in range(cfg.n_layers):
+            k, v = dec.kv(l)
+            k[:, :ctx].copy_(kv[l, 0])
+            v[:, :ctx].copy_(kv[l, 1])
+        torch.cuda.synchronize()
+
+    fill()
+    tok0 = si.make_prompt(cfg, 1, seed=10 + ctx)[0]
+    logits = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+
+    # ---- parity gate on the first step (rank 0 also times the oracle) -------
+    dec.step(tok0, ctx, logits=logits)
+    g = logits.double().cpu().numpy()
+    parity, cpu_base = None, None
+    if rank == 0:
+        budget = float(os.environ.get("AMK_CPU_BUDGET_S", "20"))
+        us, n, threads, ref = oracle_steps(cfg, w, ctx, kv, budget, 64)
+        scale = float(np.abs(ref).max())
+        err = float(np.abs(g - ref).max())
+        tol = (2e-2 if cfg.quant == "w8a16" else 1e-2) * scale
+        parity = {"verdict": "PASS" if err <= tol else "FAIL", "max_abs_dlogit": err,
+                  "tolerance": tol, "max_abs_logit": scale,
+                  "argmax_match": int(np.argmax(g)) == int(np.argmax(ref))}
+        cpu_base = {"value": us, "unit": UNIT, "cores": threads, "kind": "oracle",
+                    "sample": f"{n} full fp64 decode steps of {name} at position {ctx} "
+                              f"(~{budget:.0f} s budget), median"}
+
+    # ---- device timing --------------------------------------------------------
+    def step():
+        dec.step(-1, ctx, want_argmax=False)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            step()
+    torch.cuda.synchronize()
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            t_begin.record(stream)
+            for i in range(K):
+                starts[i].record(stream)
+                step()
+                ends[i].record(stream)
+            t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    # a step that timed out surfaces here
+    dec.step(-1, ctx, logits=logits)
+    elapsed_ms = t_begin.elapsed_time(t_end)
+    per_launch = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    elapsed_ms = max_over_ranks(world, elapsed_ms)
+    kernel_ms = max_over_ranks(world, statistics.mean(per_launch))
+
+    # ---- end to end: host token in, host logits + token out, every step ------
+    host_logits = torch.empty(cfg.vocab, dtype=torch.float32).pin_memory()
+    hl = host_logits.numpy()
+    tok = tok0
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            tok = dec.step_host(tok, ctx, hl)
+    K_e2e = max(10, min(K, 200))
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        for _ in range(K_e2e):
+            tok = dec.step_host(tok, ctx, hl)
+    e2e_s = max_over_ranks(world, time.perf_counter() - t0)
+
+    nbytes = algorithmic_bytes(cfg, ctx)
+    peak, peak_kind = measured_peak()
+    achieved = nbytes / (kernel_ms * 1e-3) / 1e9
+    value = elapsed_ms * 1e3 / (K * world)
+    st = dec.stats()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded random-init weights and KV cache)",
+            "config": dict(workload_config(name, cfg, ctx),
+                           parallelism=f"replicas{world}" if world > 1 else "single"),
+            "parity": parity,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": load_traffic(name),
+                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "kernel_us_per_launch": kernel_ms * 1e3},
+            "achieved_gbs": achieved,
+            "cpu_baseline": cpu_base,
+            "e2e": {"value": e2e_s * 1e6 / (K_e2e * world), "unit": UNIT,
+                    "h2d_bytes_per_step": 4, "d2h_bytes_per_step": cfg.vocab * 4 + 8 + 32,
+                    "steps": K_e2e},
+            "gpu_launches": K,
+            "clocks": clocks.summary(),
+            "schedule": {"tasks": st.n_tasks, "ctas": st.n_sms, "ring_stages": st.ring_stages,
+                         "stage_bytes": st.stage_bytes, "attn_splits": st.attn_splits,
+                         "smem_bytes": st.smem_bytes, "threads_per_cta": st.threads_per_cta},
+        }
+        if parity["verdict"] != "PASS":
+            line["value"] = None
+            line["error"] = "parity FAIL: timing withheld"
+        print(json.dumps(line), flush=True)
+    dec.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -451,7 +451,8 @@ int poll_pending_error(amk_handle *H)
     return absorb_error(H, *H->h_err);
 }
 
-int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev)
+int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev,
+                bool will_sync)
 {
     if (!H)
         return amk_set_error(AMK_ERR_INVALID_ARG, "NULL handle");
@@ -484,13 +485,18 @@ int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev)
                              "cooperative launch: %s", cudaGetErrorString(e));
     }
     H->epoch += 1;
-    e = cudaMemcpyAsync(H->h_err, H->d_err, sizeof(ErrorWord), cudaMemcpyDeviceToHost,
-                        H->stream);
-    if (e == cudaSuccess)
-        e = cudaEventRecord(H->err_ev, H->stream);
-    if (e != cudaSuccess)
-        return cuda_fail(e, "error word copy");
-    H->err_pending = true;
+    // The error word is read back when the caller synchronises, and every 32
+    // asynchronous steps otherwise (a failed step makes later kernels exit at
+    // once, so a late look costs no device time).
+    if (will_sync || (H->epoch % 32u) == 0u) {
+        e = cudaMemcpyAsync(H->h_err, H->d_err, sizeof(ErrorWord), cudaMemcpyDeviceToHost,
+                            H->stream);
+        if (e == cudaSuccess && !will_sync)
+            e = cudaEventRecord(H->err_ev, H->stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "error word copy");
+        H->err_pending = !will_sync;
+    }
     return AMK_OK;
 }
 
@@ -519,7 +525,7 @@ int finish_sync(amk_handle *H, int32_t *argmax_host)
 extern "C" int amk_decode_step(amk_handle *h, int32_t token_id, int32_t pos, float *logits_dev,
                                int32_t *argmax_host)
 {
-    int rc = launch_step(h, token_id, pos, logits_dev);
+    int rc = launch_step(h, token_id, pos, logits_dev, argmax_host != nullptr);
     if (rc != AMK_OK || !argmax_host)
         return rc;
     return finish_sync(h, argmax_host);
@@ -528,7 +534,7 @@ extern "C" int amk_decode_step(amk_handle *h, int32_t token_id, int32_t pos, flo
 extern "C" int amk_decode_step_host(amk_handle *h, int32_t token_id, int32_t pos,
                                     float *logits_host, int32_t *argmax_host)
 {
-    int rc = launch_step(h, token_id, pos, nullptr);
+    int rc = launch_step(h, token_id, pos, nullptr, true);
     if (rc != AMK_OK)
         return rc;
     if (logits_host) {

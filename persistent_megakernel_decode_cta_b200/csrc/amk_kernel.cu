@@ -807,11 +807,15 @@ __global__ void __launch_bounds__(kThreads, 1) amk_decode_kernel(const __grid_co
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], kConsumerWarps);
         }
-        s.flags[0] = 0;
+        // a failed earlier step poisons the device state: do no work until the
+        // host resets it (the counters no longer match the epoch)
+        s.flags[0] = ld_relaxed(&p.err->code) != 0u ? 1 : 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     __syncthreads();
+    if (s.flags[0])
+        return;
 
     if (warp == kConsumerWarps) {
         if (lane == 0)
