@@ -274,6 +274,43 @@ AMK_API int amk_get_workspace(amk_handle *h, amk_workspace *out);
 typedef struct { int32_t code, task, counter, sm; uint32_t seen, target; } amk_error_info;
 AMK_API int amk_get_error_info(amk_handle *h, amk_error_info *out);
 
+/* ---- decoding without allocating -------------------------------------- */
+/* (No counterpart in the AutoMegaKernel pages: an addition for callers that
+ * may not allocate device memory.)  Some callers cannot call cudaMalloc: a
+ * plugin inside an inference server or framework whose allocator owns every
+ * device byte, or a latency-critical loop where cudaMalloc/cudaFree would
+ * stall on an implicit device synchronisation.  amk_create allocates, so
+ * such a caller uses this entry point instead.  It runs the same decode step
+ * as amk_decode_step but allocates nothing: the caller passes the weights,
+ * the KV cache and the logits buffer, and the step's scratch (task table,
+ * counters, error word, argmax key, activations) lives in one fixed static
+ * device array of AMK_NOALLOC_SCRATCH_BYTES bytes, which every GPU that
+ * loads this library holds until the process exits.
+ *  plan:       from amk_plan_create, for at most the current device's SM count
+ *              (a host object; create it once, outside the loop).
+ *  w:          as for amk_create (device pointers, borrowed for the call).
+ *  kv_cache:   caller-owned device bf16 [n_layers][2][n_kv_heads][max_ctx][head_dim],
+ *              16-byte aligned; rows < pos must hold earlier steps' K/V (zeros
+ *              at first); the call writes row pos.
+ *  token_id:   0 <= token_id < vocab (no device-side token chaining here).
+ *  logits_dev: caller-owned device float [vocab] that receives the logits.
+ *  argmax_host: host int32 for the greedy token, or NULL.  Non-NULL makes the
+ *              call synchronise the stream and report a device error
+ *              (AMK_ERR_TIMEOUT); with NULL the call only enqueues work and
+ *              device errors are not reported.
+ * Returns AMK_ERR_UNSUPPORTED, without touching the GPU, when the model's
+ * scratch would exceed AMK_NOALLOC_SCRATCH_BYTES (amk_last_error says how
+ * much it needs).  The first call on each device looks up the static array's
+ * device address (cudaGetSymbolAddress); make that first call before any
+ * stream capture.  Every call re-uploads the schedule and clears the
+ * counters in the shared array, which keeps the last call's contents: calls
+ * that can overlap on the GPU (other streams, other host threads) race on
+ * it and must be serialised by the caller. */
+#define AMK_NOALLOC_SCRATCH_BYTES (16u << 20)
+AMK_API int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *w, void *kv_cache,
+                                    int32_t token_id, int32_t pos, float *logits_dev,
+                                    int32_t *argmax_host, void *cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -122,6 +122,8 @@ SIGNATURES = {
     "amk_get_stats": (ctypes.c_int, [c_vp, ctypes.POINTER(PlanStats)]),
     "amk_get_error_info": (ctypes.c_int, [c_vp, ctypes.POINTER(ErrorInfo)]),
     "amk_get_workspace": (ctypes.c_int, [c_vp, ctypes.POINTER(Workspace)]),
+    "amk_decode_step_noalloc": (ctypes.c_int, [c_vp, ctypes.POINTER(Weights), c_vp, c_i32,
+                                               c_i32, c_vp, ctypes.POINTER(c_i32), c_vp]),
 }
 
 _LIB = None

@@ -1,0 +1,255 @@
+// amk_noalloc.cu -- a decode step that allocates no memory.
+//
+// Some callers cannot call cudaMalloc: plugins inside an inference server or
+// a framework whose allocator owns every device byte (a stray cudaMalloc
+// breaks its accounting and can fail when the pool has reserved the rest of
+// the GPU), and latency-critical loops where cudaMalloc/cudaFree would stall
+// on an implicit device synchronisation.  amk_create allocates the KV cache
+// and the workspace, so those callers use amk_decode_step_noalloc instead:
+// the caller owns the weights, the KV cache and the logits, and the step's
+// scratch (task table, counters, error word, argmax key, activations) lives
+// in the fixed array g_scratch below, which exists once per GPU from the
+// moment the library's device code is loaded until the process exits.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "amk.h"
+#include "amk_internal.h"
+#include "amk_plan.h"
+
+extern "C" int amk_kernel_smem_bytes(int ring_stages, int stage_bytes, int vec_floats);
+extern "C" cudaError_t amk_kernel_configure(int smem_bytes);
+namespace amk {
+extern "C" cudaError_t amk_kernel_launch(const KParams *p, int n_ctas, int smem_bytes,
+                                         cudaStream_t stream);
+}
+
+namespace {
+
+constexpr size_t kScratchBytes = AMK_NOALLOC_SCRATCH_BYTES;
+__device__ __align__(256) unsigned char g_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void *g_scratch_addr[kMaxDevices];  // device address of g_scratch, per device
+
+size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+struct Layout {
+    size_t tasks, qoff, layers, ctr, err, argkey, qkv, part, xmid, xout, act, total;
+};
+
+Layout layout_of(const amk_plan &P)
+{
+    const amk_config &c = P.cfg;
+    const size_t L = (size_t)c.n_layers;
+    const size_t part = (size_t)c.n_kv_heads * P.opt.attn_splits * P.group * (c.head_dim + 2);
+    Layout o{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = off;
+        off = up256(off + bytes);
+        return at;
+    };
+    o.tasks = take(sizeof(amk::TaskDesc) * P.tasks.size());
+    o.qoff = take(sizeof(int32_t) * P.queue_off.size());
+    o.layers = take(sizeof(amk::LayerPtrs) * L);
+    o.ctr = take(sizeof(uint32_t) * (size_t)P.n_counters);
+    o.err = take(sizeof(amk::ErrorWord));
+    o.argkey = take(2 * sizeof(unsigned long long));
+    o.qkv = take(sizeof(float) * L * P.qkv_rows);
+    o.part = take(sizeof(float) * L * part);
+    o.xmid = take(sizeof(float) * L * c.hidden);
+    o.xout = take(sizeof(float) * L * c.hidden);
+    o.act = take(sizeof(float) * L * c.ffn);
+    o.total = off;
+    return o;
+}
+
+// Device address of g_scratch for the current device, looked up on the first
+// call for that device.
+int scratch_address(unsigned char **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return amk_set_error(AMK_ERR_NO_DEVICE, "amk_decode_step_noalloc: %s",
+                             cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices)
+        return amk_set_error(AMK_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_scratch);
+        if (e != cudaSuccess || !p)
+            return amk_set_error(AMK_ERR_CUDA, "cudaGetSymbolAddress(g_scratch): %s",
+                                 cudaGetErrorString(e));
+        g_scratch_addr[dev] = p;
+    }
+    *out = static_cast<unsigned char *>(g_scratch_addr[dev]);
+    return AMK_OK;
+}
+
+bool ok16(const void *p) { return p && ((uintptr_t)p % 16) == 0; }
+
+int fail_cuda(cudaError_t e, const char *what)
+{
+    return amk_set_error(AMK_ERR_CUDA, "amk_decode_step_noalloc: %s: %s", what,
+                         cudaGetErrorString(e));
+}
+
+}  // namespace
+
+extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *w,
+                                       void *kv_cache, int32_t token_id, int32_t pos,
+                                       float *logits_dev, int32_t *argmax_host,
+                                       void *cuda_stream)
+{
+    if (!plan || !w || !ok16(kv_cache) || !logits_dev || ((uintptr_t)logits_dev % 4))
+        return amk_set_error(AMK_ERR_INVALID_ARG,
+                             "amk_decode_step_noalloc: NULL or misaligned argument");
+    const amk_plan &P = *plan;
+    const amk_config &c = P.cfg;
+    if (pos < 0 || pos >= c.max_ctx || token_id < 0 || token_id >= c.vocab)
+        return amk_set_error(AMK_ERR_POS_RANGE, "amk_decode_step_noalloc: token %d / pos %d "
+                             "out of range", token_id, pos);
+    const bool q8 = c.quant == AMK_QUANT_W8A16;
+    if (!ok16(w->embed) || !ok16(w->final_norm) || !w->attn_norm || !w->ffn_norm ||
+        (!c.tied_embeddings && (!ok16(w->lm_head) || (q8 && !w->lm_head_scale))))
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_decode_step_noalloc: weights");
+    const void *const *mats[7] = {w->wq, w->wk, w->wv, w->wo, w->wgate, w->wup, w->wdown};
+    const void *const *scs[7] = {w->sq, w->sk, w->sv, w->so, w->sgate, w->sup, w->sdown};
+    for (int m = 0; m < 7; ++m)
+        if (!mats[m] || (q8 && !scs[m]))
+            return amk_set_error(AMK_ERR_INVALID_ARG, "amk_decode_step_noalloc: weights");
+    const Layout lay = layout_of(P);
+    if (lay.total > kScratchBytes)
+        return amk_set_error(AMK_ERR_UNSUPPORTED,
+                             "amk_decode_step_noalloc: this model needs %zu bytes of scratch, "
+                             "more than the %zu-byte static array; use amk_create",
+                             lay.total, kScratchBytes);
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (P.n_sms > sms)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "plan made for %d SMs, device has %d",
+                             P.n_sms, sms);
+    unsigned char *base = nullptr;
+    int rc = scratch_address(&base);
+    if (rc != AMK_OK)
+        return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    cudaError_t e;
+    // schedule tables (pageable sources: cudaMemcpyAsync stages them before
+    // returning, so the stack buffer below can be reused at once)
+    e = cudaMemcpyAsync(base + lay.tasks, P.tasks.data(), sizeof(amk::TaskDesc) * P.tasks.size(),
+                        cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(base + lay.qoff, P.queue_off.data(),
+                            sizeof(int32_t) * P.queue_off.size(), cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess)
+        return fail_cuda(e, "schedule upload");
+    amk::LayerPtrs lp[16];
+    for (int l0 = 0; l0 < c.n_layers; l0 += 16) {
+        const int n = c.n_layers - l0 < 16 ? c.n_layers - l0 : 16;
+        for (int i = 0; i < n; ++i) {
+            const int l = l0 + i;
+            if (!ok16(w->attn_norm[l]) || !ok16(w->ffn_norm[l]))
+                return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d norm NULL or misaligned", l);
+            for (int m = 0; m < 7; ++m) {
+                if (!ok16(mats[m][l]) || (q8 && !scs[m][l]))
+                    return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d weight %d", l, m);
+                lp[i].w[m] = mats[m][l];
+                lp[i].s[m] = q8 ? static_cast<const uint16_t *>(scs[m][l]) : nullptr;
+            }
+            lp[i].attn_norm = static_cast<const uint16_t *>(w->attn_norm[l]);
+            lp[i].ffn_norm = static_cast<const uint16_t *>(w->ffn_norm[l]);
+        }
+        e = cudaMemcpyAsync(base + lay.layers + sizeof(amk::LayerPtrs) * l0, lp,
+                            sizeof(amk::LayerPtrs) * n, cudaMemcpyHostToDevice, st);
+        if (e != cudaSuccess)
+            return fail_cuda(e, "layer table upload");
+    }
+    // what must start at zero: counters, error word, argmax keys
+    e = cudaMemsetAsync(base + lay.ctr, 0, lay.qkv - lay.ctr, st);
+    if (e != cudaSuccess)
+        return fail_cuda(e, "scratch clear");
+
+    amk::KParams k{};
+    k.tasks = reinterpret_cast<const amk::TaskDesc *>(base + lay.tasks);
+    k.queue_off = reinterpret_cast<const int32_t *>(base + lay.qoff);
+    k.counters = reinterpret_cast<uint32_t *>(base + lay.ctr);
+    k.err = reinterpret_cast<amk::ErrorWord *>(base + lay.err);
+    k.layers = reinterpret_cast<const amk::LayerPtrs *>(base + lay.layers);
+    k.embed = static_cast<const uint16_t *>(w->embed);
+    k.final_norm = static_cast<const uint16_t *>(w->final_norm);
+    k.lm_head = static_cast<const uint16_t *>(c.tied_embeddings ? w->embed : w->lm_head);
+    k.lm_head_scale = (q8 && !c.tied_embeddings)
+                          ? static_cast<const uint16_t *>(w->lm_head_scale) : nullptr;
+    k.qkv = reinterpret_cast<float *>(base + lay.qkv);
+    k.part = reinterpret_cast<float *>(base + lay.part);
+    k.xmid = reinterpret_cast<float *>(base + lay.xmid);
+    k.xout = reinterpret_cast<float *>(base + lay.xout);
+    k.act = reinterpret_cast<float *>(base + lay.act);
+    k.logits = logits_dev;
+    k.argkey = reinterpret_cast<unsigned long long *>(base + lay.argkey);
+    k.kv = static_cast<uint16_t *>(kv_cache);
+    k.hidden = c.hidden;
+    k.n_layers = c.n_layers;
+    k.n_heads = c.n_heads;
+    k.n_kv_heads = c.n_kv_heads;
+    k.head_dim = c.head_dim;
+    k.ffn = c.ffn;
+    k.vocab = c.vocab;
+    k.max_ctx = c.max_ctx;
+    k.qkv_rows = P.qkv_rows;
+    k.group = P.group;
+    k.attn_splits = P.opt.attn_splits;
+    k.quant = q8 ? 1 : 0;
+    k.tied = c.tied_embeddings ? 1 : 0;
+    k.rms_eps = c.rms_eps;
+    k.rope_theta = c.rope_theta;
+    k.ring_stages = P.opt.ring_stages;
+    k.stage_bytes = P.opt.stage_bytes;
+    k.vec_floats = P.vec_floats;
+    k.att_lph = P.att_lph;
+    k.att_hpb = P.att_hpb;
+    k.att_e = P.att_e;
+    k.pos = pos;
+    k.token = token_id;
+    k.epoch = 0;   // counters were cleared above
+    k.parity = 0;
+    k.timeout_ns = (uint64_t)P.opt.wait_timeout_us * 1000ull;
+    k.skip_signal_task = P.opt.debug_skip_signal_task;
+    e = amk_kernel_configure(P.smem_bytes);
+    if (e != cudaSuccess)
+        return fail_cuda(e, "cudaFuncSetAttribute");
+    e = amk::amk_kernel_launch(&k, P.n_sms, P.smem_bytes, st);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return amk_set_error(e == cudaErrorCooperativeLaunchTooLarge ? AMK_ERR_LAUNCH
+                                                                      : AMK_ERR_CUDA,
+                             "amk_decode_step_noalloc: launch: %s", cudaGetErrorString(e));
+    }
+    if (!argmax_host)
+        return AMK_OK;
+    // pageable destinations: these copies complete before the calls return
+    unsigned long long key = 0;
+    amk::ErrorWord ew;
+    e = cudaMemcpyAsync(&ew, base + lay.err, sizeof ew, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(&key, base + lay.argkey, sizeof key, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess)
+        return fail_cuda(e, "result copy");
+    if (ew.code != 0)
+        return amk_set_error(ew.code == 3 ? AMK_ERR_POS_RANGE : AMK_ERR_TIMEOUT,
+                             "amk_decode_step_noalloc: device error %u (task %d, counter %d)",
+                             ew.code, ew.task, ew.counter);
+    *argmax_host = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+    return AMK_OK;
+}
