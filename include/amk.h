@@ -108,7 +108,8 @@ typedef struct {
     int32_t n_sms;            /* persistent CTAs; 0 = all SMs of the device */
     uint32_t wait_timeout_us; /* limit of every device-side wait */
     int32_t debug_skip_signal_task; /* test hook: this task id never signals; -1 = off */
-    int32_t reserved[8];
+    int32_t profile;          /* 1: record per-CTA phase timers (amk_get_profile) */
+    int32_t reserved[7];
 } amk_options;
 
 typedef struct amk_handle amk_handle;
@@ -268,6 +269,26 @@ AMK_API int amk_get_stats(amk_handle *h, amk_plan_stats *out);
  *   act  [n_layers][ffn]       SwiGLU activations */
 typedef struct { float *qkv, *xmid, *xout, *act; int32_t qkv_rows; } amk_workspace;
 AMK_API int amk_get_workspace(amk_handle *h, amk_workspace *out);
+
+/* Phase timers of the last step, recorded when amk_options.profile was 1
+ * (tracing; README, "Honesty rules": always report the distance to the
+ * roofline and where the time goes).  Fills `out` (host, n_u64 entries) with
+ * n_sms * AMK_PROF_KINDS * AMK_PROF_FIELDS uint64 values, index
+ * ((cta * AMK_PROF_KINDS) + kind) * AMK_PROF_FIELDS + field, where kind is
+ * the task kind (1 QKV, 2 ATTN, 3 OPROJ, 4 GATEUP, 5 DOWN, 6 LMHEAD) and the
+ * fields are: 0 tasks, 1 ns waiting on counters, 2 ns in prologues, 3 ns the
+ * consumers waited for ring stages, 4 ns from the end of the counter wait to
+ * the signal, 5 ns in epilogues, 6 ns all consumer warps together waited for
+ * ring stages, 7 ns all consumer warps together spent in their GEMV or
+ * attention loops outside those waits.  Kind 0 holds per-CTA totals: field 0
+ * the kernel start (globaltimer ns), 1 the consumers' end, 2 ns the producer
+ * waited for free stages, 3 the producer's end, 4 bytes the producer copied,
+ * 5 ns the producer spent between tasks (reading descriptors and pointers).
+ * Synchronises the stream.  AMK_ERR_INVALID_ARG if profiling was off or
+ * n_u64 is too small. */
+#define AMK_PROF_KINDS 8
+#define AMK_PROF_FIELDS 8
+AMK_API int amk_get_profile(amk_handle *h, uint64_t *out, int64_t n_u64);
 
 /* After AMK_ERR_TIMEOUT: the task that gave up, the counter it waited on,
  * the value it saw and the value it needed. */

@@ -273,6 +273,16 @@ class Decoder:
         return {"qkv": view(ws.qkv, ws.qkv_rows), "xmid": view(ws.xmid, self.cfg.hidden),
                 "xout": view(ws.xout, self.cfg.hidden), "act": view(ws.act, self.cfg.ffn)}
 
+    def profile(self):
+        """Phase timers of the last step (needs options.profile = 1): a uint64
+        numpy array [n_sms, 8 kinds, 8 fields] (see amk_get_profile)."""
+        import numpy as np
+        n = self.stats().n_sms * 8 * 8
+        buf = np.zeros(n, dtype=np.uint64)
+        _check(abi.lib().amk_get_profile(self._h, buf.ctypes.data_as(
+            ctypes.POINTER(ctypes.c_uint64)), n), "amk_get_profile")
+        return buf.reshape(-1, 8, 8)
+
     def stats(self) -> abi.PlanStats:
         s = abi.PlanStats()
         _check(abi.lib().amk_get_stats(self._h, ctypes.byref(s)), "amk_get_stats")

@@ -44,7 +44,8 @@ class Weights(ctypes.Structure):
 class Options(ctypes.Structure):
     _fields_ = [("ring_stages", c_i32), ("stage_bytes", c_i32), ("attn_splits", c_i32),
                 ("tasks_per_sm", c_i32), ("n_sms", c_i32), ("wait_timeout_us", c_u32),
-                ("debug_skip_signal_task", c_i32), ("reserved", c_i32 * 8)]
+                ("debug_skip_signal_task", c_i32), ("profile", c_i32),
+                ("reserved", c_i32 * 7)]
 
 
 class GraphWait(ctypes.Structure):
@@ -122,6 +123,7 @@ SIGNATURES = {
     "amk_get_stats": (ctypes.c_int, [c_vp, ctypes.POINTER(PlanStats)]),
     "amk_get_error_info": (ctypes.c_int, [c_vp, ctypes.POINTER(ErrorInfo)]),
     "amk_get_workspace": (ctypes.c_int, [c_vp, ctypes.POINTER(Workspace)]),
+    "amk_get_profile": (ctypes.c_int, [c_vp, ctypes.POINTER(ctypes.c_uint64), c_i64]),
     "amk_decode_step_noalloc": (ctypes.c_int, [c_vp, ctypes.POINTER(Weights), c_vp, c_i32,
                                                c_i32, c_vp, ctypes.POINTER(c_i32), c_vp]),
 }

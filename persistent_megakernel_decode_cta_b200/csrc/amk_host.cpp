@@ -21,11 +21,11 @@
 
 using amk::ErrorWord;
 using amk::KParams;
-using amk::LayerPtrs;
 using amk::TaskDesc;
 
-extern "C" cudaError_t amk_kernel_configure(int smem_bytes);
-extern "C" cudaError_t amk_kernel_occupancy(int smem_bytes, int *blocks_per_sm);
+extern "C" cudaError_t amk_kernel_configure(int smem_bytes, int quant, int att_e, int generic);
+extern "C" cudaError_t amk_kernel_occupancy(int smem_bytes, int quant, int att_e, int generic,
+                                            int *blocks_per_sm);
 namespace amk {
 extern "C" cudaError_t amk_kernel_launch(const KParams *p, int n_ctas, int smem_bytes,
                                          cudaStream_t stream);
@@ -71,8 +71,8 @@ extern "C" int amk_default_options(amk_options *o)
     if (!o)
         return amk_set_error(AMK_ERR_INVALID_ARG, "amk_default_options: NULL");
     memset(o, 0, sizeof *o);
-    o->ring_stages = 6;
-    o->stage_bytes = 32768;
+    o->ring_stages = 3;
+    o->stage_bytes = 65536;
     o->attn_splits = 0;
     o->tasks_per_sm = 1;
     o->n_sms = 0;
@@ -141,10 +141,10 @@ struct amk_handle {
     int32_t *d_qoff = nullptr;
     uint32_t *d_ctr = nullptr;
     ErrorWord *d_err = nullptr;
-    LayerPtrs *d_layers = nullptr;
     float *d_qkv = nullptr, *d_part = nullptr, *d_xmid = nullptr, *d_xout = nullptr;
     float *d_act = nullptr, *d_logits = nullptr;
     unsigned long long *d_argkey = nullptr;
+    unsigned long long *d_prof = nullptr;
     uint16_t *d_kv = nullptr;
     size_t kv_bytes = 0, act_bytes = 0;
     ErrorWord *h_err = nullptr;            // pinned
@@ -307,13 +307,14 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
         return rc;
     }
     const amk_plan *P = H->plan;
-    cudaError_t e = amk_kernel_configure(P->smem_bytes);
+    const int q8 = P->cfg.quant == AMK_QUANT_W8A16 ? 1 : 0;
+    cudaError_t e = amk_kernel_configure(P->smem_bytes, q8, P->att_e, P->generic);
     if (e != cudaSuccess) {
         free_handle(H);
         return cuda_fail(e, "cudaFuncSetAttribute");
     }
     int per_sm = 0;
-    e = amk_kernel_occupancy(P->smem_bytes, &per_sm);
+    e = amk_kernel_occupancy(P->smem_bytes, q8, P->att_e, P->generic, &per_sm);
     if (e != cudaSuccess || per_sm < 1) {
         free_handle(H);
         return amk_set_error(AMK_ERR_LAUNCH, "kernel does not fit one SM (smem %d B)",
@@ -332,11 +333,13 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
         (rc = dalloc(H, &H->d_qoff, sizeof(int32_t) * P->queue_off.size())) ||
         (rc = dalloc(H, &H->d_ctr, sizeof(uint32_t) * (size_t)P->n_counters)) ||
         (rc = dalloc(H, &H->d_err, sizeof(ErrorWord))) ||
-        (rc = dalloc(H, &H->d_layers, sizeof(LayerPtrs) * (size_t)L)) ||
         (rc = dalloc(H, &act_block, H->act_bytes)) ||
         (rc = dalloc(H, &H->d_logits, sizeof(float) * (size_t)c.vocab)) ||
         (rc = dalloc(H, &H->d_argkey, 2 * sizeof(unsigned long long))) ||
-        (rc = dalloc(H, &H->d_kv, H->kv_bytes))) {
+        (rc = dalloc(H, &H->d_kv, H->kv_bytes)) ||
+        (P->opt.profile &&
+         (rc = dalloc(H, &H->d_prof, sizeof(unsigned long long) * (size_t)n_sms *
+                                         amk::kProfKinds * amk::kProfFields)))) {
         free_handle(H);
         return rc;
     }
@@ -351,25 +354,14 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
         free_handle(H);
         return cuda_fail(e, "host buffers");
     }
-    std::vector<LayerPtrs> lp(L);
-    const void *const *mats[7] = {w->wq, w->wk, w->wv, w->wo, w->wgate, w->wup, w->wdown};
-    const void *const *scs[7] = {w->sq, w->sk, w->sv, w->so, w->sgate, w->sup, w->sdown};
-    const bool q8 = c.quant == AMK_QUANT_W8A16;
-    for (int l = 0; l < L; ++l) {
-        for (int m = 0; m < 7; ++m) {
-            lp[l].w[m] = mats[m][l];
-            lp[l].s[m] = q8 ? static_cast<const uint16_t *>(scs[m][l]) : nullptr;
-        }
-        lp[l].attn_norm = static_cast<const uint16_t *>(w->attn_norm[l]);
-        lp[l].ffn_norm = static_cast<const uint16_t *>(w->ffn_norm[l]);
-    }
-    if ((e = cudaMemcpyAsync(H->d_tasks, P->tasks.data(), sizeof(TaskDesc) * P->tasks.size(),
+    std::vector<TaskDesc> resolved(P->tasks.size());
+    for (size_t t = 0; t < resolved.size(); ++t)
+        amk_resolve_task(P, w, H->d_kv, (int)t, &resolved[t]);
+    if ((e = cudaMemcpyAsync(H->d_tasks, resolved.data(), sizeof(TaskDesc) * resolved.size(),
                              cudaMemcpyHostToDevice, H->stream)) != cudaSuccess ||
         (e = cudaMemcpyAsync(H->d_qoff, P->queue_off.data(),
                              sizeof(int32_t) * P->queue_off.size(), cudaMemcpyHostToDevice,
-                             H->stream)) != cudaSuccess ||
-        (e = cudaMemcpyAsync(H->d_layers, lp.data(), sizeof(LayerPtrs) * lp.size(),
-                             cudaMemcpyHostToDevice, H->stream)) != cudaSuccess) {
+                             H->stream)) != cudaSuccess) {
         free_handle(H);
         return cuda_fail(e, "upload schedule");
     }
@@ -377,7 +369,7 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
         free_handle(H);
         return rc;
     }
-    if ((e = cudaStreamSynchronize(H->stream)) != cudaSuccess) {
+    if ((e = cudaStreamSynchronize(H->stream)) != cudaSuccess) {  // also frees `resolved`'s use
         free_handle(H);
         return cuda_fail(e, "amk_create");
     }
@@ -386,12 +378,7 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     k.queue_off = H->d_qoff;
     k.counters = H->d_ctr;
     k.err = H->d_err;
-    k.layers = H->d_layers;
     k.embed = static_cast<const uint16_t *>(w->embed);
-    k.final_norm = static_cast<const uint16_t *>(w->final_norm);
-    k.lm_head = static_cast<const uint16_t *>(c.tied_embeddings ? w->embed : w->lm_head);
-    k.lm_head_scale = (q8 && !c.tied_embeddings) ? static_cast<const uint16_t *>(w->lm_head_scale)
-                                                  : nullptr;
     k.qkv = H->d_qkv;
     k.part = H->d_part;
     k.xmid = H->d_xmid;
@@ -411,7 +398,7 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     k.qkv_rows = P->qkv_rows;
     k.group = P->group;
     k.attn_splits = P->opt.attn_splits;
-    k.quant = q8 ? 1 : 0;
+    k.quant = q8;
     k.tied = c.tied_embeddings ? 1 : 0;
     k.rms_eps = c.rms_eps;
     k.rope_theta = c.rope_theta;
@@ -421,8 +408,10 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     k.att_lph = P->att_lph;
     k.att_hpb = P->att_hpb;
     k.att_e = P->att_e;
+    k.generic = P->generic;
     k.timeout_ns = (uint64_t)P->opt.wait_timeout_us * 1000ull;
     k.skip_signal_task = P->opt.debug_skip_signal_task;
+    k.prof = H->d_prof;
     *out = H;
     return AMK_OK;
 }
@@ -477,6 +466,14 @@ int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev,
     k.parity = (int32_t)(H->epoch & 1u);
     if (logits_dev)
         k.logits = logits_dev;
+    if (H->d_prof) {
+        cudaError_t pe = cudaMemsetAsync(H->d_prof, 0,
+                                         sizeof(unsigned long long) * (size_t)H->plan->n_sms *
+                                             amk::kProfKinds * amk::kProfFields,
+                                         H->stream);
+        if (pe != cudaSuccess)
+            return cuda_fail(pe, "profile clear");
+    }
     cudaError_t e = amk::amk_kernel_launch(&k, H->plan->n_sms, H->plan->smem_bytes, H->stream);
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -597,6 +594,23 @@ extern "C" int amk_get_workspace(amk_handle *h, amk_workspace *out)
     out->xout = h->d_xout;
     out->act = h->d_act;
     out->qkv_rows = h->plan->qkv_rows;
+    return AMK_OK;
+}
+
+extern "C" int amk_get_profile(amk_handle *h, uint64_t *out, int64_t n_u64)
+{
+    if (!h || !out || !h->d_prof)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_get_profile: profiling is off or NULL");
+    const int64_t need = (int64_t)h->plan->n_sms * amk::kProfKinds * amk::kProfFields;
+    if (n_u64 < need)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_get_profile: need %lld entries",
+                             (long long)need);
+    cudaError_t e = cudaMemcpyAsync(out, h->d_prof, sizeof(uint64_t) * (size_t)need,
+                                    cudaMemcpyDeviceToHost, h->stream);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(h->stream);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "amk_get_profile");
     return AMK_OK;
 }
 

@@ -19,10 +19,20 @@ int amk_set_error(int code, const char *fmt, ...);
 
 namespace amk {
 
-// Persistent CTA shape: 8 consumer warps (compute) + 1 producer warp (TMA).
+// Persistent CTA shape: one producer warpgroup (lane 0 of its first warp
+// issues the TMA bulk copies; the warpgroup drops to kProducerRegs registers)
+// and two consumer warpgroups = 8 compute warps (raised to kConsumerRegs).
+// 128 * 56 + 256 * 224 = 384 * 168: the split uses exactly the registers the
+// block is launched with.
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kThreads = kConsumerThreads + 32;
+constexpr int kProducerThreads = 128;
+constexpr int kThreads = kProducerThreads + kConsumerThreads;
+constexpr int kLaunchRegs = 168;
+constexpr int kProducerRegs = 56;
+constexpr int kConsumerRegs = 224;
+static_assert(kProducerThreads * kProducerRegs + kConsumerThreads * kConsumerRegs ==
+                  kThreads * kLaunchRegs, "register split must equal the launch budget");
 constexpr int kMaxTaskRows = 256;   // output rows of one GEMV task (red buffer)
 constexpr int kMaxStages = 16;
 
@@ -41,16 +51,22 @@ enum TaskFlags : uint8_t {
     TF_RESET_ARGKEY = 1,  // this task clears the next step's argmax key
 };
 
-struct TaskDesc {           // 32 bytes
+struct TaskDesc {           // 80 bytes, read-only for the kernel
     uint8_t kind, mat, flags, pad;
     int32_t layer;
     int32_t wait_ctr;       // -1: no wait
     uint32_t wait_count;    // threshold t within one epoch
     uint32_t wait_total;    // producers of wait_ctr (signals per epoch)
     int32_t signal_ctr;     // -1: no signal
-    int32_t r0, r1;         // GEMV: output rows [r0, r1); ATTN: r0 = g, r1 = c
+    int32_t r0, r1;         // GEMV: output rows [r0, r1); ATTN: r0 = kv head g, r1 = chunk c
+    // resolved by the host once the weights are known:
+    const void *w0, *w1;    // GEMV: row r0 of part 0 / part 1 (gate/up); ATTN: K / V cache
+                            //   block of (layer, g)
+    const uint16_t *s0, *s1;  // fp16 row scales at row r0 (W8A16), or null
+    const uint16_t *gain;     // RMSNorm gain of the prologue, or null
+    uint64_t pad2;
 };
-static_assert(sizeof(TaskDesc) == 32, "TaskDesc is 32 bytes");
+static_assert(sizeof(TaskDesc) == 80, "TaskDesc is 80 bytes");
 
 // Per-layer weight pointers (device copies of the caller's pointers).
 struct LayerPtrs {
@@ -73,9 +89,8 @@ struct KParams {
     const int32_t *queue_off;  // [n_sms + 1]
     uint32_t *counters;
     ErrorWord *err;
-    // weights
-    const LayerPtrs *layers;
-    const uint16_t *embed, *final_norm, *lm_head, *lm_head_scale;
+    // weights (the per-task pointers live in the task records)
+    const uint16_t *embed;
     // state and activations (fp32 unless noted)
     float *qkv;       // [L][qkv_rows]: q | k | v, before RoPE
     float *part;      // [L][nkv][C][G][hd + 2]: split-K partials (m, l, o[hd])
@@ -93,13 +108,17 @@ struct KParams {
     int32_t ring_stages, stage_bytes, vec_floats;
     // attention lane layout
     int32_t att_lph, att_hpb, att_e;  // lanes per head, heads per batch, elems per lane
+    int32_t generic;            // 1: run the generic kernel instance
     // step
     int32_t pos, token;         // token < 0: previous step's argmax
     uint32_t epoch;             // steps since reset (counter targets)
     int32_t parity;             // epoch & 1
     uint64_t timeout_ns;
     int32_t skip_signal_task;   // test hook, -1 = off
+    unsigned long long *prof;   // [n_sms][kProfKinds][kProfFields] phase timers, or null
 };
+constexpr int kProfKinds = AMK_PROF_KINDS;
+constexpr int kProfFields = AMK_PROF_FIELDS;
 
 }  // namespace amk
 

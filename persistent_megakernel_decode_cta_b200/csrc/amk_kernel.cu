@@ -10,19 +10,22 @@
 // one computes (README, "Why a megakernel").
 //
 // B200 design (not the pages' sm_80..sm_120 design):
-//  * 288 threads per CTA: 8 consumer warps compute, 1 producer warp streams.
-//  * The producer walks the same queue AHEAD of the consumers and copies each
-//    task's weight rows (or KV-cache rows) into a ring of shared-memory
-//    stages with cp.async.bulk (TMA bulk copies) that complete on per-stage
-//    mbarriers.  Weights never depend on activations, so the copies run
-//    ahead across counter waits: the wait latency is hidden behind the ring.
-//  * Consumers wait on the counter (ld.acquire.gpu spin with a time limit),
-//    build the task's input vector in shared memory (RMSNorm / split-K
-//    combine prologues, all from L2 with .cg loads), run the GEMV from the
-//    ring with each warp owning a fixed K-slice whose activations sit in
-//    registers, reduce with warp shuffles, apply the fused epilogue
-//    (RoPE+KV append, SwiGLU, residual add, argmax), then release their
-//    stores with red.release.gpu on the task's counter.
+//  * 384 threads per CTA in three warpgroups.  The producer warpgroup gives
+//    up registers (setmaxnreg) and one lane walks the SM's queue AHEAD of the
+//    consumers, copying each task's weight rows (or KV-cache rows) into a
+//    ring of shared-memory stages with cp.async.bulk (TMA bulk copies) that
+//    complete on per-stage mbarriers.  Weights never depend on activations,
+//    so the copies run ahead across counter waits.
+//  * Two consumer warpgroups (8 warps) take the freed registers.  They wait
+//    on the task's counter (ld.acquire.gpu spin with a time limit), build
+//    the task's input vector in shared memory (RMSNorm / split-K combine
+//    prologues, from L2 with .cg loads), run the GEMV from the ring -- each
+//    warp owns a K-slice whose activations sit in registers -- reduce with
+//    warp shuffles, apply the fused epilogue (RoPE + KV append, SwiGLU,
+//    residual add, argmax), then release their stores with red.release.gpu
+//    on the task's counter.
+//  * Task records carry host-resolved pointers and are prefetched one task
+//    ahead, so no task boundary waits on a dependent global load.
 //  * Every wait is bounded (globaltimer + iteration cap); on expiry the CTA
 //    records the failure, drains its own TMA copies and returns.
 #include <cuda_bf16.h>
@@ -40,22 +43,20 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
 {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
 }
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
 {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-                 "r"(bytes)
-                 : "memory");
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
@@ -63,26 +64,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
-                                         uint64_t *bar, uint64_t policy)
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                         uint32_t bar, uint64_t policy)
 {
     asm volatile(
         "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint "
-        "[%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        "[%0], [%1], %2, [%3], %4;" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
         : "memory");
 }
-__device__ __forceinline__ void bulk_g2s_nohint(void *dst, const void *src, uint32_t bytes,
-                                                uint64_t *bar)
+__device__ __forceinline__ void bulk_g2s_nohint(uint32_t dst, const void *src, uint32_t bytes,
+                                                uint32_t bar)
 {
     asm volatile(
         "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
 __device__ __forceinline__ uint64_t evict_first_policy()
@@ -117,6 +118,50 @@ __device__ __forceinline__ void consumer_bar()
 {
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
 }
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Explicit shared-memory accesses by 32-bit shared address, so the hot
+// loops use ld.shared/st.shared.  Ordering against the ring's TMA writes
+// comes from the mbarrier waits (asm volatile with a memory clobber).
+__device__ __forceinline__ uint4 lds128(uint32_t a)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a)
+{
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void stsf(uint32_t a, float v)
+{
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v));
+}
 
 // ------------------------------------------------------------- number formats
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
@@ -126,44 +171,95 @@ __device__ __forceinline__ uint16_t f_to_bf16(float f)
 }
 __device__ __forceinline__ float fp16_to_f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
 
-// int8 -> float exactly: 0x4B000000 | (q + 128) is the float 2^23 + q + 128.
-__device__ __forceinline__ float i8f(uint32_t biased_word, uint32_t sel)
+// Packed pairs of floats (f32x2 arithmetic: one instruction per two lanes'
+// worth of work).
+typedef unsigned long long f2_t;
+__device__ __forceinline__ f2_t pk2(float a, float b)
 {
-    return __uint_as_float(__byte_perm(biased_word, 0x4B000000u, sel)) - 8388736.0f;
+    f2_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float sum2(f2_t r)
+{
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+    return a + b;
+}
+__device__ __forceinline__ f2_t ffma2(f2_t a, f2_t b, f2_t c)
+{
+    f2_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ f2_t fadd2(f2_t a, f2_t b)
+{
+    f2_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// two bf16 in a word -> (low, high) as a float pair
+__device__ __forceinline__ f2_t bf2(uint32_t w)
+{
+    f2_t r;
+    asm("{\n\t.reg .b32 lo, hi;\n\tshl.b32 lo, %1, 16;\n\tand.b32 hi, %1, 0xffff0000;\n\t"
+        "mov.b64 %0, {lo, hi};\n\t}"
+        : "=l"(r)
+        : "r"(w));
+    return r;
+}
+// four int8 in a word -> two float pairs, exactly: 0x4B000000 | (q + 128) is
+// the float 2^23 + q + 128, and the pair subtraction removes the offset
+__device__ __forceinline__ void i8x4(uint32_t w, f2_t &lo, f2_t &hi)
+{
+    const uint32_t b = w ^ 0x80808080u;
+    const f2_t off = pk2(-8388736.0f, -8388736.0f);
+    lo = fadd2(pk2(__uint_as_float(__byte_perm(b, 0x4B000000u, 0x7440)),
+                   __uint_as_float(__byte_perm(b, 0x4B000000u, 0x7441))), off);
+    hi = fadd2(pk2(__uint_as_float(__byte_perm(b, 0x4B000000u, 0x7442)),
+                   __uint_as_float(__byte_perm(b, 0x4B000000u, 0x7443))), off);
 }
 
-template <int ESZ>
-__device__ __forceinline__ float fma_word(uint32_t w, const float *x, float acc)
-{
-    if constexpr (ESZ == 2) {
-        acc = fmaf(__uint_as_float(w << 16), x[0], acc);
-        acc = fmaf(__uint_as_float(w & 0xffff0000u), x[1], acc);
-    } else {
-        const uint32_t b = w ^ 0x80808080u;
-        acc = fmaf(i8f(b, 0x7440), x[0], acc);
-        acc = fmaf(i8f(b, 0x7441), x[1], acc);
-        acc = fmaf(i8f(b, 0x7442), x[2], acc);
-        acc = fmaf(i8f(b, 0x7443), x[3], acc);
-    }
-    return acc;
-}
+// A weight vector of VB bytes held in registers.
+template <int VB> struct WVec;
+template <> struct WVec<16> { uint32_t w[4]; };
+template <> struct WVec<8> { uint32_t w[2]; };
+template <> struct WVec<4> { uint32_t w[1]; };
 
-template <int ESZ, int VB>
-__device__ __forceinline__ float vdot(const uint8_t *p, const float *x, float acc)
+template <int VB>
+__device__ __forceinline__ WVec<VB> ldw(uint32_t a)
 {
-    constexpr int EW = 4 / ESZ;  // elements per 32-bit word
+    WVec<VB> v;
     if constexpr (VB == 16) {
-        const uint4 w = *reinterpret_cast<const uint4 *>(p);
-        acc = fma_word<ESZ>(w.x, x, acc);
-        acc = fma_word<ESZ>(w.y, x + EW, acc);
-        acc = fma_word<ESZ>(w.z, x + 2 * EW, acc);
-        acc = fma_word<ESZ>(w.w, x + 3 * EW, acc);
+        const uint4 t = lds128(a);
+        v.w[0] = t.x;
+        v.w[1] = t.y;
+        v.w[2] = t.z;
+        v.w[3] = t.w;
     } else if constexpr (VB == 8) {
-        const uint2 w = *reinterpret_cast<const uint2 *>(p);
-        acc = fma_word<ESZ>(w.x, x, acc);
-        acc = fma_word<ESZ>(w.y, x + EW, acc);
+        const uint2 t = lds64(a);
+        v.w[0] = t.x;
+        v.w[1] = t.y;
     } else {
-        acc = fma_word<ESZ>(*reinterpret_cast<const uint32_t *>(p), x, acc);
+        v.w[0] = lds32(a);
+    }
+    return v;
+}
+
+// acc += (weights of v) . x over packed pairs; x holds VB/ESZ/2 float pairs
+template <int ESZ, int VB>
+__device__ __forceinline__ f2_t vdot2(const WVec<VB> &v, const f2_t *x, f2_t acc)
+{
+#pragma unroll
+    for (int i = 0; i < VB / 4; ++i) {
+        if constexpr (ESZ == 2) {
+            acc = ffma2(bf2(v.w[i]), x[i], acc);
+        } else {
+            f2_t lo, hi;
+            i8x4(v.w[i], lo, hi);
+            acc = ffma2(lo, x[2 * i], acc);
+            acc = ffma2(hi, x[2 * i + 1], acc);
+        }
     }
     return acc;
 }
@@ -183,8 +279,11 @@ struct SmemLayout {
     float *red;           // [kConsumerWarps][kMaxTaskRows]
     uint64_t *full;       // [kMaxStages]
     uint64_t *empty;      // [kMaxStages]
-    int *flags;           // [0] abort, [1] token, [2..] scratch
+    int *flags;           // [0] abort
     float *scr;           // 64 floats of reduction scratch
+    unsigned long long *wacc;  // [2] per-task sums over warps (profiling)
+    uint32_t ring_a, vec_a, red_a, full_a, empty_a;  // shared addresses
+    uint32_t ptask_a, ctask_a;  // [2] staged task records of producer / consumers
 };
 
 __device__ __forceinline__ SmemLayout smem_layout(uint8_t *base, const KParams &p)
@@ -204,21 +303,57 @@ __device__ __forceinline__ SmemLayout smem_layout(uint8_t *base, const KParams &
     s.flags = reinterpret_cast<int *>(base + off);
     off += 16 * 4;
     s.scr = reinterpret_cast<float *>(base + off);
+    off += 64 * 4;
+    s.wacc = reinterpret_cast<unsigned long long *>(base + off);
+    off += 16;
+    s.ptask_a = smem_u32(base + off);
+    off += 2 * sizeof(TaskDesc);
+    s.ctask_a = smem_u32(base + off);
+    s.ring_a = smem_u32(s.ring);
+    s.vec_a = smem_u32(s.vec);
+    s.red_a = smem_u32(s.red);
+    s.full_a = smem_u32(s.full);
+    s.empty_a = smem_u32(s.empty);
     return s;
+}
+
+// Copies a task record into a shared-memory slot asynchronously (cp.async,
+// five 16-byte pieces, one commit group), holding no registers; the issuing
+// thread waits for it with stage_task_wait before anyone reads the slot.
+__device__ __forceinline__ void stage_task(uint32_t slot, const TaskDesc *t)
+{
+    const uint8_t *src = reinterpret_cast<const uint8_t *>(t);
+#pragma unroll
+    for (int i = 0; i < 5; ++i)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(slot + 16 * i),
+                     "l"(src + 16 * i)
+                     : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void stage_task_wait()
+{
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ TaskDesc read_staged(uint32_t slot)
+{
+    TaskDesc d;
+    uint4 *dst = reinterpret_cast<uint4 *>(&d);
+#pragma unroll
+    for (int i = 0; i < 5; ++i)
+        dst[i] = lds128(slot + 16 * i);
+    return d;
 }
 
 // ------------------------------------------------------------- task geometry
 // Both the producer and the consumers derive a task's chunk stream from its
-// descriptor with this function, so they agree on every chunk.
+// record with this function (no memory reads), so they agree on every chunk.
 struct Geom {
     int nchunks;
     // GEMV tiles
-    const uint8_t *base0, *base1;  // row r0 of part 0 / part 1
-    const uint16_t *scale0, *scale1;
     int K, esz, RB, rpc, R, nck;
+    int VB, KS, RG;  // vector bytes; warps split K into KS slices x RG row groups
     // attention tiles
     int j0, j1, pa, pb, P;
-    const uint8_t *kb, *vb;
 };
 
 __device__ __forceinline__ int gcd16(int v)
@@ -229,13 +364,11 @@ __device__ __forceinline__ int gcd16(int v)
     return g;
 }
 
-__device__ Geom task_geom(const KParams &p, const TaskDesc &d)
+__device__ __forceinline__ Geom task_geom(const KParams &p, const TaskDesc &d)
 {
     Geom g{};
-    const int l = d.layer;
-    const int q8 = p.quant;
     if (d.kind == TK_ATTN) {
-        const int gi = d.r0, c = d.r1, hd = p.head_dim;
+        const int c = d.r1, hd = p.head_dim;
         const int n = p.pos + 1;
         const int chunk = (n + p.attn_splits - 1) / p.attn_splits;
         g.j0 = c * chunk;
@@ -245,70 +378,48 @@ __device__ Geom task_geom(const KParams &p, const TaskDesc &d)
         g.pa = g.j0;
         g.pb = max(g.pa, min(g.j1, p.pos));
         g.P = p.stage_bytes / (4 * hd);
-        const size_t blk = (size_t)p.max_ctx * hd;
-        const uint16_t *kbase = p.kv + (((size_t)l * 2 + 0) * p.n_kv_heads + gi) * blk;
-        const uint16_t *vbase = p.kv + (((size_t)l * 2 + 1) * p.n_kv_heads + gi) * blk;
-        g.kb = reinterpret_cast<const uint8_t *>(kbase);
-        g.vb = reinterpret_cast<const uint8_t *>(vbase);
         g.nchunks = (g.pb - g.pa + g.P - 1) / g.P;
         return g;
     }
-    const LayerPtrs *L = (d.kind == TK_LMHEAD) ? nullptr : &p.layers[l];
-    const void *w0 = nullptr, *w1 = nullptr;
-    const uint16_t *s0 = nullptr, *s1 = nullptr;
-    int K = p.hidden, esz = q8 ? 1 : 2, parts = 1;
-    switch (d.kind) {
-    case TK_QKV:
-        w0 = L->w[d.mat];
-        s0 = L->s[d.mat];
-        break;
-    case TK_OPROJ:
-        w0 = L->w[W_O];
-        s0 = L->s[W_O];
+    int K = p.hidden, esz = p.quant ? 1 : 2, parts = 1;
+    if (d.kind == TK_OPROJ)
         K = p.n_heads * p.head_dim;
-        break;
-    case TK_GATEUP:
-        w0 = L->w[W_GATE];
-        s0 = L->s[W_GATE];
-        w1 = L->w[W_UP];
-        s1 = L->s[W_UP];
-        parts = 2;
-        break;
-    case TK_DOWN:
-        w0 = L->w[W_DOWN];
-        s0 = L->s[W_DOWN];
+    else if (d.kind == TK_DOWN)
         K = p.ffn;
-        break;
-    default:  // TK_LMHEAD
-        if (p.tied) {
-            w0 = p.embed;
-            esz = 2;
-        } else {
-            w0 = p.lm_head;
-            s0 = p.lm_head_scale;
-        }
-        break;
-    }
+    else if (d.kind == TK_GATEUP)
+        parts = 2;
+    else if (d.kind == TK_LMHEAD && p.tied)
+        esz = 2;
     g.K = K;
     g.esz = esz;
     g.RB = K * esz;
     const int gran = 16 / gcd16(g.RB);
     int rpc = p.stage_bytes / g.RB;
     rpc -= rpc % gran;
+    // warp layout: each lane keeps at most 64 activations of its K-slice in
+    // registers; split K across more warps only when a row needs it, so that
+    // every warp reduces whole rows with as few shuffles as possible
+    g.VB = (g.RB % 16 == 0) ? 16 : ((g.RB % 8 == 0) ? 8 : 4);
+    const int NV = g.RB / g.VB;
+    const int max_vec = 64 / (g.VB / esz);  // vectors a lane may hold
+    int KS = 1;
+    while (KS < kConsumerWarps && (NV > KS * 32 * max_vec || kConsumerWarps / KS > rpc))
+        KS *= 2;
+    g.KS = KS;
+    g.RG = kConsumerWarps / KS;
+    const int step = g.RG > gran ? g.RG : gran;  // rows per chunk: a multiple of both
+    if (rpc >= step)
+        rpc -= rpc % step;
     g.rpc = rpc;
     g.R = d.r1 - d.r0;
     g.nck = (g.R + rpc - 1) / rpc;
     g.nchunks = g.nck * parts;
-    g.base0 = static_cast<const uint8_t *>(w0) + (size_t)d.r0 * g.RB;
-    g.base1 = w1 ? static_cast<const uint8_t *>(w1) + (size_t)d.r0 * g.RB : nullptr;
-    g.scale0 = s0 ? s0 + d.r0 : nullptr;
-    g.scale1 = s1 ? s1 + d.r0 : nullptr;
     return g;
 }
 
 // ------------------------------------------------------------------ producer
-// Lane 0 of the producer warp streams every chunk of every task of this SM's
-// queue into the ring.  Returns the number of chunks issued.
+// Lane 0 of the producer warpgroup streams every chunk of every task of this
+// SM's queue into the ring, one task record ahead.
 __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int qe)
 {
     const uint64_t pol_w = evict_first_policy();  // weights: streamed once per step
@@ -316,16 +427,26 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
     uint32_t k = 0;  // chunks issued
     volatile int *abort_flag = s.flags;
     bool stop = false;
+    uint64_t prof_wait = 0, prof_bytes = 0, prof_setup = 0;
+    if (qb < qe)
+        stage_task(s.ptask_a, p.tasks + qb);
     for (int ti = qb; ti < qe && !stop; ++ti) {
-        const TaskDesc d = p.tasks[ti];
+        const uint64_t ts = p.prof ? gtimer() : 0;
+        const uint64_t wait_before = prof_wait;
+        stage_task_wait();
+        const TaskDesc d = read_staged(s.ptask_a + ((ti - qb) & 1) * sizeof(TaskDesc));
+        if (ti + 1 < qe)  // the next record streams in while this task's chunks issue
+            stage_task(s.ptask_a + ((ti + 1 - qb) & 1) * sizeof(TaskDesc), p.tasks + ti + 1);
         const Geom g = task_geom(p, d);
+        const uint8_t *w0 = static_cast<const uint8_t *>(d.w0);
+        const uint8_t *w1 = static_cast<const uint8_t *>(d.w1);
         for (int i = 0; i < g.nchunks; ++i, ++k) {
             const int st = k % NS;
             if (k >= (uint32_t)NS) {
                 const uint32_t par = ((k / NS) - 1) & 1;
                 uint32_t it = 0;
                 uint64_t t0 = 0;
-                while (!mbar_try_wait(&s.empty[st], par)) {
+                while (!mbar_try_wait(s.empty_a + 8 * st, par)) {
                     if (it == 0)
                         t0 = gtimer();
                     if ((++it & 255) == 0) {
@@ -338,26 +459,39 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
                 }
                 if (stop)
                     break;
+                if (p.prof && it)
+                    prof_wait += gtimer() - t0;
             }
-            uint8_t *dst = s.ring + (size_t)st * p.stage_bytes;
+            const uint32_t dst = s.ring_a + (uint32_t)st * p.stage_bytes;
+            const uint32_t bar = s.full_a + 8 * st;
+            if (p.prof && i == 0)  // time from the task's start to its first copy
+                prof_setup += (gtimer() - ts) - (prof_wait - wait_before);
             if (d.kind == TK_ATTN) {
                 const int a = g.pa + i * g.P;
                 const int b = min(a + g.P, g.pb);
                 const uint32_t nb = (uint32_t)(b - a) * p.head_dim * 2;
-                mbar_arrive_expect_tx(&s.full[st], 2 * nb);
-                bulk_g2s_nohint(dst, g.kb + (size_t)a * p.head_dim * 2, nb, &s.full[st]);
-                bulk_g2s_nohint(dst + (size_t)g.P * p.head_dim * 2,
-                                g.vb + (size_t)a * p.head_dim * 2, nb, &s.full[st]);
+                mbar_arrive_expect_tx(bar, 2 * nb);
+                bulk_g2s_nohint(dst, w0 + (size_t)a * p.head_dim * 2, nb, bar);
+                bulk_g2s_nohint(dst + (uint32_t)g.P * p.head_dim * 2,
+                                w1 + (size_t)a * p.head_dim * 2, nb, bar);
+                prof_bytes += 2 * nb;
             } else {
                 const int part = i / g.nck, c = i % g.nck;
                 const int r = c * g.rpc;
                 const int nr = min(g.rpc, g.R - r);
                 const uint32_t nb = (uint32_t)nr * g.RB;
-                const uint8_t *src = (part ? g.base1 : g.base0) + (size_t)r * g.RB;
-                mbar_arrive_expect_tx(&s.full[st], nb);
-                bulk_g2s(dst, src, nb, &s.full[st], pol_w);
+                mbar_arrive_expect_tx(bar, nb);
+                bulk_g2s(dst, (part ? w1 : w0) + (size_t)r * g.RB, nb, bar, pol_w);
+                prof_bytes += nb;
             }
         }
+    }
+    if (p.prof) {
+        unsigned long long *pc = p.prof + (size_t)blockIdx.x * kProfKinds * kProfFields;
+        pc[2] = prof_wait;
+        pc[3] = gtimer();
+        pc[4] = prof_bytes;
+        pc[5] = prof_setup;
     }
     // Drain: wait (bounded) for the copies still in flight so that no bulk
     // copy writes into shared memory after this CTA has exited.
@@ -367,7 +501,7 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
         const uint32_t par = (j / NS) & 1;
         uint32_t it = 0;
         const uint64_t t1 = gtimer();
-        while (!mbar_try_wait(&s.full[st], par)) {
+        while (!mbar_try_wait(s.full_a + 8 * st, par)) {
             if ((++it & 255) == 0 && (gtimer() - t1 > p.timeout_ns || it > (1u << 30)))
                 break;
         }
@@ -375,12 +509,8 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
 }
 
 // ------------------------------------------------------------------ consumers
-struct CState {
-    uint32_t k;      // chunks consumed
-    bool aborted;
-};
-
-// Waits (all lanes of a warp together) until ring stage for chunk k is full.
+// Waits (all lanes of a warp together) until the ring stage of chunk k is full.
+// All lanes of a warp poll the barrier together (one SIMT instruction).
 __device__ __forceinline__ bool wait_full(const KParams &p, const SmemLayout &s, uint32_t k)
 {
     const int st = k % p.ring_stages;
@@ -389,7 +519,7 @@ __device__ __forceinline__ bool wait_full(const KParams &p, const SmemLayout &s,
     uint32_t it = 0;
     uint64_t t0 = 0;
     while (true) {
-        const bool ok = mbar_try_wait(&s.full[st], par);
+        const bool ok = mbar_try_wait(s.full_a + 8 * st, par);
         if (__all_sync(0xffffffffu, ok))
             return true;
         if (it == 0)
@@ -408,7 +538,7 @@ __device__ __forceinline__ void release_stage(const KParams &p, const SmemLayout
 {
     __syncwarp();
     if (lane == 0)
-        mbar_arrive(&s.empty[k % p.ring_stages]);
+        mbar_arrive(s.empty_a + 8 * (k % p.ring_stages));
 }
 
 __device__ void record_error(const KParams &p, uint32_t code, int task, int ctr, uint32_t seen,
@@ -431,12 +561,14 @@ __device__ bool wait_counter(const KParams &p, const TaskDesc &d, int ti)
         return true;
     const uint32_t target = p.epoch * d.wait_total + d.wait_count;
     const uint32_t *ctr = p.counters + d.wait_ctr;
-    const uint64_t t0 = gtimer();
+    uint64_t t0 = 0;
     uint32_t v = 0;
     for (uint32_t it = 0;; ++it) {
         v = ld_acquire(ctr);
         if ((int32_t)(v - target) >= 0)
             return true;
+        if (it == 0)
+            t0 = gtimer();
         if ((it & 31) == 31) {
             if (ld_relaxed(&p.err->code) != 0u)
                 return false;
@@ -449,11 +581,11 @@ __device__ bool wait_counter(const KParams &p, const TaskDesc &d, int ti)
 }
 
 // Block-wide sum over the 256 consumer threads (uses s.scr).
-__device__ float block_sum(float v, const SmemLayout &s, int tid)
+__device__ float block_sum(float v, const SmemLayout &s, int ct)
 {
     v = warp_sum(v);
-    if ((tid & 31) == 0)
-        s.scr[tid >> 5] = v;
+    if ((ct & 31) == 0)
+        s.scr[ct >> 5] = v;
     consumer_bar();
     float t = 0.f;
 #pragma unroll
@@ -464,117 +596,183 @@ __device__ float block_sum(float v, const SmemLayout &s, int tid)
 }
 
 // vec[i] = g_i * x_i / sqrt(mean x^2 + eps), x from L2 (fp32) or the
-// embedding row (bf16).
+// embedding row (bf16).  Every load of a thread is issued before any store
+// (one L2 round trip); hidden <= kMaxPerThread * 256.
+constexpr int kMaxPerThread = 16;
 __device__ void rmsnorm_prologue(const KParams &p, const SmemLayout &s, const float *x_f32,
-                                 const uint16_t *x_bf16, const uint16_t *gain, int tid)
+                                 const uint16_t *x_bf16, const uint16_t *gain, int ct)
 {
     const int n = p.hidden;
-    float ss = 0.f;
-    for (int i = tid; i < n; i += kConsumerThreads) {
-        const float v = x_f32 ? __ldcg(x_f32 + i) : bf16_to_f(__ldg(x_bf16 + i));
-        s.vec[i] = v;
-        ss = fmaf(v, v, ss);
+    float xv[kMaxPerThread], gv[kMaxPerThread];
+#pragma unroll
+    for (int j = 0; j < kMaxPerThread; ++j) {
+        const int i = ct + j * kConsumerThreads;
+        xv[j] = 0.f;
+        gv[j] = 0.f;
+        if (i < n) {
+            xv[j] = x_f32 ? __ldcg(x_f32 + i) : bf16_to_f(__ldg(x_bf16 + i));
+            gv[j] = bf16_to_f(__ldg(gain + i));
+        }
     }
-    const float tot = block_sum(ss, s, tid);
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxPerThread; ++j)
+        ss = fmaf(xv[j], xv[j], ss);
+    const float tot = block_sum(ss, s, ct);
     const float inv = rsqrtf(tot / (float)n + p.rms_eps);
-    for (int i = tid; i < n; i += kConsumerThreads)
-        s.vec[i] = bf16_to_f(__ldg(gain + i)) * (s.vec[i] * inv);
+#pragma unroll
+    for (int j = 0; j < kMaxPerThread; ++j) {
+        const int i = ct + j * kConsumerThreads;
+        if (i < n)
+            s.vec[i] = gv[j] * (xv[j] * inv);
+    }
     consumer_bar();
 }
 
-// GEMV over a task's chunks.  Each warp owns vectors [vb, ve) of every row;
-// lane l handles vb + l + 32 i.  Per-warp row sums go to red[w][row].
+// GEMV over a task's chunks.  Warp w = rg + RG * ks owns K-slice ks (vectors
+// [vb, ve) of every row, lane l holding vb + l + 32 i with its activations in
+// registers as float pairs) of the rows j = rg, rg + RG, ... of each chunk,
+// two rows at a time, and writes the slice's row sum to red[w][row]; the
+// epilogue adds the KS slices of a row.  The activations come from the
+// shared vector (prologue output) or, when xg is set, straight from L2.
 template <int ESZ, int VB>
-__device__ bool gemv_task(const KParams &p, const SmemLayout &s, const Geom &g, CState &cs,
-                          int warp, int lane)
+__device__ __forceinline__ bool gemv_task(const KParams &p, const SmemLayout &s, const Geom g,
+                                          uint32_t &kc, int warp, int lane, const float *xg,
+                                          uint64_t *wt)
 {
-    constexpr int E = VB / ESZ;
-    constexpr int NI = 48 / E;
+    constexpr int E = VB / ESZ;   // elements per vector (even)
+    constexpr int NI = 64 / E;    // vectors per lane at most (64 activations)
+    constexpr int EP = E / 2;     // float pairs per vector
     const int NV = g.RB / VB;
-    const int VPW = (NV + kConsumerWarps - 1) / kConsumerWarps;
-    const int vb = warp * VPW;
-    const int ve = min(vb + VPW, NV);
-    float xr[NI][E];
+    const int VPS = (NV + g.KS - 1) / g.KS;
+    const int RG = g.RG, RB = g.RB, rpc = g.rpc, R = g.R, nck = g.nck;
+    const int rg = warp % RG, ks = warp / RG;
+    const int vb = ks * VPS;
+    const int ve = min(vb + VPS, NV);
+    const int ni = (ve - vb - lane + 31) / 32;  // vectors this lane holds (may be <= 0)
+    f2_t xp[NI][EP];
 #pragma unroll
     for (int i = 0; i < NI; ++i) {
         const int v = vb + lane + 32 * i;
 #pragma unroll
-        for (int e = 0; e < E; ++e)
-            xr[i][e] = (v < ve) ? s.vec[v * E + e] : 0.f;
-    }
-    float *red = s.red + warp * kMaxTaskRows;
-    for (int i = 0; i < g.nchunks; ++i) {
-        if (!wait_full(p, s, cs.k))
-            return false;
-        const uint8_t *stage = s.ring + (size_t)(cs.k % p.ring_stages) * p.stage_bytes;
-        const int part = i / g.nck, c = i % g.nck;
-        const int r = c * g.rpc;
-        const int nr = min(g.rpc, g.R - r);
-        const int rowbase = part * g.R + r;
-        int j = 0;
-        for (; j + 1 < nr; j += 2) {
-            const uint8_t *row0 = stage + (size_t)j * g.RB;
-            const uint8_t *row1 = row0 + g.RB;
-            float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-            for (int t = 0; t < NI; ++t) {
-                const int v = vb + lane + 32 * t;
-                if (v < ve) {
-                    a0 = vdot<ESZ, VB>(row0 + (size_t)v * VB, xr[t], a0);
-                    a1 = vdot<ESZ, VB>(row1 + (size_t)v * VB, xr[t], a1);
+        for (int e = 0; e < E; e += 2) {
+            float a = 0.f, b = 0.f;
+            if (i < ni) {
+                if (xg) {
+                    const float2 t = __ldcg(reinterpret_cast<const float2 *>(xg + v * E + e));
+                    a = t.x;
+                    b = t.y;
+                } else {
+                    const uint2 t = lds64(s.vec_a + (uint32_t)(v * E + e) * 4);
+                    a = __uint_as_float(t.x);
+                    b = __uint_as_float(t.y);
                 }
             }
-            a0 = warp_sum(a0);
-            a1 = warp_sum(a1);
-            if (lane == 0) {
-                red[rowbase + j] = a0;
-                red[rowbase + j + 1] = a1;
-            }
+            xp[i][e / 2] = pk2(a, b);
         }
-        if (j < nr) {
-            const uint8_t *row0 = stage + (size_t)j * g.RB;
-            float a0 = 0.f;
+    }
+    const uint32_t red_a = s.red_a + (uint32_t)warp * kMaxTaskRows * 4;
+    const int NS = p.ring_stages, SB = p.stage_bytes;
+    uint64_t tA = 0, tB = 0;
+    for (int i = 0; i < g.nchunks; ++i) {
+        if (wt)
+            tA = gtimer();
+        if (!wait_full(p, s, kc))
+            return false;
+        if (wt) {
+            tB = gtimer();
+            wt[0] += tB - tA;
+        }
+        const uint32_t stage_a = s.ring_a + (uint32_t)(kc % NS) * SB;
+        const int part = i / nck, c = i - part * nck;
+        const int r = c * rpc;
+        const int nr = min(rpc, R - r);
+        const int rowbase = part * R + r;
+        const uint32_t lane_a = stage_a + (uint32_t)(vb + lane) * VB;
+        // bf16 interleaves two rows per warp (two reduction chains); int8
+        // needs the registers for unpacking and takes one row at a time
+        constexpr int ROWS = (ESZ == 2) ? 2 : 1;
+        for (int j = rg; j < nr; j += ROWS * RG) {
+            const bool two = ROWS == 2 && j + RG < nr;
+            const uint32_t ra = lane_a + (uint32_t)j * RB;
+            const uint32_t rb = ra + (uint32_t)RG * RB;
+            f2_t acc_a[4] = {0ull, 0ull, 0ull, 0ull}, acc_b[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-            for (int t = 0; t < NI; ++t) {
-                const int v = vb + lane + 32 * t;
-                if (v < ve)
-                    a0 = vdot<ESZ, VB>(row0 + (size_t)v * VB, xr[t], a0);
+            for (int t0 = 0; t0 < NI; t0 += 4) {
+                WVec<VB> wa[4], wb[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (t0 + u < NI && t0 + u < ni) {
+                        wa[u] = ldw<VB>(ra + (uint32_t)(t0 + u) * 32 * VB);
+                        if (two)
+                            wb[u] = ldw<VB>(rb + (uint32_t)(t0 + u) * 32 * VB);
+                    }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (t0 + u < NI && t0 + u < ni) {
+                        acc_a[u] = vdot2<ESZ, VB>(wa[u], xp[t0 + u], acc_a[u]);
+                        if (two)
+                            acc_b[u] = vdot2<ESZ, VB>(wb[u], xp[t0 + u], acc_b[u]);
+                    }
             }
-            a0 = warp_sum(a0);
-            if (lane == 0)
-                red[rowbase + j] = a0;
+            float sa = (sum2(acc_a[0]) + sum2(acc_a[1])) + (sum2(acc_a[2]) + sum2(acc_a[3]));
+            float sb = (sum2(acc_b[0]) + sum2(acc_b[1])) + (sum2(acc_b[2]) + sum2(acc_b[3]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                sa += __shfl_xor_sync(0xffffffffu, sa, o);
+                sb += __shfl_xor_sync(0xffffffffu, sb, o);
+            }
+            if (lane == 0) {
+                stsf(red_a + (uint32_t)(rowbase + j) * 4, sa);
+                if (two)
+                    stsf(red_a + (uint32_t)(rowbase + j + RG) * 4, sb);
+            }
         }
-        release_stage(p, s, cs.k, lane);
-        ++cs.k;
+        release_stage(p, s, kc, lane);
+        ++kc;
+        if (wt)
+            wt[1] += gtimer() - tB;
     }
     return true;
 }
 
-__device__ bool run_gemv(const KParams &p, const SmemLayout &s, const Geom &g, CState &cs,
-                         int warp, int lane)
+// Fast instances (GENERIC = 0) only run 16-byte weight vectors in the
+// model's own format; the generic instance dispatches every variant at run
+// time (models with odd row widths, or a bf16 tied head on int8 layers).
+template <int Q8, int GENERIC>
+__device__ __forceinline__ bool run_gemv(const KParams &p, const SmemLayout &s, const Geom &g,
+                                         uint32_t &kc, int warp, int lane, const float *xg,
+                                         uint64_t *wt)
 {
-    const int vbytes = (g.RB % 16 == 0) ? 16 : ((g.RB % 8 == 0) ? 8 : 4);
-    if (g.esz == 2) {
-        if (vbytes == 16)
-            return gemv_task<2, 16>(p, s, g, cs, warp, lane);
-        if (vbytes == 8)
-            return gemv_task<2, 8>(p, s, g, cs, warp, lane);
-        return gemv_task<2, 4>(p, s, g, cs, warp, lane);
+    if constexpr (!GENERIC) {
+        if constexpr (Q8)
+            return gemv_task<1, 16>(p, s, g, kc, warp, lane, xg, wt);
+        else
+            return gemv_task<2, 16>(p, s, g, kc, warp, lane, xg, wt);
+    } else {
+        if (g.esz == 2) {
+            if (g.VB == 16)
+                return gemv_task<2, 16>(p, s, g, kc, warp, lane, xg, wt);
+            if (g.VB == 8)
+                return gemv_task<2, 8>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv_task<2, 4>(p, s, g, kc, warp, lane, xg, wt);
+        }
+        if (g.VB == 16)
+            return gemv_task<1, 16>(p, s, g, kc, warp, lane, xg, wt);
+        if (g.VB == 8)
+            return gemv_task<1, 8>(p, s, g, kc, warp, lane, xg, wt);
+        return gemv_task<1, 4>(p, s, g, kc, warp, lane, xg, wt);
     }
-    if (vbytes == 16)
-        return gemv_task<1, 16>(p, s, g, cs, warp, lane);
-    if (vbytes == 8)
-        return gemv_task<1, 8>(p, s, g, cs, warp, lane);
-    return gemv_task<1, 4>(p, s, g, cs, warp, lane);
 }
 
-// Row sum over the 8 warps' partials for output row t of the task.
-__device__ __forceinline__ float row_total(const SmemLayout &s, int t)
+// Sum of the K-slice partials of output row t (task-relative, parts
+// included): the warps rg + RG * ks with rg = (row within its chunk) % RG.
+__device__ __forceinline__ float row_total(const SmemLayout &s, const Geom &g, int t)
 {
+    const int rg = (t % g.R) % g.RG;  // chunks start at multiples of RG
     float y = 0.f;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w)
-        y += s.red[w * kMaxTaskRows + t];
+    for (int ks = 0; ks < g.KS; ++ks)
+        y += s.red[(rg + g.RG * ks) * kMaxTaskRows + t];
     return y;
 }
 
@@ -583,30 +781,59 @@ __device__ __forceinline__ float row_scale(const uint16_t *scale, int t)
     return scale ? fp16_to_f(__ldg(scale + t)) : 1.f;
 }
 
-// RoPE (HF rotate_half) on a head vector in shared memory at position pos;
-// angles in double precision: a = pos * theta^(-2i/hd).
-__device__ void rope_smem(float *v, int hd, int pos, float theta, int i)
+// RoPE angle of pair i at position pos (HF rotate_half): a = pos * w_i with
+// w_i = theta^(-2i/hd), formed and reduced modulo 2*pi in double precision,
+// then sin/cos of the reduced angle in single precision.
+__device__ __forceinline__ void rope_angle(int pos, int i, int hd, float theta, float *sn,
+                                           float *cs)
 {
-    const int half = hd / 2;
-    if (i < half) {
-        const double w = exp2(-(2.0 * i / hd) * log2((double)theta));
-        double sn, cs;
-        sincos((double)pos * w, &sn, &cs);
-        const float c = (float)cs, sgn = (float)sn;
-        const float x0 = v[i], x1 = v[i + half];
-        v[i] = x0 * c - x1 * sgn;
-        v[i + half] = x1 * c + x0 * sgn;
+    const double w = exp2(-(2.0 * i / hd) * log2((double)theta));
+    const double a = (double)pos * w;
+    const double k = rint(a * 0.15915494309189535);  // a / (2 pi)
+    const double r = fma(-k, 6.283185307179586, a);  // a - 2 pi k (|k| small)
+    sincosf((float)r, sn, cs);
+}
+
+// E consecutive bf16 values at shared address a (2E-byte aligned) as floats.
+template <int E>
+__device__ __forceinline__ void lds_bf16(uint32_t a, float (&out)[E])
+{
+    if constexpr (E == 1) {
+        out[0] = __uint_as_float(lds16(a) << 16);
+    } else if constexpr (E == 2) {
+        const uint32_t w = lds32(a);
+        out[0] = __uint_as_float(w << 16);
+        out[1] = __uint_as_float(w & 0xffff0000u);
+    } else if constexpr (E == 4) {
+        const uint2 w = lds64(a);
+        out[0] = __uint_as_float(w.x << 16);
+        out[1] = __uint_as_float(w.x & 0xffff0000u);
+        out[2] = __uint_as_float(w.y << 16);
+        out[3] = __uint_as_float(w.y & 0xffff0000u);
+    } else {
+#pragma unroll
+        for (int c = 0; c < E / 8; ++c) {
+            const uint4 w = lds128(a + c * 16);
+            const uint32_t ws_[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                out[c * 8 + 2 * i] = __uint_as_float(ws_[i] << 16);
+                out[c * 8 + 2 * i + 1] = __uint_as_float(ws_[i] & 0xffff0000u);
+            }
+        }
     }
 }
 
 // Split-K attention tile for KV head g and chunk c (flash-decoding partial):
 // writes (m, l, o[hd]) per query head of the group, unnormalised.
-__device__ bool attn_task(const KParams &p, const SmemLayout &s, const TaskDesc &d,
-                          const Geom &g, CState &cs, int tid, int warp, int lane)
+template <int E>
+__device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
+                                          const TaskDesc &d, const Geom &g, uint32_t &kc,
+                                          int ct, int warp, int lane, uint64_t *wt)
 {
     const int l = d.layer, gi = d.r0, c = d.r1;
     const int hd = p.head_dim, G = p.group, nh = p.n_heads, nkv = p.n_kv_heads;
-    const int lph = p.att_lph, E = p.att_e;
+    const int lph = p.att_lph;
     float *qs = s.vec;                       // [G][hd], RoPE'd and pre-scaled
     float *kn = qs + G * hd;                 // [hd] new K row (bf16 value)
     float *vn = kn + hd;                     // [hd] new V row (bf16 value)
@@ -614,31 +841,41 @@ __device__ bool attn_task(const KParams &p, const SmemLayout &s, const TaskDesc 
     const float *qkv = p.qkv + (size_t)l * p.qkv_rows;
     if (g.j1 <= g.j0)
         return true;  // empty chunk: nothing to write, the combine skips it
-    // prologue: load q (G heads), k, v of this KV head; RoPE q and k
-    for (int i = tid; i < G * hd; i += kConsumerThreads)
-        qs[i] = __ldcg(qkv + (size_t)gi * G * hd + i);
-    for (int i = tid; i < hd; i += kConsumerThreads) {
-        kn[i] = __ldcg(qkv + (size_t)nh * hd + (size_t)gi * hd + i);
-        vn[i] = __ldcg(qkv + (size_t)(nh + nkv) * hd + (size_t)gi * hd + i);
-    }
-    consumer_bar();
-    for (int i = tid; i < (G + 1) * (hd / 2); i += kConsumerThreads) {
-        const int hh = i / (hd / 2), e = i % (hd / 2);
-        rope_smem(hh < G ? qs + hh * hd : kn, hd, p.pos, p.rope_theta, e);
-    }
-    consumer_bar();
-    const float scale = rsqrtf((float)hd);
-    for (int i = tid; i < G * hd; i += kConsumerThreads)
-        qs[i] *= scale;
-    for (int i = tid; i < hd; i += kConsumerThreads) {
-        const uint16_t kb = f_to_bf16(kn[i]), vb = f_to_bf16(vn[i]);
-        kn[i] = bf16_to_f(kb);
-        vn[i] = bf16_to_f(vb);
-        if (c == 0) {
-            const size_t blk = (size_t)p.max_ctx * hd;
-            p.kv[(((size_t)l * 2 + 0) * nkv + gi) * blk + (size_t)p.pos * hd + i] = kb;
-            p.kv[(((size_t)l * 2 + 1) * nkv + gi) * blk + (size_t)p.pos * hd + i] = vb;
+    // prologue: q of the group's G heads and k get RoPE (pairs i, i + hd/2),
+    // q is pre-scaled by 1/sqrt(hd); k and v are rounded to bf16 (the cache
+    // format) and chunk 0 appends them at row pos
+    const int half = hd / 2;
+    const float qscale = rsqrtf((float)hd);
+    uint16_t *kd = const_cast<uint16_t *>(static_cast<const uint16_t *>(d.w0)) +
+                   (size_t)p.pos * hd;
+    uint16_t *vd = const_cast<uint16_t *>(static_cast<const uint16_t *>(d.w1)) +
+                   (size_t)p.pos * hd;
+    for (int i = ct; i < (G + 1) * half; i += kConsumerThreads) {
+        const int hh = i / half, e = i % half;
+        const float *src = hh < G ? qkv + (size_t)(gi * G + hh) * hd
+                                  : qkv + (size_t)nh * hd + (size_t)gi * hd;
+        const float x0 = __ldcg(src + e), x1 = __ldcg(src + e + half);
+        float sn, cs;
+        rope_angle(p.pos, e, hd, p.rope_theta, &sn, &cs);
+        const float y0 = x0 * cs - x1 * sn, y1 = x1 * cs + x0 * sn;
+        if (hh < G) {
+            qs[hh * hd + e] = y0 * qscale;
+            qs[hh * hd + e + half] = y1 * qscale;
+        } else {
+            const uint16_t b0 = f_to_bf16(y0), b1 = f_to_bf16(y1);
+            kn[e] = bf16_to_f(b0);
+            kn[e + half] = bf16_to_f(b1);
+            if (c == 0) {
+                kd[e] = b0;
+                kd[e + half] = b1;
+            }
         }
+    }
+    for (int i = ct; i < hd; i += kConsumerThreads) {
+        const uint16_t vb = f_to_bf16(__ldcg(qkv + (size_t)(nh + nkv) * hd + (size_t)gi * hd + i));
+        vn[i] = bf16_to_f(vb);
+        if (c == 0)
+            vd[i] = vb;
     }
     consumer_bar();
     // lane layout: head jh = lane / lph (within the group), elements
@@ -646,20 +883,98 @@ __device__ bool attn_task(const KParams &p, const SmemLayout &s, const TaskDesc 
     const int jh = lane / lph;
     const int e0 = (lane % lph) * E;
     const bool active = jh < G;
-    float q[32], o[32];
+    float q[E], o[E];
     float m = -INFINITY, lsum = 0.f;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-        q[e] = (active && e < E) ? qs[jh * hd + e0 + e] : 0.f;
+    for (int e = 0; e < E; ++e) {
+        q[e] = active ? qs[jh * hd + e0 + e] : 0.f;
         o[e] = 0.f;
     }
-    auto visit = [&](const float *krow_f, const uint16_t *krow_b, const float *vrow_f,
-                     const uint16_t *vrow_b) {
+    bool fail = false;
+    uint64_t tA = 0, tB = 0;
+    for (int i = 0; i < g.nchunks; ++i) {
+        if (wt)
+            tA = gtimer();
+        if (!wait_full(p, s, kc)) {
+            fail = true;
+            break;
+        }
+        if (wt) {
+            tB = gtimer();
+            wt[0] += tB - tA;
+        }
+        const uint32_t ka = s.ring_a + (uint32_t)(kc % p.ring_stages) * p.stage_bytes +
+                            (uint32_t)e0 * 2;
+        const uint32_t va = ka + (uint32_t)g.P * hd * 2;
+        const int a = g.pa + i * g.P;
+        const int n = min(g.P, g.pb - a);
+        // four positions per warp at a time: independent dot products and
+        // shuffle reductions, then one online-softmax update
+        for (int j0 = warp; j0 < n; j0 += 4 * kConsumerWarps) {
+            float sc[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int j = j0 + b * kConsumerWarps;
+                float kv_[E];
+                lds_bf16<E>(ka + (uint32_t)(j < n ? j : j0) * hd * 2, kv_);
+                float d_ = 0.f;
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    d_ = fmaf(q[e], kv_[e], d_);
+                sc[b] = d_;
+            }
+            for (int off = lph >> 1; off > 0; off >>= 1) {
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    sc[b] += __shfl_xor_sync(0xffffffffu, sc[b], off);
+            }
+            float mn = m;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                if (j0 + b * kConsumerWarps >= n)
+                    sc[b] = -INFINITY;
+                mn = fmaxf(mn, sc[b]);
+            }
+            const float corr = __expf(m - mn);
+            float pr[4];
+            lsum *= corr;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                pr[b] = __expf(sc[b] - mn);
+                lsum += pr[b];
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                o[e] *= corr;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int j = j0 + b * kConsumerWarps;
+                if (j < n) {
+                    float vv[E];
+                    lds_bf16<E>(va + (uint32_t)j * hd * 2, vv);
+#pragma unroll
+                    for (int e = 0; e < E; ++e)
+                        o[e] = fmaf(pr[b], vv[e], o[e]);
+                }
+            }
+            m = mn;
+        }
+        release_stage(p, s, kc, lane);
+        ++kc;
+        if (wt)
+            wt[1] += gtimer() - tB;
+    }
+    if (fail && lane == 0)
+        s.flags[0] = 1;
+    consumer_bar();
+    if (*reinterpret_cast<volatile int *>(s.flags))
+        return false;
+    if (g.j0 <= p.pos && p.pos < g.j1 && warp == 0) {
+        // the new position: K and V rows of this step (bf16 values as floats)
         float sc = 0.f;
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-            if (e < E)
-                sc = fmaf(q[e], krow_b ? bf16_to_f(krow_b[e0 + e]) : krow_f[e0 + e], sc);
+        for (int e = 0; e < E; ++e)
+            sc = fmaf(q[e], kn[e0 + e], sc);
         for (int off = lph >> 1; off > 0; off >>= 1)
             sc += __shfl_xor_sync(0xffffffffu, sc, off);
         const float mn = fmaxf(m, sc);
@@ -667,41 +982,16 @@ __device__ bool attn_task(const KParams &p, const SmemLayout &s, const TaskDesc 
         const float pr = __expf(sc - mn);
         lsum = lsum * corr + pr;
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-            if (e < E)
-                o[e] = o[e] * corr + pr * (vrow_b ? bf16_to_f(vrow_b[e0 + e]) : vrow_f[e0 + e]);
+        for (int e = 0; e < E; ++e)
+            o[e] = o[e] * corr + pr * vn[e0 + e];
         m = mn;
-    };
-    bool fail = false;
-    for (int i = 0; i < g.nchunks; ++i) {
-        if (!wait_full(p, s, cs.k)) {
-            fail = true;
-            break;
-        }
-        const uint8_t *stage = s.ring + (size_t)(cs.k % p.ring_stages) * p.stage_bytes;
-        const uint16_t *Ks = reinterpret_cast<const uint16_t *>(stage);
-        const uint16_t *Vs = reinterpret_cast<const uint16_t *>(stage + (size_t)g.P * hd * 2);
-        const int a = g.pa + i * g.P;
-        const int n = min(g.P, g.pb - a);
-        for (int j = warp; j < n; j += kConsumerWarps)
-            visit(nullptr, Ks + (size_t)j * hd, nullptr, Vs + (size_t)j * hd);
-        release_stage(p, s, cs.k, lane);
-        ++cs.k;
     }
-    if (fail && lane == 0)
-        s.flags[0] = 1;
-    consumer_bar();
-    if (*reinterpret_cast<volatile int *>(s.flags))
-        return false;
-    if (g.j0 <= p.pos && p.pos < g.j1 && warp == 0)
-        visit(kn, nullptr, vn, nullptr);
     // per-warp state -> ws[w][jh][hd + 2]
     float *mine = ws + (size_t)warp * G * (hd + 2);
     if (active) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-            if (e < E)
-                mine[jh * (hd + 2) + 2 + e0 + e] = o[e];
+        for (int e = 0; e < E; ++e)
+            mine[jh * (hd + 2) + 2 + e0 + e] = o[e];
         if (lane % lph == 0) {
             mine[jh * (hd + 2) + 0] = m;
             mine[jh * (hd + 2) + 1] = lsum;
@@ -709,7 +999,7 @@ __device__ bool attn_task(const KParams &p, const SmemLayout &s, const TaskDesc 
     }
     consumer_bar();
     float *out = p.part + ((((size_t)l * nkv + gi) * p.attn_splits + c) * G) * (hd + 2);
-    for (int i = tid; i < G * hd; i += kConsumerThreads) {
+    for (int i = ct; i < G * hd; i += kConsumerThreads) {
         const int hh = i / hd, e = i % hd;
         float M = -INFINITY;
 #pragma unroll
@@ -733,40 +1023,62 @@ __device__ bool attn_task(const KParams &p, const SmemLayout &s, const TaskDesc 
 }
 
 // O-projection prologue: combine the split-K partials of every head into
-// the attention output vec[h * hd + e] = sum_c w_c o_c[e] / L.
-__device__ void combine_prologue(const KParams &p, const SmemLayout &s, int l, int tid)
+// the attention output vec[h * hd + e] = sum_c e^(m_c - M) o_c[e] / L with
+// M = max_c m_c and L = sum_c e^(m_c - M) l_c.  Per split, every load of a
+// thread is issued before the arithmetic (one L2 round trip per split);
+// n_heads * head_dim <= kMaxPerThread * 256.
+__device__ void combine_prologue(const KParams &p, const SmemLayout &s, int l, int ct)
 {
     const int hd = p.head_dim, nh = p.n_heads, G = p.group, C = p.attn_splits;
     const int n = p.pos + 1;
     const int chunk = (n + C - 1) / C;
     const int nne = (n + chunk - 1) / chunk;  // non-empty splits
-    float *wts = s.vec + (size_t)nh * hd;     // [nh][C]
     const float *part = p.part + (size_t)l * p.n_kv_heads * C * G * (hd + 2);
-    for (int h = tid; h < nh; h += kConsumerThreads) {
-        const int gi = h / G, jh = h % G;
-        float M = -INFINITY;
-        for (int c = 0; c < nne; ++c)
-            M = fmaxf(M, __ldcg(part + (((size_t)gi * C + c) * G + jh) * (hd + 2)));
-        float L = 0.f;
-        for (int c = 0; c < nne; ++c) {
-            const float *pc = part + (((size_t)gi * C + c) * G + jh) * (hd + 2);
-            const float f = __expf(__ldcg(pc) - M);
-            wts[(size_t)h * C + c] = f;
-            L = fmaf(__ldcg(pc + 1), f, L);
+    const int N = nh * hd;
+    const size_t cstride = (size_t)G * (hd + 2);
+    constexpr int B = 8;  // elements per batch of independent loads
+    for (int j0 = 0; j0 < kMaxPerThread; j0 += B) {
+        if (ct + j0 * kConsumerThreads >= N)
+            break;
+        float M[B], L[B], O[B];
+#pragma unroll
+        for (int j = 0; j < B; ++j) {
+            M[j] = -INFINITY;
+            L[j] = 0.f;
+            O[j] = 0.f;
         }
-        const float inv = 1.f / L;
-        for (int c = 0; c < nne; ++c)
-            wts[(size_t)h * C + c] *= inv;
-    }
-    consumer_bar();
-    for (int i = tid; i < nh * hd; i += kConsumerThreads) {
-        const int h = i / hd, e = i % hd;
-        const int gi = h / G, jh = h % G;
-        float acc = 0.f;
-        for (int c = 0; c < nne; ++c)
-            acc = fmaf(wts[(size_t)h * C + c],
-                       __ldcg(part + (((size_t)gi * C + c) * G + jh) * (hd + 2) + 2 + e), acc);
-        s.vec[i] = acc;
+        for (int c = 0; c < nne; ++c) {
+            float2 ml[B];
+            float oc[B];
+#pragma unroll
+            for (int j = 0; j < B; ++j) {
+                const int i = ct + (j0 + j) * kConsumerThreads;
+                if (i < N) {
+                    const int h = i / hd;
+                    const float *pc =
+                        part + ((size_t)(h / G) * C * G + (h % G)) * (hd + 2) + c * cstride;
+                    ml[j] = __ldcg(reinterpret_cast<const float2 *>(pc));
+                    oc[j] = __ldcg(pc + 2 + (i - h * hd));
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < B; ++j) {
+                const int i = ct + (j0 + j) * kConsumerThreads;
+                if (i < N) {
+                    const float Mn = fmaxf(M[j], ml[j].x);
+                    const float a = __expf(M[j] - Mn), b = __expf(ml[j].x - Mn);
+                    L[j] = L[j] * a + ml[j].y * b;
+                    O[j] = O[j] * a + oc[j] * b;
+                    M[j] = Mn;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < B; ++j) {
+            const int i = ct + (j0 + j) * kConsumerThreads;
+            if (i < N)
+                s.vec[i] = O[j] / L[j];
+        }
     }
     consumer_bar();
 }
@@ -793,126 +1105,145 @@ __device__ int resolve_token(const KParams &p)
     return t;
 }
 
-// ------------------------------------------------------------------- kernel
-__global__ void __launch_bounds__(kThreads, 1) amk_decode_kernel(const __grid_constant__ KParams p)
+// ---------------------------------------------------------- consumer loop
+template <int Q8, int ATT_E, int GENERIC>
+__device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout &s, int qb,
+                                              int qe, int ct)
 {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const SmemLayout s = smem_layout(smem_raw, p);
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int qb = p.queue_off[blockIdx.x], qe = p.queue_off[blockIdx.x + 1];
-
-    if (tid == 0) {
-        for (int i = 0; i < p.ring_stages; ++i) {
-            mbar_init(&s.full[i], 1);
-            mbar_init(&s.empty[i], kConsumerWarps);
-        }
-        // a failed earlier step poisons the device state: do no work until the
-        // host resets it (the counters no longer match the epoch)
-        s.flags[0] = ld_relaxed(&p.err->code) != 0u ? 1 : 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
-    __syncthreads();
-    if (s.flags[0])
-        return;
-
-    if (warp == kConsumerWarps) {
-        if (lane == 0)
-            producer_loop(p, s, qb, qe);
-        return;
-    }
-
-    CState cs{0u, false};
+    const int warp = ct >> 5, lane = ct & 31;
+    unsigned long long *prof =
+        (p.prof && ct == 0) ? p.prof + (size_t)blockIdx.x * kProfKinds * kProfFields : nullptr;
+    if (prof)
+        prof[0] = gtimer();
+    const bool wprof = p.prof != nullptr && lane == 0;
+    uint64_t wt_store[2] = {0, 0};
+    uint64_t *wt = wprof ? wt_store : nullptr;
+    uint32_t kc = 0;  // chunks consumed
     int token = -1;
+    if (ct == 0 && qb < qe)
+        stage_task(s.ctask_a, p.tasks + qb);
     for (int ti = qb; ti < qe; ++ti) {
-        const TaskDesc d = p.tasks[ti];
-        if (tid == 0) {
+        const uint32_t slot = s.ctask_a + ((ti - qb) & 1) * sizeof(TaskDesc);
+        if (ct == 0)
+            stage_task_wait();  // record of task ti (issued one task ago)
+        consumer_bar();
+        const TaskDesc d = read_staged(slot);
+        uint64_t t_w0 = 0, t_w1 = 0, t_pro = 0, t_epi = 0;
+        if (prof) {
+            t_w0 = gtimer();
+            s.wacc[0] = s.wacc[1] = 0ull;
+        }
+        if (wprof)
+            wt_store[0] = wt_store[1] = 0;
+        if (ct == 0) {
+            if (ti + 1 < qe)  // the slot read at ti - 1 is free again (barrier above)
+                stage_task(s.ctask_a + ((ti + 1 - qb) & 1) * sizeof(TaskDesc), p.tasks + ti + 1);
             if (!wait_counter(p, d, ti))
                 s.flags[0] = 1;
         }
         consumer_bar();
         if (*reinterpret_cast<volatile int *>(s.flags))
             break;
+        if (prof)
+            t_w1 = gtimer();
         const Geom g = task_geom(p, d);
         const int l = d.layer;
         bool ok = true;
         if (d.kind == TK_ATTN) {
-            ok = attn_task(p, s, d, g, cs, tid, warp, lane);
+            if constexpr (!GENERIC) {
+                ok = attn_task<ATT_E>(p, s, d, g, kc, ct, warp, lane, wt);
+            } else {
+                switch (p.att_e) {
+                case 1: ok = attn_task<1>(p, s, d, g, kc, ct, warp, lane, wt); break;
+                case 2: ok = attn_task<2>(p, s, d, g, kc, ct, warp, lane, wt); break;
+                case 4: ok = attn_task<4>(p, s, d, g, kc, ct, warp, lane, wt); break;
+                case 8: ok = attn_task<8>(p, s, d, g, kc, ct, warp, lane, wt); break;
+                default: ok = attn_task<16>(p, s, d, g, kc, ct, warp, lane, wt); break;
+                }
+            }
+            if (prof)
+                t_pro = t_epi = gtimer();
         } else {
             // prologue -> s.vec
             if (d.kind == TK_QKV) {
                 if (l == 0) {
                     if (token < 0)
                         token = resolve_token(p);
-                    rmsnorm_prologue(p, s, nullptr, p.embed + (size_t)token * p.hidden,
-                                     p.layers[0].attn_norm, tid);
+                    rmsnorm_prologue(p, s, nullptr, p.embed + (size_t)token * p.hidden, d.gain,
+                                     ct);
                 } else {
-                    rmsnorm_prologue(p, s, p.xout + (size_t)(l - 1) * p.hidden, nullptr,
-                                     p.layers[l].attn_norm, tid);
+                    rmsnorm_prologue(p, s, p.xout + (size_t)(l - 1) * p.hidden, nullptr, d.gain,
+                                     ct);
                 }
             } else if (d.kind == TK_OPROJ) {
-                combine_prologue(p, s, l, tid);
+                combine_prologue(p, s, l, ct);
             } else if (d.kind == TK_GATEUP) {
-                rmsnorm_prologue(p, s, p.xmid + (size_t)l * p.hidden, nullptr,
-                                 p.layers[l].ffn_norm, tid);
+                rmsnorm_prologue(p, s, p.xmid + (size_t)l * p.hidden, nullptr, d.gain, ct);
             } else if (d.kind == TK_DOWN) {
-                const float *a = p.act + (size_t)l * p.ffn;
-                for (int i = tid; i < p.ffn; i += kConsumerThreads)
-                    s.vec[i] = __ldcg(a + i);
-                consumer_bar();
+                // no prologue: each warp loads its slice of the SwiGLU
+                // activations from L2 straight into registers
             } else {  // TK_LMHEAD
                 rmsnorm_prologue(p, s, p.xout + (size_t)(p.n_layers - 1) * p.hidden, nullptr,
-                                 p.final_norm, tid);
+                                 d.gain, ct);
             }
-            ok = run_gemv(p, s, g, cs, warp, lane);
+            // residual inputs of the epilogue are ready now: fetch them while
+            // the GEMV runs (thread t owns output row r0 + t; R <= 256)
+            float base = 0.f;
+            if (ct < g.R) {
+                const int r = d.r0 + ct;
+                if (d.kind == TK_OPROJ) {
+                    if (l == 0) {
+                        if (token < 0)
+                            token = resolve_token(p);
+                        base = bf16_to_f(__ldg(p.embed + (size_t)token * p.hidden + r));
+                    } else {
+                        base = __ldcg(p.xout + (size_t)(l - 1) * p.hidden + r);
+                    }
+                } else if (d.kind == TK_DOWN) {
+                    base = __ldcg(p.xmid + (size_t)l * p.hidden + r);
+                }
+            }
+            if (prof)
+                t_pro = gtimer();
+            ok = run_gemv<Q8, GENERIC>(p, s, g, kc, warp, lane,
+                          d.kind == TK_DOWN ? p.act + (size_t)l * p.ffn : nullptr, wt);
             if (!ok && lane == 0) {
                 record_error(p, 2u, ti, -1, 0u, 0u);
                 s.flags[0] = 1;
             }
             consumer_bar();
+            if (prof)
+                t_epi = gtimer();
             ok = *reinterpret_cast<volatile int *>(s.flags) == 0;
             if (ok) {
                 // epilogue: thread t finalises output row r0 + t
+                const uint16_t *s0 = d.s0, *s1 = d.s1;
                 if (d.kind == TK_QKV) {
                     const int off = d.mat == 0 ? 0
                                     : d.mat == 1 ? p.n_heads * p.head_dim
                                                  : (p.n_heads + p.n_kv_heads) * p.head_dim;
                     float *out = p.qkv + (size_t)l * p.qkv_rows + off + d.r0;
-                    for (int t = tid; t < g.R; t += kConsumerThreads)
-                        out[t] = row_total(s, t) * row_scale(g.scale0, t);
+                    for (int t = ct; t < g.R; t += kConsumerThreads)
+                        out[t] = row_total(s, g, t) * row_scale(s0, t);
                 } else if (d.kind == TK_OPROJ) {
-                    for (int t = tid; t < g.R; t += kConsumerThreads) {
-                        const int r = d.r0 + t;
-                        float base;
-                        if (l == 0) {
-                            if (token < 0)
-                                token = resolve_token(p);
-                            base = bf16_to_f(__ldg(p.embed + (size_t)token * p.hidden + r));
-                        } else {
-                            base = __ldcg(p.xout + (size_t)(l - 1) * p.hidden + r);
-                        }
-                        p.xmid[(size_t)l * p.hidden + r] =
-                            base + row_total(s, t) * row_scale(g.scale0, t);
-                    }
+                    if (ct < g.R)
+                        p.xmid[(size_t)l * p.hidden + d.r0 + ct] =
+                            base + row_total(s, g, ct) * row_scale(s0, ct);
                 } else if (d.kind == TK_GATEUP) {
-                    for (int t = tid; t < g.R; t += kConsumerThreads) {
-                        const float gt = row_total(s, t) * row_scale(g.scale0, t);
-                        const float up = row_total(s, g.R + t) * row_scale(g.scale1, t);
+                    for (int t = ct; t < g.R; t += kConsumerThreads) {
+                        const float gt = row_total(s, g, t) * row_scale(s0, t);
+                        const float up = row_total(s, g, g.R + t) * row_scale(s1, t);
                         const float silu = gt / (1.f + __expf(-gt));
                         p.act[(size_t)l * p.ffn + d.r0 + t] = silu * up;
                     }
                 } else if (d.kind == TK_DOWN) {
-                    for (int t = tid; t < g.R; t += kConsumerThreads) {
-                        const int r = d.r0 + t;
-                        p.xout[(size_t)l * p.hidden + r] =
-                            __ldcg(p.xmid + (size_t)l * p.hidden + r) +
-                            row_total(s, t) * row_scale(g.scale0, t);
-                    }
+                    if (ct < g.R)
+                        p.xout[(size_t)l * p.hidden + d.r0 + ct] =
+                            base + row_total(s, g, ct) * row_scale(s0, ct);
                 } else {  // TK_LMHEAD
                     unsigned long long best = 0ull;
-                    for (int t = tid; t < g.R; t += kConsumerThreads) {
-                        const float y = row_total(s, t) * row_scale(g.scale0, t);
+                    for (int t = ct; t < g.R; t += kConsumerThreads) {
+                        const float y = row_total(s, g, t) * row_scale(s0, t);
                         p.logits[d.r0 + t] = y;
                         const unsigned long long kk = argmax_key(y, d.r0 + t);
                         best = kk > best ? kk : best;
@@ -926,7 +1257,7 @@ __global__ void __launch_bounds__(kThreads, 1) amk_decode_kernel(const __grid_co
                     if (lane == 0)
                         sk[warp] = best;
                     consumer_bar();
-                    if (tid == 0) {
+                    if (ct == 0) {
                         unsigned long long b = 0ull;
                         for (int w = 0; w < kConsumerWarps; ++w)
                             b = sk[w] > b ? sk[w] : b;
@@ -939,14 +1270,67 @@ __global__ void __launch_bounds__(kThreads, 1) amk_decode_kernel(const __grid_co
         }
         if (!ok)
             s.flags[0] = 1;
+        if (wprof) {
+            atomicAdd(&s.wacc[0], (unsigned long long)wt_store[0]);
+            atomicAdd(&s.wacc[1], (unsigned long long)wt_store[1]);
+        }
         consumer_bar();
         if (*reinterpret_cast<volatile int *>(s.flags))
             break;
-        if (tid == 0 && d.signal_ctr >= 0 && ti != p.skip_signal_task) {
-            __threadfence();
+        // release: the CTA barrier above orders every thread's stores before
+        // this release-add (cumulativity), so the waiters' acquire sees them
+        if (ct == 0 && d.signal_ctr >= 0 && ti != p.skip_signal_task)
             red_release_add(p.counters + d.signal_ctr, 1u);
+        if (prof) {
+            const uint64_t t_end = gtimer();
+            unsigned long long *pk = prof + (size_t)d.kind * kProfFields;
+            pk[0] += 1;
+            pk[1] += t_w1 - t_w0;
+            pk[2] += t_pro - t_w1;
+            pk[3] += 0;
+            pk[4] += t_end - t_w1;
+            pk[5] += t_end - t_epi;
+            pk[6] += s.wacc[0];
+            pk[7] += s.wacc[1];
         }
     }
+    if (prof)
+        prof[1] = gtimer();
+}
+
+// ------------------------------------------------------------------- kernel
+// One fast instance per (weight format, attention lane width), holding only
+// the paths its models use, plus one generic instance for the rest.
+template <int Q8, int ATT_E, int GENERIC>
+__global__ void __launch_bounds__(kThreads, 1) amk_decode_kernel(const __grid_constant__ KParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const SmemLayout s = smem_layout(smem_raw, p);
+    const int tid = threadIdx.x;
+    const int qb = p.queue_off[blockIdx.x], qe = p.queue_off[blockIdx.x + 1];
+
+    if (tid == 0) {
+        for (int i = 0; i < p.ring_stages; ++i) {
+            mbar_init(s.full_a + 8 * i, 1);
+            mbar_init(s.empty_a + 8 * i, kConsumerWarps);
+        }
+        // a failed earlier step poisons the device state: do no work until the
+        // host resets it (the counters no longer match the epoch)
+        s.flags[0] = ld_relaxed(&p.err->code) != 0u ? 1 : 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncthreads();
+    if (s.flags[0])
+        return;
+    if (tid < kProducerThreads) {
+        setmaxnreg_dec<kProducerRegs>();
+        if (tid == 0)
+            producer_loop(p, s, qb, qe);
+        return;
+    }
+    setmaxnreg_inc<kConsumerRegs>();
+    consumer_loop<Q8, ATT_E, GENERIC>(p, s, qb, qe, tid - kProducerThreads);
     // On abort the producer notices the flag, drains its copies and returns.
 }
 
@@ -956,18 +1340,37 @@ __global__ void __launch_bounds__(kThreads, 1) amk_decode_kernel(const __grid_co
 extern "C" int amk_kernel_smem_bytes(int ring_stages, int stage_bytes, int vec_floats)
 {
     return ring_stages * stage_bytes + vec_floats * 4 + kConsumerWarps * kMaxTaskRows * 4 +
-           2 * kMaxStages * 8 + 16 * 4 + 64 * 4;
+           2 * kMaxStages * 8 + 16 * 4 + 64 * 4 + 2 * 8 + 4 * (int)sizeof(TaskDesc);
 }
 
-extern "C" cudaError_t amk_kernel_configure(int smem_bytes)
+namespace {
+const void *kernel_for(int quant, int att_e, int generic)
 {
-    return cudaFuncSetAttribute(amk_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                smem_bytes);
+    if (generic)
+        return reinterpret_cast<const void *>(amk_decode_kernel<0, 0, 1>);
+#define AMK_K(Q, E) reinterpret_cast<const void *>(amk_decode_kernel<Q, E, 0>)
+    static const void *const table[2][5] = {
+        {AMK_K(0, 1), AMK_K(0, 2), AMK_K(0, 4), AMK_K(0, 8), AMK_K(0, 16)},
+        {AMK_K(1, 1), AMK_K(1, 2), AMK_K(1, 4), AMK_K(1, 8), AMK_K(1, 16)}};
+#undef AMK_K
+    int e = 0;
+    while (e < 4 && (1 << e) < att_e)
+        ++e;
+    return table[quant ? 1 : 0][e];
+}
+}  // namespace
+
+extern "C" cudaError_t amk_kernel_configure(int smem_bytes, int quant, int att_e, int generic)
+{
+    return cudaFuncSetAttribute(kernel_for(quant, att_e, generic),
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
 }
 
-extern "C" cudaError_t amk_kernel_occupancy(int smem_bytes, int *blocks_per_sm)
+extern "C" cudaError_t amk_kernel_occupancy(int smem_bytes, int quant, int att_e, int generic,
+                                            int *blocks_per_sm)
 {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, amk_decode_kernel,
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm,
+                                                         kernel_for(quant, att_e, generic),
                                                          kThreads, smem_bytes);
 }
 
@@ -975,9 +1378,8 @@ extern "C" cudaError_t amk_kernel_launch(const KParams *p, int n_ctas, int smem_
                                          cudaStream_t stream)
 {
     void *args[] = {const_cast<KParams *>(p)};
-    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(amk_decode_kernel),
-                                       dim3(n_ctas), dim3(kThreads), args, (size_t)smem_bytes,
-                                       stream);
+    return cudaLaunchCooperativeKernel(kernel_for(p->quant, p->att_e, p->generic), dim3(n_ctas),
+                                       dim3(kThreads), args, (size_t)smem_bytes, stream);
 }
 
 }  // namespace amk

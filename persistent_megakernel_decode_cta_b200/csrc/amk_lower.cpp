@@ -79,6 +79,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         if (opt_in->tasks_per_sm > 0) opt.tasks_per_sm = opt_in->tasks_per_sm;
         if (opt_in->wait_timeout_us > 0) opt.wait_timeout_us = opt_in->wait_timeout_us;
         opt.debug_skip_signal_task = opt_in->debug_skip_signal_task;
+        opt.profile = opt_in->profile;
         opt.n_sms = opt_in->n_sms;
     }
     const amk_config &c = *cfg;
@@ -105,7 +106,11 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     int lph = 32;
     while (lph > 1 && (lph * G > 32 || hd % lph))
         lph >>= 1;
-    if (G > 32 || lph * G > 32 || hd % lph || hd / lph > 32)
+    const int att_e = hd / lph;
+    if (h > 16 * 256 || nh * hd > 16 * 256 || F > 3 * 16 * 256 * 4)
+        return amk_set_error(AMK_ERR_UNSUPPORTED, "hidden or heads*head_dim above 4096, or ffn "
+                             "above 49152 (prologue register blocking)");
+    if (G > 32 || lph * G > 32 || hd % lph || att_e > 16 || (att_e & (att_e - 1)))
         return amk_set_error(AMK_ERR_UNSUPPORTED, "attention layout: group %d x head_dim %d "
                              "does not fit one warp", G, hd);
     const int esz = c.quant == AMK_QUANT_W8A16 ? 1 : 2;
@@ -140,7 +145,10 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         C = std::max(1, std::min(by_sms, by_combine));
     }
     C = std::min(C, c.max_ctx);
-    int vec = std::max({h, F, nh * hd + nh * C,
+    // the shared vector holds a prologue's output: the normed hidden state,
+    // the combined attention output (+ per-head weights), or the attention
+    // tile's scratch; DOWN tiles read their activations from L2 directly
+    int vec = std::max({h, nh * hd + nh * C,
                         G * hd + 2 * hd + amk::kConsumerWarps * G * (hd + 2)});
     vec = (vec + 3) & ~3;
     int stages = opt.ring_stages;
@@ -162,6 +170,10 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     P->att_lph = lph;
     P->att_hpb = 32 / lph;
     P->att_e = hd / lph;
+    P->generic = (c.tied_embeddings && c.quant == AMK_QUANT_W8A16) ? 1 : 0;
+    for (const Mat &m : mats)
+        if (((int64_t)m.K * m.esz) % 16)
+            P->generic = 1;
 
     // ---- logical tasks per level ---------------------------------------------
     enum { LV_QKV, LV_ATTN, LV_OPROJ, LV_GATEUP, LV_DOWN, LV_N };
@@ -422,4 +434,62 @@ void amk_plan_view(const amk_plan *P, amk_graph *g)
     g->buffers = P->gbufs.data();
     g->queue_offsets = P->queue_off.data();
     g->queue_tasks = P->gqueue.data();
+}
+
+void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *kv, int t,
+                      amk::TaskDesc *out)
+{
+    const amk_config &c = P->cfg;
+    amk::TaskDesc d = P->tasks[t];
+    const int l = d.layer;
+    const bool q8 = c.quant == AMK_QUANT_W8A16;
+    const int esz = q8 ? 1 : 2;
+    auto row = [](const void *base, int64_t r, int64_t row_bytes) {
+        return static_cast<const void *>(static_cast<const uint8_t *>(base) + r * row_bytes);
+    };
+    auto srow = [&](const void *const *arr, int64_t r) -> const uint16_t * {
+        return q8 ? static_cast<const uint16_t *>(arr[l]) + r : nullptr;
+    };
+    d.w0 = d.w1 = nullptr;
+    d.s0 = d.s1 = d.gain = nullptr;
+    const int h = c.hidden;
+    switch (d.kind) {
+    case amk::TK_QKV: {
+        const void *const *mats[3] = {w->wq, w->wk, w->wv};
+        const void *const *scs[3] = {w->sq, w->sk, w->sv};
+        d.w0 = row(mats[d.mat][l], d.r0, (int64_t)h * esz);
+        d.s0 = srow(scs[d.mat], d.r0);
+        d.gain = static_cast<const uint16_t *>(w->attn_norm[l]);
+        break;
+    }
+    case amk::TK_ATTN: {
+        const size_t blk = (size_t)c.max_ctx * c.head_dim;
+        d.w0 = kv + (((size_t)l * 2 + 0) * c.n_kv_heads + d.r0) * blk;
+        d.w1 = kv + (((size_t)l * 2 + 1) * c.n_kv_heads + d.r0) * blk;
+        break;
+    }
+    case amk::TK_OPROJ:
+        d.w0 = row(w->wo[l], d.r0, (int64_t)c.n_heads * c.head_dim * esz);
+        d.s0 = srow(w->so, d.r0);
+        break;
+    case amk::TK_GATEUP:
+        d.w0 = row(w->wgate[l], d.r0, (int64_t)h * esz);
+        d.w1 = row(w->wup[l], d.r0, (int64_t)h * esz);
+        d.s0 = srow(w->sgate, d.r0);
+        d.s1 = srow(w->sup, d.r0);
+        d.gain = static_cast<const uint16_t *>(w->ffn_norm[l]);
+        break;
+    case amk::TK_DOWN:
+        d.w0 = row(w->wdown[l], d.r0, (int64_t)c.ffn * esz);
+        d.s0 = srow(w->sdown, d.r0);
+        break;
+    default: {  // TK_LMHEAD
+        const bool head_q8 = q8 && !c.tied_embeddings;
+        d.w0 = row(c.tied_embeddings ? w->embed : w->lm_head, d.r0, (int64_t)h * (head_q8 ? 1 : 2));
+        d.s0 = head_q8 ? static_cast<const uint16_t *>(w->lm_head_scale) + d.r0 : nullptr;
+        d.gain = static_cast<const uint16_t *>(w->final_norm);
+        break;
+    }
+    }
+    *out = d;
 }

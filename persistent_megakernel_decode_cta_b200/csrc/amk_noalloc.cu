@@ -21,7 +21,7 @@
 #include "amk_plan.h"
 
 extern "C" int amk_kernel_smem_bytes(int ring_stages, int stage_bytes, int vec_floats);
-extern "C" cudaError_t amk_kernel_configure(int smem_bytes);
+extern "C" cudaError_t amk_kernel_configure(int smem_bytes, int quant, int att_e, int generic);
 namespace amk {
 extern "C" cudaError_t amk_kernel_launch(const KParams *p, int n_ctas, int smem_bytes,
                                          cudaStream_t stream);
@@ -39,7 +39,7 @@ void *g_scratch_addr[kMaxDevices];  // device address of g_scratch, per device
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t tasks, qoff, layers, ctr, err, argkey, qkv, part, xmid, xout, act, total;
+    size_t tasks, qoff, ctr, err, argkey, qkv, part, xmid, xout, act, total;
 };
 
 Layout layout_of(const amk_plan &P)
@@ -56,7 +56,6 @@ Layout layout_of(const amk_plan &P)
     };
     o.tasks = take(sizeof(amk::TaskDesc) * P.tasks.size());
     o.qoff = take(sizeof(int32_t) * P.queue_off.size());
-    o.layers = take(sizeof(amk::LayerPtrs) * L);
     o.ctr = take(sizeof(uint32_t) * (size_t)P.n_counters);
     o.err = take(sizeof(amk::ErrorWord));
     o.argkey = take(2 * sizeof(unsigned long long));
@@ -143,35 +142,32 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
         return rc;
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     cudaError_t e;
-    // schedule tables (pageable sources: cudaMemcpyAsync stages them before
-    // returning, so the stack buffer below can be reused at once)
-    e = cudaMemcpyAsync(base + lay.tasks, P.tasks.data(), sizeof(amk::TaskDesc) * P.tasks.size(),
+    // per-layer pointers must all be present before any task is resolved
+    for (int l = 0; l < c.n_layers; ++l) {
+        if (!ok16(w->attn_norm[l]) || !ok16(w->ffn_norm[l]))
+            return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d norm NULL or misaligned", l);
+        for (int m = 0; m < 7; ++m)
+            if (!ok16(mats[m][l]) || (q8 && !scs[m][l]))
+                return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d weight %d", l, m);
+    }
+    // schedule tables with resolved pointers, in batches through a stack
+    // buffer (pageable sources: cudaMemcpyAsync stages them before returning,
+    // so the buffer can be reused at once)
+    e = cudaMemcpyAsync(base + lay.qoff, P.queue_off.data(), sizeof(int32_t) * P.queue_off.size(),
                         cudaMemcpyHostToDevice, st);
-    if (e == cudaSuccess)
-        e = cudaMemcpyAsync(base + lay.qoff, P.queue_off.data(),
-                            sizeof(int32_t) * P.queue_off.size(), cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess)
         return fail_cuda(e, "schedule upload");
-    amk::LayerPtrs lp[16];
-    for (int l0 = 0; l0 < c.n_layers; l0 += 16) {
-        const int n = c.n_layers - l0 < 16 ? c.n_layers - l0 : 16;
-        for (int i = 0; i < n; ++i) {
-            const int l = l0 + i;
-            if (!ok16(w->attn_norm[l]) || !ok16(w->ffn_norm[l]))
-                return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d norm NULL or misaligned", l);
-            for (int m = 0; m < 7; ++m) {
-                if (!ok16(mats[m][l]) || (q8 && !scs[m][l]))
-                    return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d weight %d", l, m);
-                lp[i].w[m] = mats[m][l];
-                lp[i].s[m] = q8 ? static_cast<const uint16_t *>(scs[m][l]) : nullptr;
-            }
-            lp[i].attn_norm = static_cast<const uint16_t *>(w->attn_norm[l]);
-            lp[i].ffn_norm = static_cast<const uint16_t *>(w->ffn_norm[l]);
-        }
-        e = cudaMemcpyAsync(base + lay.layers + sizeof(amk::LayerPtrs) * l0, lp,
-                            sizeof(amk::LayerPtrs) * n, cudaMemcpyHostToDevice, st);
+    amk::TaskDesc batch[64];
+    const uint16_t *kv = static_cast<const uint16_t *>(kv_cache);
+    const int T = (int)P.tasks.size();
+    for (int t0 = 0; t0 < T; t0 += 64) {
+        const int n = T - t0 < 64 ? T - t0 : 64;
+        for (int i = 0; i < n; ++i)
+            amk_resolve_task(&P, w, kv, t0 + i, &batch[i]);
+        e = cudaMemcpyAsync(base + lay.tasks + sizeof(amk::TaskDesc) * (size_t)t0, batch,
+                            sizeof(amk::TaskDesc) * (size_t)n, cudaMemcpyHostToDevice, st);
         if (e != cudaSuccess)
-            return fail_cuda(e, "layer table upload");
+            return fail_cuda(e, "schedule upload");
     }
     // what must start at zero: counters, error word, argmax keys
     e = cudaMemsetAsync(base + lay.ctr, 0, lay.qkv - lay.ctr, st);
@@ -183,12 +179,7 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     k.queue_off = reinterpret_cast<const int32_t *>(base + lay.qoff);
     k.counters = reinterpret_cast<uint32_t *>(base + lay.ctr);
     k.err = reinterpret_cast<amk::ErrorWord *>(base + lay.err);
-    k.layers = reinterpret_cast<const amk::LayerPtrs *>(base + lay.layers);
     k.embed = static_cast<const uint16_t *>(w->embed);
-    k.final_norm = static_cast<const uint16_t *>(w->final_norm);
-    k.lm_head = static_cast<const uint16_t *>(c.tied_embeddings ? w->embed : w->lm_head);
-    k.lm_head_scale = (q8 && !c.tied_embeddings)
-                          ? static_cast<const uint16_t *>(w->lm_head_scale) : nullptr;
     k.qkv = reinterpret_cast<float *>(base + lay.qkv);
     k.part = reinterpret_cast<float *>(base + lay.part);
     k.xmid = reinterpret_cast<float *>(base + lay.xmid);
@@ -218,13 +209,14 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     k.att_lph = P.att_lph;
     k.att_hpb = P.att_hpb;
     k.att_e = P.att_e;
+    k.generic = P.generic;
     k.pos = pos;
     k.token = token_id;
     k.epoch = 0;   // counters were cleared above
     k.parity = 0;
     k.timeout_ns = (uint64_t)P.opt.wait_timeout_us * 1000ull;
     k.skip_signal_task = P.opt.debug_skip_signal_task;
-    e = amk_kernel_configure(P.smem_bytes);
+    e = amk_kernel_configure(P.smem_bytes, q8 ? 1 : 0, P.att_e, P.generic);
     if (e != cudaSuccess)
         return fail_cuda(e, "cudaFuncSetAttribute");
     e = amk::amk_kernel_launch(&k, P.n_sms, P.smem_bytes, st);

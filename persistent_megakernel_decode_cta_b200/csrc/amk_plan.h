@@ -14,6 +14,7 @@ struct amk_plan {
     int n_sms = 0;
     int group = 0, qkv_rows = 0, vec_floats = 0, smem_bytes = 0;
     int att_lph = 0, att_hpb = 0, att_e = 0;
+    int generic = 0;  // 1: odd row widths or a bf16 tied head on int8 layers
     std::vector<amk::TaskDesc> tasks;  // grouped by SM, queue order
     std::vector<int32_t> queue_off;    // [n_sms + 1]
     int n_counters = 0;
@@ -32,5 +33,10 @@ struct amk_plan {
 int amk_lower(const amk_config *cfg, const amk_options *opt, int n_sms, amk_plan *P);
 // A non-owning amk_graph view of P's graph arrays.
 void amk_plan_view(const amk_plan *P, amk_graph *g);
+// Copies plan task t into *out with its device pointers resolved: weight
+// rows, row scales and norm gain from w, KV-cache blocks from kv (bf16
+// [L][2][nkv][max_ctx][hd]).  Host only; reads only host memory.
+void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *kv, int t,
+                      amk::TaskDesc *out);
 
 #endif
