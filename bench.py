@@ -65,12 +65,11 @@ KERNEL_SOURCES = ["persistent_megakernel_decode_cta_b200/csrc/amk_kernel.cu",
 
 def algorithmic_bytes(cfg, ctx: int) -> int:
     """Bytes one decode step must move: every weight byte once (int8 scales,
-    norm gains and one embedding row included), the KV rows 0..ctx-1 of every
-    layer, the new K/V row, and the logits."""
-    b = si.model_bytes(cfg)
+    norm gains, one embedding row and the LM head -- the embedding table when
+    tied -- included), the KV rows 0..ctx-1 of every layer, the new K/V row,
+    and the logits."""
     kv_row = 2 * cfg.n_layers * cfg.n_kv_heads * cfg.head_dim * 2
-    return (b["linear"] + b["scales"] + b["head"] + b["norms"] + b["embed_row"]
-            + kv_row * ctx + kv_row + cfg.vocab * 4)
+    return si.streamed_weight_bytes(cfg) + kv_row * ctx + kv_row + cfg.vocab * 4
 
 
 def kernel_hash() -> str:

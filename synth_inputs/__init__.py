@@ -41,6 +41,7 @@ __all__ = [
     "make_prompt",
     "make_kv_fill",
     "model_bytes",
+    "streamed_weight_bytes",
 ]
 
 
@@ -223,3 +224,12 @@ def model_bytes(cfg) -> Dict[str, int]:
         "norms": norms, "embed_row": h * 2,
         "embed_table": cfg.vocab * h * 2,
     }
+
+
+def streamed_weight_bytes(cfg) -> int:
+    """Weight bytes one decode step reads: every linear weight (and int8 row
+    scale) once, the LM head -- the whole embedding table when tied --, the
+    norm gains and the one embedding row of the input token."""
+    b = model_bytes(cfg)
+    head = b["embed_table"] if get_config(cfg).tied else b["head"]
+    return b["linear"] + b["scales"] + head + b["norms"] + b["embed_row"]
