@@ -596,23 +596,23 @@ __device__ float block_sum(float v, const SmemLayout &s, int ct)
 }
 
 // vec[i] = g_i * x_i / sqrt(mean x^2 + eps), x from L2 (fp32) or the
-// embedding row (bf16).  Every load of a thread is issued before any store
-// (one L2 round trip); hidden <= kMaxPerThread * 256.
+// embedding row (bf16).  The gains gv (thread t: elements t + 256 j) were
+// loaded before the task's counter wait, so that their first touch in HBM
+// is off the critical path; every load of x is issued before any store (one
+// L2 round trip); hidden <= kMaxPerThread * 256.
 constexpr int kMaxPerThread = 16;
 __device__ void rmsnorm_prologue(const KParams &p, const SmemLayout &s, const float *x_f32,
-                                 const uint16_t *x_bf16, const uint16_t *gain, int ct)
+                                 const uint16_t *x_bf16, const float (&gv)[kMaxPerThread],
+                                 int ct)
 {
     const int n = p.hidden;
-    float xv[kMaxPerThread], gv[kMaxPerThread];
+    float xv[kMaxPerThread];
 #pragma unroll
     for (int j = 0; j < kMaxPerThread; ++j) {
         const int i = ct + j * kConsumerThreads;
         xv[j] = 0.f;
-        gv[j] = 0.f;
-        if (i < n) {
+        if (i < n)
             xv[j] = x_f32 ? __ldcg(x_f32 + i) : bf16_to_f(__ldg(x_bf16 + i));
-            gv[j] = bf16_to_f(__ldg(gain + i));
-        }
     }
     float ss = 0.f;
 #pragma unroll
@@ -1135,6 +1135,22 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
         }
         if (wprof)
             wt_store[0] = wt_store[1] = 0;
+        // loads that do not depend on this step's activations go out before
+        // the counter wait: the RMSNorm gains and the int8 row scales of the
+        // epilogue (thread t finalises row r0 + t; R <= 256)
+        const Geom g = task_geom(p, d);
+        float gv[kMaxPerThread];
+        const bool norm = d.kind == TK_QKV || d.kind == TK_GATEUP || d.kind == TK_LMHEAD;
+#pragma unroll
+        for (int j = 0; j < kMaxPerThread; ++j) {
+            const int i = ct + j * kConsumerThreads;
+            gv[j] = (norm && i < p.hidden) ? bf16_to_f(__ldg(d.gain + i)) : 0.f;
+        }
+        float sc0 = 1.f, sc1 = 1.f;
+        if (d.kind != TK_ATTN && ct < g.R) {
+            sc0 = row_scale(d.s0, ct);
+            sc1 = row_scale(d.s1, ct);
+        }
         if (ct == 0) {
             if (ti + 1 < qe)  // the slot read at ti - 1 is free again (barrier above)
                 stage_task(s.ctask_a + ((ti + 1 - qb) & 1) * sizeof(TaskDesc), p.tasks + ti + 1);
@@ -1146,7 +1162,6 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
             break;
         if (prof)
             t_w1 = gtimer();
-        const Geom g = task_geom(p, d);
         const int l = d.layer;
         bool ok = true;
         if (d.kind == TK_ATTN) {
@@ -1169,22 +1184,20 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
                 if (l == 0) {
                     if (token < 0)
                         token = resolve_token(p);
-                    rmsnorm_prologue(p, s, nullptr, p.embed + (size_t)token * p.hidden, d.gain,
-                                     ct);
+                    rmsnorm_prologue(p, s, nullptr, p.embed + (size_t)token * p.hidden, gv, ct);
                 } else {
-                    rmsnorm_prologue(p, s, p.xout + (size_t)(l - 1) * p.hidden, nullptr, d.gain,
-                                     ct);
+                    rmsnorm_prologue(p, s, p.xout + (size_t)(l - 1) * p.hidden, nullptr, gv, ct);
                 }
             } else if (d.kind == TK_OPROJ) {
                 combine_prologue(p, s, l, ct);
             } else if (d.kind == TK_GATEUP) {
-                rmsnorm_prologue(p, s, p.xmid + (size_t)l * p.hidden, nullptr, d.gain, ct);
+                rmsnorm_prologue(p, s, p.xmid + (size_t)l * p.hidden, nullptr, gv, ct);
             } else if (d.kind == TK_DOWN) {
                 // no prologue: each warp loads its slice of the SwiGLU
                 // activations from L2 straight into registers
             } else {  // TK_LMHEAD
                 rmsnorm_prologue(p, s, p.xout + (size_t)(p.n_layers - 1) * p.hidden, nullptr,
-                                 d.gain, ct);
+                                 gv, ct);
             }
             // residual inputs of the epilogue are ready now: fetch them while
             // the GEMV runs (thread t owns output row r0 + t; R <= 256)
@@ -1217,33 +1230,32 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
             ok = *reinterpret_cast<volatile int *>(s.flags) == 0;
             if (ok) {
                 // epilogue: thread t finalises output row r0 + t
-                const uint16_t *s0 = d.s0, *s1 = d.s1;
                 if (d.kind == TK_QKV) {
                     const int off = d.mat == 0 ? 0
                                     : d.mat == 1 ? p.n_heads * p.head_dim
                                                  : (p.n_heads + p.n_kv_heads) * p.head_dim;
                     float *out = p.qkv + (size_t)l * p.qkv_rows + off + d.r0;
                     for (int t = ct; t < g.R; t += kConsumerThreads)
-                        out[t] = row_total(s, g, t) * row_scale(s0, t);
+                        out[t] = row_total(s, g, t) * sc0;
                 } else if (d.kind == TK_OPROJ) {
                     if (ct < g.R)
                         p.xmid[(size_t)l * p.hidden + d.r0 + ct] =
-                            base + row_total(s, g, ct) * row_scale(s0, ct);
+                            base + row_total(s, g, ct) * sc0;
                 } else if (d.kind == TK_GATEUP) {
                     for (int t = ct; t < g.R; t += kConsumerThreads) {
-                        const float gt = row_total(s, g, t) * row_scale(s0, t);
-                        const float up = row_total(s, g, g.R + t) * row_scale(s1, t);
+                        const float gt = row_total(s, g, t) * sc0;
+                        const float up = row_total(s, g, g.R + t) * sc1;
                         const float silu = gt / (1.f + __expf(-gt));
                         p.act[(size_t)l * p.ffn + d.r0 + t] = silu * up;
                     }
                 } else if (d.kind == TK_DOWN) {
                     if (ct < g.R)
                         p.xout[(size_t)l * p.hidden + d.r0 + ct] =
-                            base + row_total(s, g, ct) * row_scale(s0, ct);
+                            base + row_total(s, g, ct) * sc0;
                 } else {  // TK_LMHEAD
                     unsigned long long best = 0ull;
                     for (int t = ct; t < g.R; t += kConsumerThreads) {
-                        const float y = row_total(s, g, t) * row_scale(s0, t);
+                        const float y = row_total(s, g, t) * sc0;
                         p.logits[d.r0 + t] = y;
                         const unsigned long long kk = argmax_key(y, d.r0 + t);
                         best = kk > best ? kk : best;
