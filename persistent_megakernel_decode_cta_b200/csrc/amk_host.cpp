@@ -141,7 +141,8 @@ struct amk_handle {
     int32_t *d_qoff = nullptr;
     uint32_t *d_ctr = nullptr;
     ErrorWord *d_err = nullptr;
-    float *d_qkv = nullptr, *d_part = nullptr, *d_xmid = nullptr, *d_xout = nullptr;
+    float *d_qkv = nullptr, *d_part = nullptr, *d_attn = nullptr, *d_xmid = nullptr,
+          *d_xout = nullptr;
     float *d_act = nullptr, *d_logits = nullptr;
     unsigned long long *d_argkey = nullptr;
     unsigned long long *d_prof = nullptr;
@@ -153,6 +154,7 @@ struct amk_handle {
     bool err_pending = false;
     KParams kp{};
     uint32_t epoch = 0;
+    uint32_t arrive_base = 0;  // attention chunk arrivals so far, per (layer, kv head)
     bool poisoned = false;
     amk_error_info last_err{};
 };
@@ -237,7 +239,8 @@ int zero_state(amk_handle *H)
     cudaError_t e;
     e = cudaMemsetAsync(H->d_kv, 0, H->kv_bytes, H->stream);
     if (e == cudaSuccess)
-        e = cudaMemsetAsync(H->d_ctr, 0, sizeof(uint32_t) * (size_t)P->n_counters, H->stream);
+        e = cudaMemsetAsync(H->d_ctr, 0, sizeof(uint32_t) * (size_t)(P->n_counters + P->n_arrive),
+                            H->stream);
     if (e == cudaSuccess)
         e = cudaMemsetAsync(H->d_err, 0, sizeof(ErrorWord), H->stream);
     if (e == cudaSuccess)
@@ -247,6 +250,7 @@ int zero_state(amk_handle *H)
     if (e != cudaSuccess)
         return cuda_fail(e, "amk_reset_kv");
     H->epoch = 0;
+    H->arrive_base = 0;
     H->poisoned = false;
     H->err_pending = false;
     memset(&H->last_err, 0, sizeof H->last_err);
@@ -324,14 +328,15 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     const int L = c.n_layers, nkv = c.n_kv_heads, hd = c.head_dim;
     const size_t part_floats = (size_t)nkv * P->opt.attn_splits * P->group * (hd + 2);
     const size_t qkv_f = (size_t)L * P->qkv_rows, part_f = (size_t)L * part_floats;
+    const size_t attn_f = (size_t)L * c.n_heads * hd;
     const size_t h_f = (size_t)L * c.hidden, act_f = (size_t)L * c.ffn;
     H->kv_bytes = (size_t)L * 2 * nkv * c.max_ctx * hd * sizeof(uint16_t);
-    // activations in one block: qkv | part | xmid | xout | act
-    H->act_bytes = (qkv_f + part_f + 2 * h_f + act_f) * sizeof(float);
+    // activations in one block: qkv | part | attn | xmid | xout | act
+    H->act_bytes = (qkv_f + part_f + attn_f + 2 * h_f + act_f) * sizeof(float);
     float *act_block = nullptr;
     if ((rc = dalloc(H, &H->d_tasks, sizeof(TaskDesc) * P->tasks.size())) ||
         (rc = dalloc(H, &H->d_qoff, sizeof(int32_t) * P->queue_off.size())) ||
-        (rc = dalloc(H, &H->d_ctr, sizeof(uint32_t) * (size_t)P->n_counters)) ||
+        (rc = dalloc(H, &H->d_ctr, sizeof(uint32_t) * (size_t)(P->n_counters + P->n_arrive))) ||
         (rc = dalloc(H, &H->d_err, sizeof(ErrorWord))) ||
         (rc = dalloc(H, &act_block, H->act_bytes)) ||
         (rc = dalloc(H, &H->d_logits, sizeof(float) * (size_t)c.vocab)) ||
@@ -345,7 +350,8 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     }
     H->d_qkv = act_block;
     H->d_part = H->d_qkv + qkv_f;
-    H->d_xmid = H->d_part + part_f;
+    H->d_attn = H->d_part + part_f;
+    H->d_xmid = H->d_attn + attn_f;
     H->d_xout = H->d_xmid + h_f;
     H->d_act = H->d_xout + h_f;
     if ((e = cudaMallocHost(&H->h_err, sizeof(ErrorWord))) != cudaSuccess ||
@@ -381,6 +387,8 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     k.embed = static_cast<const uint16_t *>(w->embed);
     k.qkv = H->d_qkv;
     k.part = H->d_part;
+    k.attn = H->d_attn;
+    k.arrive = H->d_ctr + P->n_counters;
     k.xmid = H->d_xmid;
     k.xout = H->d_xout;
     k.act = H->d_act;
@@ -463,6 +471,7 @@ int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev,
     k.pos = pos;
     k.token = token_id;
     k.epoch = H->epoch;
+    k.arrive_base = H->arrive_base;
     k.parity = (int32_t)(H->epoch & 1u);
     if (logits_dev)
         k.logits = logits_dev;
@@ -482,6 +491,12 @@ int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev,
                              "cooperative launch: %s", cudaGetErrorString(e));
     }
     H->epoch += 1;
+    {  // non-empty attention chunks of this step: each arrives once unless alone
+        const int C = H->plan->opt.attn_splits, n = pos + 1;
+        const int chunk = (n + C - 1) / C, nne = (n + chunk - 1) / chunk;
+        if (nne > 1)
+            H->arrive_base += (uint32_t)nne;
+    }
     // The error word is read back when the caller synchronises, and every 32
     // asynchronous steps otherwise (a failed step makes later kernels exit at
     // once, so a late look costs no device time).

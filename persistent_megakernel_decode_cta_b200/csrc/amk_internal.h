@@ -40,8 +40,9 @@ constexpr int kMaxStages = 16;
 // epilogues, and the split-K attention tile).
 enum TaskKind : uint8_t {
     TK_QKV = 1,     // rows of Wq|Wk|Wv (mat 0/1/2), RMSNorm prologue, raw q/k/v out
-    TK_ATTN = 2,    // (kv head g, split c): RoPE, KV append (c == 0), partial softmax
-    TK_OPROJ = 3,   // rows of Wo, split-K combine prologue, residual epilogue
+    TK_ATTN = 2,    // (kv head g, split c): RoPE, KV append (c == 0), partial softmax;
+                    // the head's last chunk to finish merges all of them
+    TK_OPROJ = 3,   // rows of Wo, attention-output prologue, residual epilogue
     TK_GATEUP = 4,  // rows of Wgate and Wup, RMSNorm prologue, SwiGLU epilogue
     TK_DOWN = 5,    // rows of Wdown, residual epilogue
     TK_LMHEAD = 6,  // rows of the LM head, final RMSNorm prologue, argmax epilogue
@@ -88,12 +89,14 @@ struct KParams {
     const TaskDesc *tasks;     // grouped by SM, in queue order
     const int32_t *queue_off;  // [n_sms + 1]
     uint32_t *counters;
+    uint32_t *arrive;          // [L][nkv]: attention chunk tasks arrived, monotonic
     ErrorWord *err;
     // weights (the per-task pointers live in the task records)
     const uint16_t *embed;
     // state and activations (fp32 unless noted)
     float *qkv;       // [L][qkv_rows]: q | k | v, before RoPE
     float *part;      // [L][nkv][C][G][hd + 2]: split-K partials (m, l, o[hd])
+    float *attn;      // [L][nh * hd]: attention output (the chunks merged)
     float *xmid;      // [L][h]: residual after attention
     float *xout;      // [L][h]: residual after the FFN
     float *act;       // [L][ffn]: SwiGLU activations
@@ -112,6 +115,7 @@ struct KParams {
     // step
     int32_t pos, token;         // token < 0: previous step's argmax
     uint32_t epoch;             // steps since reset (counter targets)
+    uint32_t arrive_base;       // attention arrivals of earlier steps per (layer, kv head)
     int32_t parity;             // epoch & 1
     uint64_t timeout_ns;
     int32_t skip_signal_task;   // test hook, -1 = off

@@ -827,7 +827,7 @@ __device__ __forceinline__ void lds_bf16(uint32_t a, float (&out)[E])
 // Split-K attention tile for KV head g and chunk c (flash-decoding partial):
 // writes (m, l, o[hd]) per query head of the group, unnormalised.
 template <int E>
-__device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
+__device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s,
                                           const TaskDesc &d, const Geom &g, uint32_t &kc,
                                           int ct, int warp, int lane, uint64_t *wt)
 {
@@ -840,7 +840,7 @@ __device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
     float *ws = vn + hd;                     // [8][G][hd + 2] per-warp partials
     const float *qkv = p.qkv + (size_t)l * p.qkv_rows;
     if (g.j1 <= g.j0)
-        return true;  // empty chunk: nothing to write, the combine skips it
+        return true;  // empty chunk: no partial (the merge skips it)
     // prologue: q of the group's G heads and k get RoPE (pairs i, i + hd/2),
     // q is pre-scaled by 1/sqrt(hd); k and v are rounded to bf16 (the cache
     // format) and chunk 0 appends them at row pos
@@ -998,7 +998,11 @@ __device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
         }
     }
     consumer_bar();
+    // the only non-empty chunk of the step writes the normalised output of
+    // its heads directly; otherwise the partial (m, l, o) for the merge
+    const bool direct = g.j0 == 0 && g.j1 == p.pos + 1;
     float *out = p.part + ((((size_t)l * nkv + gi) * p.attn_splits + c) * G) * (hd + 2);
+    float *fin = p.attn + (size_t)l * nh * hd + (size_t)gi * G * hd;
     for (int i = ct; i < G * hd; i += kConsumerThreads) {
         const int hh = i / hd, e = i % hd;
         float M = -INFINITY;
@@ -1013,6 +1017,10 @@ __device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
             L = fmaf(pw[1], f, L);
             O = fmaf(pw[2 + e], f, O);
         }
+        if (direct) {
+            fin[i] = O / L;
+            continue;
+        }
         out[(size_t)hh * (hd + 2) + 2 + e] = O;
         if (e == 0) {
             out[(size_t)hh * (hd + 2) + 0] = M;
@@ -1022,63 +1030,150 @@ __device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
     return true;
 }
 
-// O-projection prologue: combine the split-K partials of every head into
-// the attention output vec[h * hd + e] = sum_c e^(m_c - M) o_c[e] / L with
-// M = max_c m_c and L = sum_c e^(m_c - M) l_c.  Per split, every load of a
-// thread is issued before the arithmetic (one L2 round trip per split);
-// n_heads * head_dim <= kMaxPerThread * 256.
-__device__ void combine_prologue(const KParams &p, const SmemLayout &s, int l, int ct)
+// Merge of split-K partials: out[i] = sum_c e^(m_c - M) o_c[e] / L with
+// M = max_c m_c and L = sum_c e^(m_c - M) l_c over the non-empty chunks c,
+// for the attention-output elements first + i, i < count (element = head *
+// hd + e; count <= kMaxPerThread * 256).  Thread t owns i = t + 256 j, in
+// batches of B; for a batch the
+// (m, l, o) of up to K chunks are loaded at once (one L2 round trip) and
+// merged online in registers; address math is done once per element.
+// K = 1 serves a single non-empty chunk (short contexts: out = o / l).
+template <int K, int B>
+__device__ __forceinline__ void merge_batches(const KParams &p, const float *part, int nne,
+                                              int first, int count, float *out, int ct)
 {
-    const int hd = p.head_dim, nh = p.n_heads, G = p.group, C = p.attn_splits;
-    const int n = p.pos + 1;
-    const int chunk = (n + C - 1) / C;
-    const int nne = (n + chunk - 1) / chunk;  // non-empty splits
-    const float *part = p.part + (size_t)l * p.n_kv_heads * C * G * (hd + 2);
-    const int N = nh * hd;
-    const size_t cstride = (size_t)G * (hd + 2);
-    constexpr int B = 8;  // elements per batch of independent loads
+    const int hd = p.head_dim, G = p.group, C = p.attn_splits;
+    const size_t cstride = (size_t)G * (hd + 2);  // chunk c + 1 of a head is this far on
     for (int j0 = 0; j0 < kMaxPerThread; j0 += B) {
-        if (ct + j0 * kConsumerThreads >= N)
+        if (ct + j0 * kConsumerThreads >= count)
             break;
+        const float *rp[B];  // (m, l, o[hd]) record of the element's head in chunk 0
+        int eo[B];
         float M[B], L[B], O[B];
 #pragma unroll
         for (int j = 0; j < B; ++j) {
+            const int i = ct + (j0 + j) * kConsumerThreads;
+            rp[j] = nullptr;
+            eo[j] = 0;
+            if (i < count) {
+                const int h = (first + i) / hd;
+                rp[j] = part + ((size_t)(h / G) * C * G + (h % G)) * (hd + 2);
+                eo[j] = 2 + (first + i - h * hd);
+            }
             M[j] = -INFINITY;
             L[j] = 0.f;
             O[j] = 0.f;
         }
-        for (int c = 0; c < nne; ++c) {
-            float2 ml[B];
-            float oc[B];
+        for (int c0 = 0; c0 < nne; c0 += K) {
+            float2 ml[K][B];
+            float oc[K][B];
 #pragma unroll
-            for (int j = 0; j < B; ++j) {
-                const int i = ct + (j0 + j) * kConsumerThreads;
-                if (i < N) {
-                    const int h = i / hd;
-                    const float *pc =
-                        part + ((size_t)(h / G) * C * G + (h % G)) * (hd + 2) + c * cstride;
-                    ml[j] = __ldcg(reinterpret_cast<const float2 *>(pc));
-                    oc[j] = __ldcg(pc + 2 + (i - h * hd));
-                }
-            }
+            for (int k = 0; k < K; ++k)
 #pragma unroll
-            for (int j = 0; j < B; ++j) {
-                const int i = ct + (j0 + j) * kConsumerThreads;
-                if (i < N) {
-                    const float Mn = fmaxf(M[j], ml[j].x);
-                    const float a = __expf(M[j] - Mn), b = __expf(ml[j].x - Mn);
-                    L[j] = L[j] * a + ml[j].y * b;
-                    O[j] = O[j] * a + oc[j] * b;
-                    M[j] = Mn;
+                for (int j = 0; j < B; ++j) {
+                    ml[k][j] = make_float2(-INFINITY, 0.f);
+                    oc[k][j] = 0.f;
+                    if (rp[j] && c0 + k < nne) {
+                        const float *r = rp[j] + (c0 + k) * cstride;
+                        ml[k][j] = __ldcg(reinterpret_cast<const float2 *>(r));
+                        oc[k][j] = __ldcg(r + eo[j]);
+                    }
                 }
+            if constexpr (K == 1) {
+#pragma unroll
+                for (int j = 0; j < B; ++j) {
+                    L[j] = ml[0][j].y;
+                    O[j] = oc[0][j];
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < K; ++k)
+#pragma unroll
+                    for (int j = 0; j < B; ++j) {
+                        if (rp[j] && c0 + k < nne) {
+                            const float Mn = fmaxf(M[j], ml[k][j].x);
+                            const float a = __expf(M[j] - Mn), b = __expf(ml[k][j].x - Mn);
+                            L[j] = L[j] * a + ml[k][j].y * b;
+                            O[j] = O[j] * a + oc[k][j] * b;
+                            M[j] = Mn;
+                        }
+                    }
             }
         }
 #pragma unroll
         for (int j = 0; j < B; ++j) {
             const int i = ct + (j0 + j) * kConsumerThreads;
-            if (i < N)
-                s.vec[i] = O[j] / L[j];
+            if (i < count)
+                out[i] = O[j] / L[j];
         }
+    }
+}
+
+// Attention task (KV head g, chunk c): its partial, then the arrival.  With
+// a single non-empty chunk (pos < chunk length) that chunk writes the output
+// itself.  Otherwise each non-empty chunk task of (layer, g) adds one to the
+// group's arrival counter with an acquire-release atomic behind its partial
+// stores (the barrier before it makes them the CTA's, the release makes
+// them visible first); the task that brings the count to this step's total
+// merges the group's partials into the attention output of its G heads (its
+// acquire orders those loads after every other chunk's stores).  The host
+// counts the arrivals each step expects: arrive_base + nne.
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v)
+{
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "l"(p), "r"(v)
+                 : "memory");
+    return old;
+}
+
+template <int E>
+__device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
+                                          const TaskDesc &d, const Geom &g, uint32_t &kc,
+                                          int ct, int warp, int lane, uint64_t *wt)
+{
+    if (!attn_chunk<E>(p, s, d, g, kc, ct, warp, lane, wt))
+        return false;
+    const int l = d.layer, gi = d.r0, C = p.attn_splits;
+    const int n = p.pos + 1;
+    const int chunk = (n + C - 1) / C;
+    const int nne = (n + chunk - 1) / chunk;  // non-empty chunks: 0 .. nne-1
+    if (nne == 1 || g.j1 <= g.j0)
+        return true;  // written directly, or empty
+    consumer_bar();  // every partial store of this task is issued
+    int *last = s.flags + 1;
+    if (ct == 0) {
+        const uint32_t old = atom_add_acq_rel(p.arrive + (size_t)l * p.n_kv_heads + gi, 1u);
+        *last = old == p.arrive_base + (uint32_t)(nne - 1);
+    }
+    consumer_bar();
+    if (*reinterpret_cast<volatile int *>(last)) {
+        const int hd = p.head_dim, G = p.group, N = p.n_heads * hd;
+        const float *part = p.part + (size_t)l * p.n_kv_heads * C * G * (hd + 2);
+        float *out = p.attn + (size_t)l * N + (size_t)gi * G * hd;
+        merge_batches<4, 4>(p, part, nne, gi * G * hd, G * hd, out, ct);
+    }
+    return true;
+}
+
+// O-projection prologue: the merged attention output of layer l -> vec
+// (one L2 round trip).  n_heads * head_dim <= kMaxPerThread * 256.
+__device__ void attn_prologue(const KParams &p, const SmemLayout &s, int l, int ct)
+{
+    const int N = p.n_heads * p.head_dim;
+    const float *src = p.attn + (size_t)l * N;
+    float v[kMaxPerThread];
+#pragma unroll
+    for (int j = 0; j < kMaxPerThread; ++j) {
+        const int i = ct + j * kConsumerThreads;
+        v[j] = i < N ? __ldcg(src + i) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxPerThread; ++j) {
+        const int i = ct + j * kConsumerThreads;
+        if (i < N)
+            s.vec[i] = v[j];
     }
     consumer_bar();
 }
@@ -1189,7 +1284,7 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
                     rmsnorm_prologue(p, s, p.xout + (size_t)(l - 1) * p.hidden, nullptr, gv, ct);
                 }
             } else if (d.kind == TK_OPROJ) {
-                combine_prologue(p, s, l, ct);
+                attn_prologue(p, s, l, ct);
             } else if (d.kind == TK_GATEUP) {
                 rmsnorm_prologue(p, s, p.xmid + (size_t)l * p.hidden, nullptr, gv, ct);
             } else if (d.kind == TK_DOWN) {

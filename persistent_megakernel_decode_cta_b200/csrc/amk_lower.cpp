@@ -138,17 +138,18 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     if (4 * hd > opt.stage_bytes)
         return amk_set_error(AMK_ERR_UNSUPPORTED, "head_dim too large for the ring stage");
 
+    // split-K chunks per KV head: as many as keep every attention task of a
+    // layer on its own SM, at most 8 (the merge of a head's chunks by the last
+    // one to finish then takes two L2 round trips)
     int C = opt.attn_splits;
-    if (C <= 0) {
-        const int by_sms = (n_sms + nkv - 1) / nkv;
-        const int by_combine = std::max(1, 65536 / (nh * (hd + 2) * 4));
-        C = std::max(1, std::min(by_sms, by_combine));
-    }
+    if (C <= 0)
+        C = std::max(1, std::min(n_sms / nkv, 8));
     C = std::min(C, c.max_ctx);
     // the shared vector holds a prologue's output: the normed hidden state,
-    // the combined attention output (+ per-head weights), or the attention
-    // tile's scratch; DOWN tiles read their activations from L2 directly
-    int vec = std::max({h, nh * hd + nh * C,
+    // the combined attention output (+ per-(head, chunk) m / weight and l),
+    // or the attention tile's scratch; DOWN tiles read their activations
+    // from L2 directly
+    int vec = std::max({h, nh * hd + 2 * nh * C,
                         G * hd + 2 * hd + amk::kConsumerWarps * G * (hd + 2)});
     vec = (vec + 3) & ~3;
     int stages = opt.ring_stages;
@@ -298,21 +299,25 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     }
     P->queue_off[n_sms] = (int32_t)P->tasks.size();
     P->n_counters = n_ctr;
+    P->n_arrive = L * nkv;
 
     // ---- the validator's graph ----------------------------------------------
     const int T = (int)P->tasks.size();
     auto B_QKV = [](int l) { return 6 * l + 0; };
-    auto B_PART = [](int l) { return 6 * l + 1; };
+    // the attention output of layer l: the ATTN tasks of KV head g accumulate
+    // the heads of g (their split-K partials are merged by whichever chunk
+    // task of g arrives last, an arrival-counter protocol inside the kernel:
+    // a commutative reduction, modelled as ACCUM)
+    auto B_ATTN = [](int l) { return 6 * l + 1; };
     auto B_XMID = [](int l) { return 6 * l + 2; };
     auto B_XOUT = [](int l) { return 6 * l + 3; };
     auto B_ACT = [](int l) { return 6 * l + 4; };
     auto B_KVNEW = [](int l) { return 6 * l + 5; };
     const int B_LOGITS = 6 * L, B_KEY = 6 * L + 1, B_KEYNEXT = 6 * L + 2;
     P->gbufs.assign(6 * L + 3, amk_graph_buffer{0, 0, -1});
-    const int64_t part_sz = (int64_t)nkv * C * G * (hd + 2);
     for (int l = 0; l < L; ++l) {
         P->gbufs[B_QKV(l)].size = P->qkv_rows;
-        P->gbufs[B_PART(l)].size = part_sz;
+        P->gbufs[B_ATTN(l)].size = (int64_t)nh * hd;
         P->gbufs[B_XMID(l)].size = h;
         P->gbufs[B_XOUT(l)].size = h;
         P->gbufs[B_ACT(l)].size = F;
@@ -363,14 +368,13 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
                     (int64_t)nh * hd + (g + 1) * hd);
                 acc(B_QKV(l), AMK_ACC_READ, (int64_t)(nh + nkv) * hd + g * hd,
                     (int64_t)(nh + nkv) * hd + (g + 1) * hd);
-                const int64_t slot = ((int64_t)g * C + ci) * G * (hd + 2);
-                acc(B_PART(l), AMK_ACC_WRITE, slot, slot + (int64_t)G * (hd + 2));
+                acc(B_ATTN(l), AMK_ACC_ACCUM, (int64_t)g * G * hd, (int64_t)(g + 1) * G * hd);
                 if (ci == 0)
                     acc(B_KVNEW(l), AMK_ACC_WRITE, (int64_t)g * 2 * hd, (int64_t)(g + 1) * 2 * hd);
                 break;
             }
             case amk::TK_OPROJ:
-                acc(B_PART(l), AMK_ACC_READ, 0, part_sz);
+                acc(B_ATTN(l), AMK_ACC_READ, 0, (int64_t)nh * hd);
                 if (l > 0)
                     acc(B_XOUT(l - 1), AMK_ACC_READ, d.r0, d.r1);
                 else

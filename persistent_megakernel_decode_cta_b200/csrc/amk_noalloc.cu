@@ -39,7 +39,7 @@ void *g_scratch_addr[kMaxDevices];  // device address of g_scratch, per device
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t tasks, qoff, ctr, err, argkey, qkv, part, xmid, xout, act, total;
+    size_t tasks, qoff, ctr, err, argkey, qkv, part, attn, xmid, xout, act, total;
 };
 
 Layout layout_of(const amk_plan &P)
@@ -56,11 +56,12 @@ Layout layout_of(const amk_plan &P)
     };
     o.tasks = take(sizeof(amk::TaskDesc) * P.tasks.size());
     o.qoff = take(sizeof(int32_t) * P.queue_off.size());
-    o.ctr = take(sizeof(uint32_t) * (size_t)P.n_counters);
+    o.ctr = take(sizeof(uint32_t) * (size_t)(P.n_counters + P.n_arrive));
     o.err = take(sizeof(amk::ErrorWord));
     o.argkey = take(2 * sizeof(unsigned long long));
     o.qkv = take(sizeof(float) * L * P.qkv_rows);
     o.part = take(sizeof(float) * L * part);
+    o.attn = take(sizeof(float) * L * c.n_heads * c.head_dim);
     o.xmid = take(sizeof(float) * L * c.hidden);
     o.xout = take(sizeof(float) * L * c.hidden);
     o.act = take(sizeof(float) * L * c.ffn);
@@ -182,6 +183,8 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     k.embed = static_cast<const uint16_t *>(w->embed);
     k.qkv = reinterpret_cast<float *>(base + lay.qkv);
     k.part = reinterpret_cast<float *>(base + lay.part);
+    k.attn = reinterpret_cast<float *>(base + lay.attn);
+    k.arrive = reinterpret_cast<uint32_t *>(base + lay.ctr) + P.n_counters;
     k.xmid = reinterpret_cast<float *>(base + lay.xmid);
     k.xout = reinterpret_cast<float *>(base + lay.xout);
     k.act = reinterpret_cast<float *>(base + lay.act);
@@ -213,6 +216,7 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     k.pos = pos;
     k.token = token_id;
     k.epoch = 0;   // counters were cleared above
+    k.arrive_base = 0;
     k.parity = 0;
     k.timeout_ns = (uint64_t)P.opt.wait_timeout_us * 1000ull;
     k.skip_signal_task = P.opt.debug_skip_signal_task;
