@@ -109,7 +109,9 @@ typedef struct {
     uint32_t wait_timeout_us; /* limit of every device-side wait */
     int32_t debug_skip_signal_task; /* test hook: this task id never signals; -1 = off */
     int32_t profile;          /* 1: record per-CTA phase timers (amk_get_profile) */
-    int32_t reserved[7];
+    int32_t l2_prefetch_kb;   /* while its ring is full, each SM prefetches this many KiB
+                                 of its coming weight stream into L2; 0 = off */
+    int32_t reserved[6];
 } amk_options;
 
 typedef struct amk_handle amk_handle;

@@ -11,6 +11,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -419,6 +420,7 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     k.generic = P->generic;
     k.timeout_ns = (uint64_t)P->opt.wait_timeout_us * 1000ull;
     k.skip_signal_task = P->opt.debug_skip_signal_task;
+    k.lookahead = (uint32_t)std::max(0, P->opt.l2_prefetch_kb) * 1024u;
     k.prof = H->d_prof;
     *out = H;
     return AMK_OK;

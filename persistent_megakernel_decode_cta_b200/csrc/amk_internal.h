@@ -118,6 +118,7 @@ struct KParams {
     uint32_t arrive_base;       // attention arrivals of earlier steps per (layer, kv head)
     int32_t parity;             // epoch & 1
     uint64_t timeout_ns;
+    uint32_t lookahead;         // L2 prefetch distance past the ring copies (bytes), 0 = off
     int32_t skip_signal_task;   // test hook, -1 = off
     unsigned long long *prof;   // [n_sms][kProfKinds][kProfFields] phase timers, or null
 };

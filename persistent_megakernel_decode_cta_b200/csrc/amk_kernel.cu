@@ -86,6 +86,12 @@ __device__ __forceinline__ void bulk_g2s_nohint(uint32_t dst, const void *src, u
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
+// Fetches [src, src + bytes) from HBM into L2 only (no shared-memory
+// destination, no completion tracking).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ uint64_t evict_first_policy()
 {
     uint64_t pol;
@@ -418,6 +424,79 @@ __device__ __forceinline__ Geom task_geom(const KParams &p, const TaskDesc &d)
 }
 
 // ------------------------------------------------------------------ producer
+// L2 lookahead (optional).  A task's byte stream is at most two contiguous
+// regions (the rows of a GEMV tile, or of its gate and up halves; the K and
+// V rows of an attention chunk range), copied into the ring in that order.
+// While the ring is full -- typically while the consumers wait at a level
+// boundary -- the producer walks a second cursor over the same streams and
+// prefetches up to `lookahead` bytes past its copy cursor into L2, so that
+// HBM keeps streaming and the ring refills from L2 once the consumers resume.
+struct Lookahead {
+    const uint8_t *a, *b;  // regions of the cursor's task
+    uint32_t na, nb;
+    uint32_t off;          // bytes of the current region already passed
+    int ti;                // task of the cursor (qe: end of the queue)
+    int part;              // 0: region a, 1: region b, 2: task exhausted
+    uint64_t pos;          // stream position of the cursor
+};
+
+__device__ __forceinline__ void lookahead_load(const KParams &p, Lookahead &la)
+{
+    const uint8_t *rec = reinterpret_cast<const uint8_t *>(p.tasks + la.ti);
+    TaskDesc d{};
+    d.kind = (uint8_t)__ldg(reinterpret_cast<const uint32_t *>(rec));
+    const int4 q = __ldg(reinterpret_cast<const int4 *>(rec + 16));  // ..., r0, r1
+    const longlong2 w = __ldg(reinterpret_cast<const longlong2 *>(rec + 32));  // w0, w1
+    d.r0 = q.z;
+    d.r1 = q.w;
+    const Geom g = task_geom(p, d);
+    const uint8_t *w0 = reinterpret_cast<const uint8_t *>(w.x);
+    const uint8_t *w1 = reinterpret_cast<const uint8_t *>(w.y);
+    if (d.kind == TK_ATTN) {
+        const size_t o = (size_t)g.pa * p.head_dim * 2;
+        la.a = w0 + o;
+        la.b = w1 + o;
+        la.na = la.nb = (uint32_t)(g.pb - g.pa) * p.head_dim * 2;
+    } else {
+        la.a = w0;
+        la.b = w1;
+        la.na = (uint32_t)g.R * g.RB;
+        la.nb = g.nchunks > g.nck ? la.na : 0u;
+    }
+    la.part = 0;
+    la.off = 0;
+}
+
+// Advances the cursor to stream position `hi`, prefetching the bytes at or
+// past `lo` (the copy cursor: bytes before it are in the ring already).
+__device__ __forceinline__ void lookahead_pump(const KParams &p, Lookahead &la, int qe,
+                                               uint64_t lo, uint64_t hi)
+{
+    constexpr uint32_t kPiece = 32768;
+    while (la.pos < hi && la.ti < qe) {
+        if (la.part >= 2) {
+            if (++la.ti >= qe)
+                return;
+            lookahead_load(p, la);
+            continue;
+        }
+        const uint8_t *base = la.part ? la.b : la.a;
+        const uint32_t n = la.part ? la.nb : la.na;
+        if (la.off >= n) {
+            ++la.part;
+            la.off = 0;
+            continue;
+        }
+        uint32_t piece = min(n - la.off, kPiece);
+        if (la.pos < lo)  // already copied: skip without prefetching
+            piece = (uint32_t)min((uint64_t)piece, lo - la.pos);
+        else
+            bulk_prefetch_l2(base + la.off, piece);
+        la.off += piece;
+        la.pos += piece;
+    }
+}
+
 // Lane 0 of the producer warpgroup streams every chunk of every task of this
 // SM's queue into the ring, one task record ahead.
 __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int qe)
@@ -428,6 +507,10 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
     volatile int *abort_flag = s.flags;
     bool stop = false;
     uint64_t prof_wait = 0, prof_bytes = 0, prof_setup = 0;
+    uint64_t cpos = 0;  // stream position of the copy cursor
+    Lookahead la{};
+    la.ti = qb - 1;
+    la.part = 2;
     if (qb < qe)
         stage_task(s.ptask_a, p.tasks + qb);
     for (int ti = qb; ti < qe && !stop; ++ti) {
@@ -447,8 +530,11 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
                 uint32_t it = 0;
                 uint64_t t0 = 0;
                 while (!mbar_try_wait(s.empty_a + 8 * st, par)) {
-                    if (it == 0)
+                    if (it == 0) {
                         t0 = gtimer();
+                        if (p.lookahead)
+                            lookahead_pump(p, la, qe, cpos, cpos + p.lookahead);
+                    }
                     if ((++it & 255) == 0) {
                         if (*abort_flag || gtimer() - t0 > p.timeout_ns * 4 ||
                             it > (1u << 30)) {
@@ -475,6 +561,7 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
                 bulk_g2s_nohint(dst + (uint32_t)g.P * p.head_dim * 2,
                                 w1 + (size_t)a * p.head_dim * 2, nb, bar);
                 prof_bytes += 2 * nb;
+                cpos += 2 * nb;
             } else {
                 const int part = i / g.nck, c = i % g.nck;
                 const int r = c * g.rpc;
@@ -483,6 +570,7 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
                 mbar_arrive_expect_tx(bar, nb);
                 bulk_g2s(dst, (part ? w1 : w0) + (size_t)r * g.RB, nb, bar, pol_w);
                 prof_bytes += nb;
+                cpos += nb;
             }
         }
     }

@@ -80,6 +80,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         if (opt_in->wait_timeout_us > 0) opt.wait_timeout_us = opt_in->wait_timeout_us;
         opt.debug_skip_signal_task = opt_in->debug_skip_signal_task;
         opt.profile = opt_in->profile;
+        if (opt_in->l2_prefetch_kb > 0) opt.l2_prefetch_kb = opt_in->l2_prefetch_kb;
         opt.n_sms = opt_in->n_sms;
     }
     const amk_config &c = *cfg;
