@@ -417,6 +417,7 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     k.att_lph = P->att_lph;
     k.att_hpb = P->att_hpb;
     k.att_e = P->att_e;
+    k.att_pg = P->att_pg;
     k.generic = P->generic;
     k.timeout_ns = (uint64_t)P->opt.wait_timeout_us * 1000ull;
     k.skip_signal_task = P->opt.debug_skip_signal_task;

@@ -111,6 +111,7 @@ struct KParams {
     int32_t ring_stages, stage_bytes, vec_floats;
     // attention lane layout
     int32_t att_lph, att_hpb, att_e;  // lanes per head, heads per batch, elems per lane
+    int32_t att_pg;                   // position groups per warp (lph * G lanes each)
     int32_t generic;            // 1: run the generic kernel instance
     // step
     int32_t pos, token;         // token < 0: previous step's argmax

@@ -921,7 +921,7 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
 {
     const int l = d.layer, gi = d.r0, c = d.r1;
     const int hd = p.head_dim, G = p.group, nh = p.n_heads, nkv = p.n_kv_heads;
-    const int lph = p.att_lph;
+    const int lph = p.att_lph;  // lanes per head
     float *qs = s.vec;                       // [G][hd], RoPE'd and pre-scaled
     float *kn = qs + G * hd;                 // [hd] new K row (bf16 value)
     float *vn = kn + hd;                     // [hd] new V row (bf16 value)
@@ -966,20 +966,41 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
             vd[i] = vb;
     }
     consumer_bar();
-    // lane layout: head jh = lane / lph (within the group), elements
-    // [e0, e0 + E) of that head
-    const int jh = lane / lph;
-    const int e0 = (lane % lph) * E;
-    const bool active = jh < G;
+    // lane layout: lph lanes per head hold E = hd / lph of its elements; the
+    // G heads of the group take lph * G lanes, and the warp's 32 lanes hold
+    // PG such groups, each scoring a different position at the same time.
+    // Lane li of a head holds, for E >= 8, the 8-element pieces (k lph + li)
+    // (so that 8 neighbouring lanes read 128 contiguous bytes of a row, free
+    // of bank conflicts), else elements [li E, li E + E).
+    const int PG = p.att_pg;
+    const int pg = lane / (lph * G), jh = (lane / lph) % G, li = lane % lph;
+    const bool active = pg < PG;
+    auto elem = [&](int k) { return E >= 8 ? ((k / 8) * lph + li) * 8 + (k % 8) : li * E + k; };
+    // E bf16 values of the lane from the row at shared address row
+    auto ldrow = [&](uint32_t row, float(&out)[E]) {
+        if constexpr (E >= 8) {
+#pragma unroll
+            for (int c8 = 0; c8 < E / 8; ++c8) {
+                float t[8];
+                lds_bf16<8>(row + (uint32_t)((c8 * lph + li) * 16), t);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    out[c8 * 8 + u] = t[u];
+            }
+        } else {
+            lds_bf16<E>(row + (uint32_t)(li * E * 2), out);
+        }
+    };
     float q[E], o[E];
     float m = -INFINITY, lsum = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-        q[e] = active ? qs[jh * hd + e0 + e] : 0.f;
+        q[e] = active ? qs[jh * hd + elem(e)] : 0.f;
         o[e] = 0.f;
     }
     bool fail = false;
     uint64_t tA = 0, tB = 0;
+    const int gstride = kConsumerWarps * PG;  // positions between a group's batches
     for (int i = 0; i < g.nchunks; ++i) {
         if (wt)
             tA = gtimer();
@@ -991,20 +1012,19 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
             tB = gtimer();
             wt[0] += tB - tA;
         }
-        const uint32_t ka = s.ring_a + (uint32_t)(kc % p.ring_stages) * p.stage_bytes +
-                            (uint32_t)e0 * 2;
+        const uint32_t ka = s.ring_a + (uint32_t)(kc % p.ring_stages) * p.stage_bytes;
         const uint32_t va = ka + (uint32_t)g.P * hd * 2;
         const int a = g.pa + i * g.P;
         const int n = min(g.P, g.pb - a);
-        // four positions per warp at a time: independent dot products and
-        // shuffle reductions, then one online-softmax update
-        for (int j0 = warp; j0 < n; j0 += 4 * kConsumerWarps) {
+        // four positions per group at a time (4 PG per warp): independent dot
+        // products and shuffle reductions, then one online-softmax update
+        for (int j0 = warp; j0 < n; j0 += 4 * gstride) {
             float sc[4];
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-                const int j = j0 + b * kConsumerWarps;
+                const int j = j0 + kConsumerWarps * pg + b * gstride;
                 float kv_[E];
-                lds_bf16<E>(ka + (uint32_t)(j < n ? j : j0) * hd * 2, kv_);
+                ldrow(ka + (uint32_t)(j < n ? j : j0) * hd * 2, kv_);
                 float d_ = 0.f;
 #pragma unroll
                 for (int e = 0; e < E; ++e)
@@ -1019,10 +1039,12 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
             float mn = m;
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-                if (j0 + b * kConsumerWarps >= n)
+                if (!active || j0 + kConsumerWarps * pg + b * gstride >= n)
                     sc[b] = -INFINITY;
                 mn = fmaxf(mn, sc[b]);
             }
+            if (mn == -INFINITY)  // this group has no position in the batch
+                continue;
             const float corr = __expf(m - mn);
             float pr[4];
             lsum *= corr;
@@ -1036,10 +1058,10 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
                 o[e] *= corr;
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-                const int j = j0 + b * kConsumerWarps;
-                if (j < n) {
+                const int j = j0 + kConsumerWarps * pg + b * gstride;
+                if (active && j < n) {
                     float vv[E];
-                    lds_bf16<E>(va + (uint32_t)j * hd * 2, vv);
+                    ldrow(va + (uint32_t)j * hd * 2, vv);
 #pragma unroll
                     for (int e = 0; e < E; ++e)
                         o[e] = fmaf(pr[b], vv[e], o[e]);
@@ -1058,29 +1080,56 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
     if (*reinterpret_cast<volatile int *>(s.flags))
         return false;
     if (g.j0 <= p.pos && p.pos < g.j1 && warp == 0) {
-        // the new position: K and V rows of this step (bf16 values as floats)
+        // the new position: K and V rows of this step (bf16 values as
+        // floats), taken by position group 0
         float sc = 0.f;
 #pragma unroll
         for (int e = 0; e < E; ++e)
-            sc = fmaf(q[e], kn[e0 + e], sc);
+            sc = fmaf(q[e], kn[elem(e)], sc);
         for (int off = lph >> 1; off > 0; off >>= 1)
             sc += __shfl_xor_sync(0xffffffffu, sc, off);
-        const float mn = fmaxf(m, sc);
-        const float corr = __expf(m - mn);
-        const float pr = __expf(sc - mn);
-        lsum = lsum * corr + pr;
+        if (pg == 0) {
+            const float mn = fmaxf(m, sc);
+            const float corr = __expf(m - mn);
+            const float pr = __expf(sc - mn);
+            lsum = lsum * corr + pr;
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                o[e] = o[e] * corr + pr * vn[elem(e)];
+            m = mn;
+        }
+    }
+    // merge the position groups of the warp into group 0, as a tree: group
+    // pg takes group pg + st (lanes st lph G further on hold the same head
+    // elements) when pg is a multiple of 2 st; a group that saw no position
+    // has m = -inf, l = 0
+    for (int st = 1; st < PG; st <<= 1) {
+        const int src = min(lane + st * lph * G, 31);
+        const bool take = active && pg % (2 * st) == 0 && pg + st < PG;
+        const float m2 = __shfl_sync(0xffffffffu, m, src);
+        const float l2 = __shfl_sync(0xffffffffu, lsum, src);
+        float ob[E];
 #pragma unroll
         for (int e = 0; e < E; ++e)
-            o[e] = o[e] * corr + pr * vn[e0 + e];
-        m = mn;
+            ob[e] = __shfl_sync(0xffffffffu, o[e], src);
+        if (take) {
+            const float mn = fmaxf(m, m2);
+            const float fa = m == -INFINITY ? 0.f : __expf(m - mn);
+            const float fb = m2 == -INFINITY ? 0.f : __expf(m2 - mn);
+            lsum = lsum * fa + l2 * fb;
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                o[e] = o[e] * fa + ob[e] * fb;
+            m = mn;
+        }
     }
     // per-warp state -> ws[w][jh][hd + 2]
     float *mine = ws + (size_t)warp * G * (hd + 2);
-    if (active) {
+    if (pg == 0) {
 #pragma unroll
         for (int e = 0; e < E; ++e)
-            mine[jh * (hd + 2) + 2 + e0 + e] = o[e];
-        if (lane % lph == 0) {
+            mine[jh * (hd + 2) + 2 + elem(e)] = o[e];
+        if (li == 0) {
             mine[jh * (hd + 2) + 0] = m;
             mine[jh * (hd + 2) + 1] = lsum;
         }

@@ -103,10 +103,18 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         return amk_set_error(AMK_ERR_INVALID_ARG, "ring_stages in [2,%d], stage_bytes a "
                              "multiple of 1024", amk::kMaxStages);
     const int G = nh / nkv;
-    // attention lane layout: lph lanes per head, E elements per lane
+    // attention lane layout: lph lanes per head, E = hd / lph elements per
+    // lane, the G heads of a group side by side, and as many position groups
+    // of lph * G lanes as fit a warp.  By default the heads spread over the
+    // warp (lph = largest power of two with lph * G <= 32); heads of 128 or
+    // more elements take 16 per lane instead, so that a warp scores several
+    // positions at once with fewer shuffle steps (measured: faster for
+    // Llama-7B shapes, slower for short chunks of 64-element heads)
     int lph = 32;
     while (lph > 1 && (lph * G > 32 || hd % lph))
         lph >>= 1;
+    if (hd >= 128 && hd % 16 == 0 && hd / lph < 16)
+        lph = hd / 16;
     const int att_e = hd / lph;
     if (h > 16 * 256 || nh * hd > 16 * 256 || F > 3 * 16 * 256 * 4)
         return amk_set_error(AMK_ERR_UNSUPPORTED, "hidden or heads*head_dim above 4096, or ffn "
@@ -171,6 +179,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     P->smem_bytes = smem;
     P->att_lph = lph;
     P->att_hpb = 32 / lph;
+    P->att_pg = std::max(1, 32 / (lph * G));
     P->att_e = hd / lph;
     P->generic = (c.tied_embeddings && c.quant == AMK_QUANT_W8A16) ? 1 : 0;
     for (const Mat &m : mats)

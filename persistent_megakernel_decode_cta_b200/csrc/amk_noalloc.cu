@@ -212,6 +212,7 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     k.att_lph = P.att_lph;
     k.att_hpb = P.att_hpb;
     k.att_e = P.att_e;
+    k.att_pg = P.att_pg;
     k.generic = P.generic;
     k.pos = pos;
     k.token = token_id;

@@ -18,7 +18,8 @@ struct amk_plan {
     std::vector<amk::TaskDesc> tasks;  // grouped by SM, queue order
     std::vector<int32_t> queue_off;    // [n_sms + 1]
     int n_counters = 0;  // level counters (the validator's graph)
-    int n_arrive = 0;    // attention arrival counters, [L][nkv], after them
+    int n_arrive = 0;
+    int att_pg = 1;      // attention position groups per warp    // attention arrival counters, [L][nkv], after them
     // the validator's view
     std::vector<amk_graph_task> gtasks;
     std::vector<amk_graph_wait> gwaits;
