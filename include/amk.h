@@ -111,7 +111,14 @@ typedef struct {
     int32_t profile;          /* 1: record per-CTA phase timers (amk_get_profile) */
     int32_t l2_prefetch_kb;   /* while its ring is full, each SM prefetches this many KiB
                                  of its coming weight stream into L2; 0 = off */
-    int32_t reserved[6];
+    int32_t ffn_fused;        /* one FFN level per layer: gate/up, SwiGLU and the matching
+                                 Wdown columns in one task, the slices' down projections
+                                 summed into the residual in 64-bit fixed point (amk_create
+                                 keeps a packed copy of every Wdown for it).  1 (default):
+                                 when the shape allows and hidden * element size <= 2 KB;
+                                 2: whenever the shape allows; -1: separate gate/up and
+                                 down levels */
+    int32_t reserved[5];
 } amk_options;
 
 typedef struct amk_handle amk_handle;

@@ -45,7 +45,7 @@ class Options(ctypes.Structure):
     _fields_ = [("ring_stages", c_i32), ("stage_bytes", c_i32), ("attn_splits", c_i32),
                 ("tasks_per_sm", c_i32), ("n_sms", c_i32), ("wait_timeout_us", c_u32),
                 ("debug_skip_signal_task", c_i32), ("profile", c_i32),
-                ("l2_prefetch_kb", c_i32), ("reserved", c_i32 * 6)]
+                ("l2_prefetch_kb", c_i32), ("ffn_fused", c_i32), ("reserved", c_i32 * 5)]
 
 
 class GraphWait(ctypes.Structure):

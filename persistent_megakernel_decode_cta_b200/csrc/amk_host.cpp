@@ -25,6 +25,8 @@ using amk::KParams;
 using amk::TaskDesc;
 
 extern "C" cudaError_t amk_kernel_configure(int smem_bytes, int quant, int att_e, int generic);
+extern "C" cudaError_t amk_pack_down(const void *wd, void *out, int h, int ffn, int esz,
+                                     cudaStream_t stream);
 extern "C" cudaError_t amk_kernel_occupancy(int smem_bytes, int quant, int att_e, int generic,
                                             int *blocks_per_sm);
 namespace amk {
@@ -79,6 +81,7 @@ extern "C" int amk_default_options(amk_options *o)
     o->n_sms = 0;
     o->wait_timeout_us = 1000000;  // 1 s
     o->debug_skip_signal_task = -1;
+    o->ffn_fused = 1;
     return AMK_OK;
 }
 
@@ -146,6 +149,9 @@ struct amk_handle {
           *d_xout = nullptr;
     float *d_act = nullptr, *d_logits = nullptr;
     unsigned long long *d_argkey = nullptr;
+    long long *d_xacc = nullptr;    // [L][h] fixed-point residual (fused FFN)
+    void *d_act_block = nullptr;    // every activation buffer, one allocation
+    void *d_dpack = nullptr;        // [L] packed Wdown (fused FFN), see KParams::dpack
     unsigned long long *d_prof = nullptr;
     uint16_t *d_kv = nullptr;
     size_t kv_bytes = 0, act_bytes = 0;
@@ -247,7 +253,7 @@ int zero_state(amk_handle *H)
     if (e == cudaSuccess)
         e = cudaMemsetAsync(H->d_argkey, 0, 2 * sizeof(unsigned long long), H->stream);
     if (e == cudaSuccess)
-        e = cudaMemsetAsync(H->d_qkv, 0, H->act_bytes, H->stream);
+        e = cudaMemsetAsync(H->d_act_block, 0, H->act_bytes, H->stream);
     if (e != cudaSuccess)
         return cuda_fail(e, "amk_reset_kv");
     H->epoch = 0;
@@ -332,8 +338,9 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     const size_t attn_f = (size_t)L * c.n_heads * hd;
     const size_t h_f = (size_t)L * c.hidden, act_f = (size_t)L * c.ffn;
     H->kv_bytes = (size_t)L * 2 * nkv * c.max_ctx * hd * sizeof(uint16_t);
-    // activations in one block: qkv | part | attn | xmid | xout | act
-    H->act_bytes = (qkv_f + part_f + attn_f + 2 * h_f + act_f) * sizeof(float);
+    // activations in one block: xacc (int64) | qkv | part | attn | xmid | xout | act
+    const size_t xacc_b = P->ffn_fused ? (size_t)L * c.hidden * sizeof(long long) : 0;
+    H->act_bytes = xacc_b + (qkv_f + part_f + attn_f + 2 * h_f + act_f) * sizeof(float);
     float *act_block = nullptr;
     if ((rc = dalloc(H, &H->d_tasks, sizeof(TaskDesc) * P->tasks.size())) ||
         (rc = dalloc(H, &H->d_qoff, sizeof(int32_t) * P->queue_off.size())) ||
@@ -342,6 +349,8 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
         (rc = dalloc(H, &act_block, H->act_bytes)) ||
         (rc = dalloc(H, &H->d_logits, sizeof(float) * (size_t)c.vocab)) ||
         (rc = dalloc(H, &H->d_argkey, 2 * sizeof(unsigned long long))) ||
+        (P->ffn_fused &&
+         (rc = dalloc(H, &H->d_dpack, (size_t)L * c.hidden * c.ffn * (q8 ? 1 : 2)))) ||
         (rc = dalloc(H, &H->d_kv, H->kv_bytes)) ||
         (P->opt.profile &&
          (rc = dalloc(H, &H->d_prof, sizeof(unsigned long long) * (size_t)n_sms *
@@ -349,7 +358,9 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
         free_handle(H);
         return rc;
     }
-    H->d_qkv = act_block;
+    H->d_act_block = act_block;
+    H->d_xacc = P->ffn_fused ? reinterpret_cast<long long *>(act_block) : nullptr;
+    H->d_qkv = reinterpret_cast<float *>(reinterpret_cast<char *>(act_block) + xacc_b);
     H->d_part = H->d_qkv + qkv_f;
     H->d_attn = H->d_part + part_f;
     H->d_xmid = H->d_attn + attn_f;
@@ -364,6 +375,15 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     std::vector<TaskDesc> resolved(P->tasks.size());
     for (size_t t = 0; t < resolved.size(); ++t)
         amk_resolve_task(P, w, H->d_kv, (int)t, &resolved[t]);
+    // fused FFN: the handle's packed copy of every layer's Wdown
+    for (int l = 0; P->ffn_fused && l < L; ++l) {
+        const size_t lb = (size_t)c.hidden * c.ffn * (q8 ? 1 : 2);
+        if ((e = amk_pack_down(w->wdown[l], static_cast<uint8_t *>(H->d_dpack) + l * lb,
+                               c.hidden, c.ffn, q8 ? 1 : 2, H->stream)) != cudaSuccess) {
+            free_handle(H);
+            return cuda_fail(e, "pack Wdown");
+        }
+    }
     if ((e = cudaMemcpyAsync(H->d_tasks, resolved.data(), sizeof(TaskDesc) * resolved.size(),
                              cudaMemcpyHostToDevice, H->stream)) != cudaSuccess ||
         (e = cudaMemcpyAsync(H->d_qoff, P->queue_off.data(),
@@ -393,6 +413,11 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     k.xmid = H->d_xmid;
     k.xout = H->d_xout;
     k.act = H->d_act;
+    k.xacc = H->d_xacc;
+    k.dmaps = nullptr;
+    k.dpack = static_cast<const uint8_t *>(H->d_dpack);
+    k.ffn_fused = P->ffn_fused;
+    k.ffn_box_rows = P->ffn_box_rows;
     k.logits = H->d_logits;
     k.argkey = H->d_argkey;
     k.kv = H->d_kv;

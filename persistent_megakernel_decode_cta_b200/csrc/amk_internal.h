@@ -46,6 +46,9 @@ enum TaskKind : uint8_t {
     TK_GATEUP = 4,  // rows of Wgate and Wup, RMSNorm prologue, SwiGLU epilogue
     TK_DOWN = 5,    // rows of Wdown, residual epilogue
     TK_LMHEAD = 6,  // rows of the LM head, final RMSNorm prologue, argmax epilogue
+    TK_FFN = 7,     // FFN slice [r0, r1): RMSNorm prologue, rows of Wgate and Wup, SwiGLU,
+                    // then the columns [r0, r1) of Wdown (2-D TMA boxes); the partial
+                    // down projection is added into the layer's fixed-point residual
 };
 
 enum TaskFlags : uint8_t {
@@ -65,7 +68,7 @@ struct TaskDesc {           // 80 bytes, read-only for the kernel
                             //   block of (layer, g)
     const uint16_t *s0, *s1;  // fp16 row scales at row r0 (W8A16), or null
     const uint16_t *gain;     // RMSNorm gain of the prologue, or null
-    uint64_t pad2;
+    const uint16_t *s2;       // TK_FFN: fp16 row scales of Wdown [hidden] (W8A16), or null
 };
 static_assert(sizeof(TaskDesc) == 80, "TaskDesc is 80 bytes");
 
@@ -100,6 +103,12 @@ struct KParams {
     float *xmid;      // [L][h]: residual after attention
     float *xout;      // [L][h]: residual after the FFN
     float *act;       // [L][ffn]: SwiGLU activations
+    long long *xacc;  // [L][h]: residual after the FFN in fixed point (value * 2^32), when
+                      // the FFN level is fused: OPROJ writes the residual, FFN slices add
+    const void *dmaps;  // [L] 128-byte tensor maps of Wdown (fused FFN), 64-byte aligned
+    const uint8_t *dpack;  // fused FFN: Wdown of every layer packed in 16-byte column
+                           // groups, [L][ffn * esz / 16][hidden][16 B], or null: the
+                           // tensor maps read the caller's Wdown
     float *logits;    // [vocab]
     unsigned long long *argkey;  // [2] packed (ordered logit << 32 | ~index)
     uint16_t *kv;     // bf16 [L][2][nkv][max_ctx][hd]
@@ -113,6 +122,7 @@ struct KParams {
     int32_t att_lph, att_hpb, att_e;  // lanes per head, heads per batch, elems per lane
     int32_t att_pg;                   // position groups per warp (lph * G lanes each)
     int32_t generic;            // 1: run the generic kernel instance
+    int32_t ffn_fused, ffn_box_rows;
     // step
     int32_t pos, token;         // token < 0: previous step's argmax
     uint32_t epoch;             // steps since reset (counter targets)

@@ -86,6 +86,19 @@ __device__ __forceinline__ void bulk_g2s_nohint(uint32_t dst, const void *src, u
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
+// Tiled 2-D TMA load of the box at (x, y) of the tensor map at tmap (a
+// generic address of a 64-byte aligned CUtensorMap in global memory) into
+// shared memory, completing on the mbarrier bar.  No multicast.  x (the
+// innermost coordinate) times the element size is a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int x, int y,
+                                            uint32_t bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(tmap), "r"(x), "r"(y), "r"(bar), "l"(policy)
+        : "memory");
+}
 // Fetches [src, src + bytes) from HBM into L2 only (no shared-memory
 // destination, no completion tracking).
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes)
@@ -113,6 +126,18 @@ __device__ __forceinline__ uint32_t ld_relaxed(const uint32_t *p)
 __device__ __forceinline__ void red_release_add(uint32_t *p, uint32_t v)
 {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// The residual after a fused FFN level is held in fixed point (value * 2^32
+// in an int64): integer addition is associative, so the FFN slices' partial
+// down projections add up to the same bits in any order.  |value| < 2^31.
+__device__ __forceinline__ long long to_fix(float v) { return __float2ll_rn(v * 4294967296.0f); }
+__device__ __forceinline__ float from_fix(long long a)
+{
+    return (float)((double)a * (1.0 / 4294967296.0));
+}
+__device__ __forceinline__ void red_add_fix(long long *p, long long v)
+{
+    asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 __device__ __forceinline__ uint64_t gtimer()
 {
@@ -355,8 +380,13 @@ __device__ __forceinline__ TaskDesc read_staged(uint32_t slot)
 // record with this function (no memory reads), so they agree on every chunk.
 struct Geom {
     int nchunks;
+    int ngu;  // chunks of the row-GEMV parts (all of them but a fused FFN's Wdown part)
     // GEMV tiles
     int K, esz, RB, rpc, R, nck;
+    // fused FFN, Wdown part: the slice's columns in boxes of 16 bytes x BR rows;
+    // chunk c covers rows [c rpc2, min(h, (c + 1) rpc2)), rpc2 a multiple of 256
+    // or all of h
+    int ncb, rpc2, nck2;
     int VB, KS, RG;  // vector bytes; warps split K into KS slices x RG row groups
     // attention tiles
     int j0, j1, pa, pb, P;
@@ -392,7 +422,7 @@ __device__ __forceinline__ Geom task_geom(const KParams &p, const TaskDesc &d)
         K = p.n_heads * p.head_dim;
     else if (d.kind == TK_DOWN)
         K = p.ffn;
-    else if (d.kind == TK_GATEUP)
+    else if (d.kind == TK_GATEUP || d.kind == TK_FFN)
         parts = 2;
     else if (d.kind == TK_LMHEAD && p.tied)
         esz = 2;
@@ -420,6 +450,19 @@ __device__ __forceinline__ Geom task_geom(const KParams &p, const TaskDesc &d)
     g.R = d.r1 - d.r0;
     g.nck = (g.R + rpc - 1) / rpc;
     g.nchunks = g.nck * parts;
+    g.ngu = g.nchunks;
+    if (d.kind == TK_FFN) {
+        const int row_bytes = g.R * esz, br = p.ffn_box_rows;
+        g.ncb = row_bytes / 16;
+        if (p.dpack) {  // contiguous column groups: any row count per chunk
+            g.rpc2 = min(p.hidden, p.stage_bytes / row_bytes);
+        } else {        // TMA boxes of br rows
+            const int fit = (p.stage_bytes / (row_bytes * br)) * br;  // rows per stage
+            g.rpc2 = fit >= p.hidden ? p.hidden : fit / 256 * 256;
+        }
+        g.nck2 = (p.hidden + g.rpc2 - 1) / g.rpc2;
+        g.nchunks += g.nck2;
+    }
     return g;
 }
 
@@ -562,6 +605,33 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
                                 w1 + (size_t)a * p.head_dim * 2, nb, bar);
                 prof_bytes += 2 * nb;
                 cpos += 2 * nb;
+            } else if (i >= g.ngu) {
+                // fused FFN, Wdown part: rows [r0w, r0w + nrows) of the slice's
+                // 16-byte column groups jb, at (jb nrows + row) * 16 in the stage:
+                // one bulk copy per group from the packed copy, or TMA boxes of
+                // 16 bytes x br rows from the caller's Wdown
+                const int r0w = (i - g.ngu) * g.rpc2;
+                const int nrows = min(g.rpc2, p.hidden - r0w);
+                const uint32_t nb = (uint32_t)(nrows * g.ncb * 16);
+                mbar_arrive_expect_tx(bar, nb);
+                if (p.dpack) {
+                    const uint8_t *src = p.dpack + (size_t)d.layer * p.hidden * p.ffn * g.esz +
+                                         ((size_t)(d.r0 / (16 / g.esz)) * p.hidden + r0w) * 16;
+                    for (int jb = 0; jb < g.ncb; ++jb)
+                        bulk_g2s(dst + (uint32_t)(jb * nrows * 16),
+                                 src + (size_t)jb * p.hidden * 16, (uint32_t)nrows * 16, bar,
+                                 pol_w);
+                } else {
+                    const int br = p.ffn_box_rows;
+                    const void *tmap =
+                        static_cast<const uint8_t *>(p.dmaps) + (size_t)d.layer * 128;
+                    for (int ib = 0; ib < nrows / br; ++ib)
+                        for (int jb = 0; jb < g.ncb; ++jb)
+                            tma_load_2d(dst + (uint32_t)((jb * nrows + ib * br) * 16), tmap,
+                                        d.r0 + jb * (16 / g.esz), r0w + ib * br, bar, pol_w);
+                }
+                prof_bytes += nb;
+                cpos += nb;
             } else {
                 const int part = i / g.nck, c = i % g.nck;
                 const int r = c * g.rpc;
@@ -690,8 +760,8 @@ __device__ float block_sum(float v, const SmemLayout &s, int ct)
 // L2 round trip); hidden <= kMaxPerThread * 256.
 constexpr int kMaxPerThread = 16;
 __device__ void rmsnorm_prologue(const KParams &p, const SmemLayout &s, const float *x_f32,
-                                 const uint16_t *x_bf16, const float (&gv)[kMaxPerThread],
-                                 int ct)
+                                 const uint16_t *x_bf16, const long long *x_fix,
+                                 const float (&gv)[kMaxPerThread], int ct)
 {
     const int n = p.hidden;
     float xv[kMaxPerThread];
@@ -700,7 +770,8 @@ __device__ void rmsnorm_prologue(const KParams &p, const SmemLayout &s, const fl
         const int i = ct + j * kConsumerThreads;
         xv[j] = 0.f;
         if (i < n)
-            xv[j] = x_f32 ? __ldcg(x_f32 + i) : bf16_to_f(__ldg(x_bf16 + i));
+            xv[j] = x_f32 ? __ldcg(x_f32 + i)
+                          : x_fix ? from_fix(__ldcg(x_fix + i)) : bf16_to_f(__ldg(x_bf16 + i));
     }
     float ss = 0.f;
 #pragma unroll
@@ -762,7 +833,7 @@ __device__ __forceinline__ bool gemv_task(const KParams &p, const SmemLayout &s,
     const uint32_t red_a = s.red_a + (uint32_t)warp * kMaxTaskRows * 4;
     const int NS = p.ring_stages, SB = p.stage_bytes;
     uint64_t tA = 0, tB = 0;
-    for (int i = 0; i < g.nchunks; ++i) {
+    for (int i = 0; i < g.ngu; ++i) {
         if (wt)
             tA = gtimer();
         if (!wait_full(p, s, kc))
@@ -1337,6 +1408,75 @@ __device__ int resolve_token(const KParams &p)
     return t;
 }
 
+// Fused FFN, after its gate/up GEMV: the slice's SwiGLU activations
+// act[j] = silu(gate_j) up_j go to vec[0, R); then the slice's columns of
+// Wdown stream through the ring, 16-byte column group jb of chunk row lr at
+// (jb nrows + lr) * 16 of the stage.  Thread t owns the rows t + 256 k of
+// each chunk: it forms sum_j W[row][r0 + j] act[j] (times the row's int8
+// scale, loaded before the chunk's ring wait) and adds it into the layer's
+// fixed-point residual.  The 16-byte pieces a warp reads at once are
+// consecutive: free of bank conflicts.
+template <int ESZ>
+__device__ __forceinline__ bool ffn_down_part(const KParams &p, const SmemLayout &s,
+                                              const Geom &g, const TaskDesc &d, uint32_t &kc,
+                                              int ct, int lane)
+{
+    constexpr int E = 16 / ESZ;  // elements per box row
+    const int ncb = g.ncb, h = p.hidden;
+    long long *acc_out = p.xacc + (size_t)d.layer * h;
+    for (int c2 = 0; c2 < g.nck2; ++c2) {
+        const int r0w = c2 * g.rpc2, nrows = min(g.rpc2, h - r0w);
+        float scl[16];  // rows per thread per chunk <= stage / (16 B * 256)
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int lr = ct + kConsumerThreads * k;
+            scl[k] = (d.s2 && lr < nrows) ? fp16_to_f(__ldg(d.s2 + r0w + lr)) : 1.f;
+        }
+        if (!wait_full(p, s, kc))
+            return false;
+        const uint32_t st_a = s.ring_a + (uint32_t)(kc % p.ring_stages) * p.stage_bytes;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int lr = ct + kConsumerThreads * k;
+            if (lr < nrows) {
+                f2_t acc = 0ull;
+                for (int jb = 0; jb < ncb; ++jb) {
+                    const WVec<16> w = ldw<16>(st_a + (uint32_t)((jb * nrows + lr) * 16));
+                    f2_t x[E / 2];
+#pragma unroll
+                    for (int u = 0; u < E / 2; ++u) {
+                        const uint2 t = lds64(s.vec_a + (uint32_t)(jb * E + 2 * u) * 4);
+                        x[u] = pk2(__uint_as_float(t.x), __uint_as_float(t.y));
+                    }
+                    acc = vdot2<ESZ, 16>(w, x, acc);
+                }
+                red_add_fix(acc_out + r0w + lr, to_fix(sum2(acc) * scl[k]));
+            }
+        }
+        release_stage(p, s, kc, lane);
+        ++kc;
+    }
+    return true;
+}
+
+template <int Q8, int GENERIC>
+__device__ __forceinline__ bool ffn_down(const KParams &p, const SmemLayout &s, const Geom &g,
+                                         const TaskDesc &d, uint32_t &kc, int ct, int lane,
+                                         float sc0, float sc1)
+{
+    if (ct < g.R) {
+        const float gt = row_total(s, g, ct) * sc0;
+        const float up = row_total(s, g, g.R + ct) * sc1;
+        s.vec[ct] = gt / (1.f + __expf(-gt)) * up;
+    }
+    consumer_bar();
+    if constexpr (GENERIC)
+        return g.esz == 1 ? ffn_down_part<1>(p, s, g, d, kc, ct, lane)
+                          : ffn_down_part<2>(p, s, g, d, kc, ct, lane);
+    else
+        return ffn_down_part<Q8 ? 1 : 2>(p, s, g, d, kc, ct, lane);
+}
+
 // ---------------------------------------------------------- consumer loop
 template <int Q8, int ATT_E, int GENERIC>
 __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout &s, int qb,
@@ -1372,7 +1512,8 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
         // epilogue (thread t finalises row r0 + t; R <= 256)
         const Geom g = task_geom(p, d);
         float gv[kMaxPerThread];
-        const bool norm = d.kind == TK_QKV || d.kind == TK_GATEUP || d.kind == TK_LMHEAD;
+        const bool norm = d.kind == TK_QKV || d.kind == TK_GATEUP || d.kind == TK_FFN ||
+                          d.kind == TK_LMHEAD;
 #pragma unroll
         for (int j = 0; j < kMaxPerThread; ++j) {
             const int i = ct + j * kConsumerThreads;
@@ -1416,20 +1557,29 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
                 if (l == 0) {
                     if (token < 0)
                         token = resolve_token(p);
-                    rmsnorm_prologue(p, s, nullptr, p.embed + (size_t)token * p.hidden, gv, ct);
+                    rmsnorm_prologue(p, s, nullptr, p.embed + (size_t)token * p.hidden, nullptr,
+                                     gv, ct);
+                } else if (p.ffn_fused) {
+                    rmsnorm_prologue(p, s, nullptr, nullptr, p.xacc + (size_t)(l - 1) * p.hidden,
+                                     gv, ct);
                 } else {
-                    rmsnorm_prologue(p, s, p.xout + (size_t)(l - 1) * p.hidden, nullptr, gv, ct);
+                    rmsnorm_prologue(p, s, p.xout + (size_t)(l - 1) * p.hidden, nullptr, nullptr,
+                                     gv, ct);
                 }
             } else if (d.kind == TK_OPROJ) {
                 attn_prologue(p, s, l, ct);
-            } else if (d.kind == TK_GATEUP) {
-                rmsnorm_prologue(p, s, p.xmid + (size_t)l * p.hidden, nullptr, gv, ct);
+            } else if (d.kind == TK_GATEUP || d.kind == TK_FFN) {
+                rmsnorm_prologue(p, s, p.xmid + (size_t)l * p.hidden, nullptr, nullptr, gv, ct);
             } else if (d.kind == TK_DOWN) {
                 // no prologue: each warp loads its slice of the SwiGLU
                 // activations from L2 straight into registers
             } else {  // TK_LMHEAD
-                rmsnorm_prologue(p, s, p.xout + (size_t)(p.n_layers - 1) * p.hidden, nullptr,
-                                 gv, ct);
+                if (p.ffn_fused)
+                    rmsnorm_prologue(p, s, nullptr, nullptr,
+                                     p.xacc + (size_t)(p.n_layers - 1) * p.hidden, gv, ct);
+                else
+                    rmsnorm_prologue(p, s, p.xout + (size_t)(p.n_layers - 1) * p.hidden, nullptr,
+                                     nullptr, gv, ct);
             }
             // residual inputs of the epilogue are ready now: fetch them while
             // the GEMV runs (thread t owns output row r0 + t; R <= 256)
@@ -1441,6 +1591,8 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
                         if (token < 0)
                             token = resolve_token(p);
                         base = bf16_to_f(__ldg(p.embed + (size_t)token * p.hidden + r));
+                    } else if (p.ffn_fused) {
+                        base = from_fix(__ldcg(p.xacc + (size_t)(l - 1) * p.hidden + r));
                     } else {
                         base = __ldcg(p.xout + (size_t)(l - 1) * p.hidden + r);
                     }
@@ -1470,9 +1622,14 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
                     for (int t = ct; t < g.R; t += kConsumerThreads)
                         out[t] = row_total(s, g, t) * sc0;
                 } else if (d.kind == TK_OPROJ) {
-                    if (ct < g.R)
-                        p.xmid[(size_t)l * p.hidden + d.r0 + ct] =
-                            base + row_total(s, g, ct) * sc0;
+                    if (ct < g.R) {
+                        const float v = base + row_total(s, g, ct) * sc0;
+                        p.xmid[(size_t)l * p.hidden + d.r0 + ct] = v;
+                        if (p.ffn_fused)  // the FFN slices add into this
+                            p.xacc[(size_t)l * p.hidden + d.r0 + ct] = to_fix(v);
+                    }
+                } else if (d.kind == TK_FFN) {
+                    ok = ffn_down<Q8, GENERIC>(p, s, g, d, kc, ct, lane, sc0, sc1);
                 } else if (d.kind == TK_GATEUP) {
                     for (int t = ct; t < g.R; t += kConsumerThreads) {
                         const float gt = row_total(s, g, t) * sc0;
@@ -1580,6 +1737,19 @@ __global__ void __launch_bounds__(kThreads, 1) amk_decode_kernel(const __grid_co
 
 }  // namespace
 
+// Wdown of one layer, [hidden][ffn] row-major, re-laid once per handle as
+// 16-byte column groups, [ffn * esz / 16][hidden][16 B], so that a fused FFN
+// slice's columns for a run of rows are contiguous: one thread per (column
+// group, row), consecutive threads on consecutive rows (coalesced stores).
+__global__ void amk_pack_down_kernel(const uint4 *wd, uint4 *out, int h, int ncg)
+{
+    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (size_t)h * ncg)
+        return;
+    const int row = (int)(idx % h), cg = (int)(idx / h);
+    out[(size_t)cg * h + row] = wd[(size_t)row * ncg + cg];
+}
+
 // Host-visible launch helpers -------------------------------------------------
 extern "C" int amk_kernel_smem_bytes(int ring_stages, int stage_bytes, int vec_floats)
 {
@@ -1616,6 +1786,16 @@ extern "C" cudaError_t amk_kernel_occupancy(int smem_bytes, int quant, int att_e
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm,
                                                          kernel_for(quant, att_e, generic),
                                                          kThreads, smem_bytes);
+}
+
+extern "C" cudaError_t amk_pack_down(const void *wd, void *out, int h, int ffn, int esz,
+                                     cudaStream_t stream)
+{
+    const int ncg = ffn * esz / 16;
+    const size_t n = (size_t)h * ncg;
+    amk_pack_down_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
+        static_cast<const uint4 *>(wd), static_cast<uint4 *>(out), h, ncg);
+    return cudaGetLastError();
 }
 
 extern "C" cudaError_t amk_kernel_launch(const KParams *p, int n_ctas, int smem_bytes,

@@ -25,6 +25,10 @@
 #include "amk_internal.h"
 #include "amk_plan.h"
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
 extern "C" int amk_kernel_smem_bytes(int ring_stages, int stage_bytes, int vec_floats);
 
 namespace {
@@ -81,6 +85,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         opt.debug_skip_signal_task = opt_in->debug_skip_signal_task;
         opt.profile = opt_in->profile;
         if (opt_in->l2_prefetch_kb > 0) opt.l2_prefetch_kb = opt_in->l2_prefetch_kb;
+        if (opt_in->ffn_fused != 0) opt.ffn_fused = opt_in->ffn_fused;
         opt.n_sms = opt_in->n_sms;
     }
     const amk_config &c = *cfg;
@@ -186,8 +191,38 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         if (((int64_t)m.K * m.esz) % 16)
             P->generic = 1;
 
+    // FFN fusion: the columns [a, b) of Wdown come as 2-D TMA boxes of 16
+    // bytes x box_rows rows, so the slice starts and the row pitch must be
+    // 16-byte multiples and the box rows must divide hidden
+    int box_rows = 0;
+    for (int br : {256, 128, 64})
+        if (!box_rows && h % br == 0)
+            box_rows = br;
+    // slice width: a multiple of 16 bytes of a Wdown row, about one slice per
+    // SM, at most 128 (the gate/up half of the red buffer)
+    const int ffn_gran = 16 / esz;
+    const int ffn_units = F / ffn_gran, n_target = n_sms * std::max(1, opt.tasks_per_sm);
+    const int ffn_w = std::min((ffn_units + n_target - 1) / n_target * ffn_gran,
+                               amk::kMaxTaskRows / 2 / ffn_gran * ffn_gran);
+    const int64_t ffn_fit = box_rows ? (int64_t)opt.stage_bytes /
+                                           ((int64_t)ffn_w * esz * box_rows) * box_rows
+                                     : 0;
+    // default (ffn_fused = 1): fuse when a residual row is at most 2 KB.  The
+    // fused level adds every slice's partial down projection into the same
+    // hidden-sized accumulator with 64-bit atomics, whose contention grows with
+    // the width; measured on B200 it gains 23% (SmolLM2 shape, 1152 B) and 5%
+    // (Llama-1B W8A16, 2 KB) but loses 3% (TinyLlama, 4 KB) and 8% (Llama-7B,
+    // 8 KB).  ffn_fused = 2 fuses whenever the shape allows.
+    const bool shape_ok = F % ffn_gran == 0 && box_rows > 0 && ((int64_t)F * esz) % 16 == 0 &&
+                          (ffn_fit >= h || ffn_fit >= 256);
+    const bool fused = shape_ok && (opt.ffn_fused >= 2 ||
+                                    (opt.ffn_fused == 1 && (int64_t)h * esz <= 2048));
+    P->ffn_fused = fused ? 1 : 0;
+    P->ffn_box_rows = fused ? box_rows : 0;
+
     // ---- logical tasks per level ---------------------------------------------
-    enum { LV_QKV, LV_ATTN, LV_OPROJ, LV_GATEUP, LV_DOWN, LV_N };
+    // unfused: QKV, ATTN, OPROJ, GATEUP, DOWN; fused: QKV, ATTN, OPROJ, FFN
+    const int LV_N = fused ? 4 : 5;
     auto ctr_of = [&](int layer, int lv) { return layer * LV_N + lv; };
     const int n_ctr = L * LV_N;
     std::vector<std::vector<Logical>> levels;
@@ -242,6 +277,15 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         std::vector<Logical> o, gu, dn;
         gemv_level(amk::TK_OPROJ, l, h, nh * hd, esz, target, amk::kMaxTaskRows, 0, o);
         levels.push_back(std::move(o));
+        if (fused) {
+            std::vector<Logical> ffn;
+            for (int a = 0; a < F; a += ffn_w) {
+                const int b = std::min(a + ffn_w, F);
+                ffn.push_back({mk(amk::TK_FFN, l, a, b), (int64_t)(b - a) * h * esz * 3});
+            }
+            levels.push_back(std::move(ffn));
+            continue;
+        }
         gemv_level(amk::TK_GATEUP, l, F, h, esz, target, amk::kMaxTaskRows / 2, 0, gu);
         for (auto &t : gu)
             t.cost *= 2;
@@ -257,7 +301,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     }
     // waits / signals: level i of layer l signals ctr(l, i); waits on the
     // previous level's counter at full count (QKV of layer l > 0 waits on
-    // DOWN of layer l-1; LMHEAD waits on DOWN of the last layer)
+    // the last level of layer l-1; LMHEAD on the last level of the last layer)
     std::vector<uint32_t> total(n_ctr, 0);
     for (size_t li = 0; li + 1 < levels.size(); ++li) {
         const int layer = (int)li / LV_N, lv = (int)li % LV_N;
@@ -390,6 +434,12 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
                 else
                     acc(B_KEYNEXT, AMK_ACC_READ_PREV, 0, 1);
                 acc(B_XMID(l), AMK_ACC_WRITE, d.r0, d.r1);
+                if (fused)  // the FFN's accumulator starts at the residual
+                    acc(B_XOUT(l), AMK_ACC_WRITE, d.r0, d.r1);
+                break;
+            case amk::TK_FFN:
+                acc(B_XMID(l), AMK_ACC_READ, 0, h);
+                acc(B_XOUT(l), AMK_ACC_ACCUM, 0, h);
                 break;
             case amk::TK_GATEUP:
                 acc(B_XMID(l), AMK_ACC_READ, 0, h);
@@ -465,7 +515,7 @@ void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *k
         return q8 ? static_cast<const uint16_t *>(arr[l]) + r : nullptr;
     };
     d.w0 = d.w1 = nullptr;
-    d.s0 = d.s1 = d.gain = nullptr;
+    d.s0 = d.s1 = d.s2 = d.gain = nullptr;
     const int h = c.hidden;
     switch (d.kind) {
     case amk::TK_QKV: {
@@ -497,6 +547,14 @@ void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *k
         d.w0 = row(w->wdown[l], d.r0, (int64_t)c.ffn * esz);
         d.s0 = srow(w->sdown, d.r0);
         break;
+    case amk::TK_FFN:  // Wdown comes through the layer's tensor map
+        d.w0 = row(w->wgate[l], d.r0, (int64_t)h * esz);
+        d.w1 = row(w->wup[l], d.r0, (int64_t)h * esz);
+        d.s0 = srow(w->sgate, d.r0);
+        d.s1 = srow(w->sup, d.r0);
+        d.s2 = srow(w->sdown, 0);
+        d.gain = static_cast<const uint16_t *>(w->ffn_norm[l]);
+        break;
     default: {  // TK_LMHEAD
         const bool head_q8 = q8 && !c.tied_embeddings;
         d.w0 = row(c.tied_embeddings ? w->embed : w->lm_head, d.r0, (int64_t)h * (head_q8 ? 1 : 2));
@@ -506,4 +564,40 @@ void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *k
     }
     }
     *out = d;
+}
+
+int amk_encode_down_maps(const amk_plan *P, const amk_weights *w, int l0, int n, void *out)
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return amk_set_error(AMK_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const amk_config &c = P->cfg;
+    const bool q8 = c.quant == AMK_QUANT_W8A16;
+    const int esz = q8 ? 1 : 2;
+    for (int l = l0; l < l0 + n; ++l) {
+        CUtensorMap map;
+        CUtensorMap *m = &map;
+        const cuuint64_t dims[2] = {(cuuint64_t)c.ffn, (cuuint64_t)c.hidden};
+        const cuuint64_t strides[1] = {(cuuint64_t)c.ffn * esz};
+        const cuuint32_t box[2] = {(cuuint32_t)(16 / esz), (cuuint32_t)P->ffn_box_rows};
+        const cuuint32_t estr[2] = {1, 1};
+        const CUresult r = encode(m, q8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                                  2, const_cast<void *>(w->wdown[l]), dims, strides, box, estr,
+                                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS)
+            return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d: Wdown tensor map (error %d)", l,
+                                 (int)r);
+        static_assert(sizeof(CUtensorMap) == 128, "CUtensorMap is 128 bytes");
+        memcpy(static_cast<uint8_t *>(out) + 128 * (size_t)(l - l0), &map, sizeof map);
+    }
+    return AMK_OK;
 }

@@ -39,7 +39,7 @@ void *g_scratch_addr[kMaxDevices];  // device address of g_scratch, per device
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t tasks, qoff, ctr, err, argkey, qkv, part, attn, xmid, xout, act, total;
+    size_t tasks, qoff, ctr, err, argkey, qkv, part, attn, xmid, xout, act, xacc, dmaps, total;
 };
 
 Layout layout_of(const amk_plan &P)
@@ -65,6 +65,8 @@ Layout layout_of(const amk_plan &P)
     o.xmid = take(sizeof(float) * L * c.hidden);
     o.xout = take(sizeof(float) * L * c.hidden);
     o.act = take(sizeof(float) * L * c.ffn);
+    o.xacc = take(P.ffn_fused ? sizeof(long long) * L * c.hidden : 0);
+    o.dmaps = take(P.ffn_fused ? 128 * L : 0);
     o.total = off;
     return o;
 }
@@ -170,6 +172,20 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
         if (e != cudaSuccess)
             return fail_cuda(e, "schedule upload");
     }
+    // tensor maps of Wdown (fused FFN), through a stack buffer
+    if (P.ffn_fused) {
+        alignas(64) unsigned char mbuf[128 * 16];
+        for (int l0 = 0; l0 < c.n_layers; l0 += 16) {
+            const int n = c.n_layers - l0 < 16 ? c.n_layers - l0 : 16;
+            const int mrc = amk_encode_down_maps(&P, w, l0, n, mbuf);
+            if (mrc != AMK_OK)
+                return mrc;
+            e = cudaMemcpyAsync(base + lay.dmaps + 128 * (size_t)l0, mbuf, 128 * (size_t)n,
+                                cudaMemcpyHostToDevice, st);
+            if (e != cudaSuccess)
+                return fail_cuda(e, "tensor map upload");
+        }
+    }
     // what must start at zero: counters, error word, argmax keys
     e = cudaMemsetAsync(base + lay.ctr, 0, lay.qkv - lay.ctr, st);
     if (e != cudaSuccess)
@@ -188,6 +204,11 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     k.xmid = reinterpret_cast<float *>(base + lay.xmid);
     k.xout = reinterpret_cast<float *>(base + lay.xout);
     k.act = reinterpret_cast<float *>(base + lay.act);
+    k.xacc = reinterpret_cast<long long *>(base + lay.xacc);
+    k.dmaps = base + lay.dmaps;
+    k.dpack = nullptr;  // no room for a packed copy: the tensor maps read the caller's Wdown
+    k.ffn_fused = P.ffn_fused;
+    k.ffn_box_rows = P.ffn_box_rows;
     k.logits = logits_dev;
     k.argkey = reinterpret_cast<unsigned long long *>(base + lay.argkey);
     k.kv = static_cast<uint16_t *>(kv_cache);

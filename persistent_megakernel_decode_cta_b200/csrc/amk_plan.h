@@ -19,7 +19,9 @@ struct amk_plan {
     std::vector<int32_t> queue_off;    // [n_sms + 1]
     int n_counters = 0;  // level counters (the validator's graph)
     int n_arrive = 0;
-    int att_pg = 1;      // attention position groups per warp    // attention arrival counters, [L][nkv], after them
+    int att_pg = 1;      // attention position groups per warp
+    int ffn_fused = 0;   // 1: one FFN level per layer (gate/up + down column slice)
+    int ffn_box_rows = 0;  // rows of a Wdown TMA box (divides hidden)    // attention arrival counters, [L][nkv], after them
     // the validator's view
     std::vector<amk_graph_task> gtasks;
     std::vector<amk_graph_wait> gwaits;
@@ -38,6 +40,11 @@ void amk_plan_view(const amk_plan *P, amk_graph *g);
 // Copies plan task t into *out with its device pointers resolved: weight
 // rows, row scales and norm gain from w, KV-cache blocks from kv (bf16
 // [L][2][nkv][max_ctx][hd]).  Host only; reads only host memory.
+// Tensor maps of the Wdown of layers [l0, l0 + n) for a fused FFN (128 bytes
+// each, to be copied to 64-byte aligned device memory): a 2-D [hidden][ffn]
+// view with boxes of 16 bytes x ffn_box_rows rows.  Returns an amk status.
+int amk_encode_down_maps(const amk_plan *P, const amk_weights *w, int l0, int n, void *out);
+
 void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *kv, int t,
                       amk::TaskDesc *out);
 

@@ -105,6 +105,27 @@ def test_full_size_single_steps(name, ctxs):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("name,ctx,fused", [
+    ("tinyllama", 256, 2),     # the fused FFN level where the default keeps it split
+    ("llama7b_w8", 0, 2),
+    ("smol135", 128, -1),      # split levels where the default fuses
+    ("llama1b_w8", 512, -1),
+])
+def test_ffn_level_variants(name, ctx, fused):
+    """Both FFN schedules (one fused level with fixed-point accumulation of
+    the down projection, or separate gate/up and down levels) against the
+    oracle, on the shapes where the default picks the other one."""
+    cfg = si.get_config(name)
+    pair = Pair(cfg, options=amk.default_options(ffn_fused=fused))
+    if ctx:
+        pair.fill_kv(ctx)
+    tok = si.make_prompt(cfg, 1, seed=10 + ctx)[0]
+    g, am, ref, ref_am = pair.step(tok, ctx)
+    compare(cfg, g, am, ref, ref_am, what=f"{name} ctx {ctx} ffn_fused {fused}")
+    del pair
+    torch.cuda.empty_cache()
+
+
 def test_smol_greedy_32_steps():
     cfg = si.get_config("smol135")
     pair = Pair(cfg)

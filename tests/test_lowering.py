@@ -12,7 +12,8 @@ from persistent_megakernel_decode_cta_b200 import abi, build
 import synth_inputs as si
 from oracle import interleave as bf
 
-KIND = {1: "QKV", 2: "ATTN", 3: "OPROJ", 4: "GATEUP", 5: "DOWN", 6: "LMHEAD"}
+KIND = {1: "QKV", 2: "ATTN", 3: "OPROJ", 4: "GATEUP", 5: "DOWN", 6: "LMHEAD", 7: "FFN"}
+ORDER = ["QKV", "ATTN", "OPROJ", "GATEUP", "DOWN", "FFN", "LMHEAD"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -20,11 +21,11 @@ def built():
     build.build()
 
 
-def _writes(g, buf):
+def _writes(g, buf, kind=None):
     out = []
     for t, task in enumerate(g["tasks"]):
         for (b, k, lo, hi) in task["accesses"]:
-            if b == buf and k == abi.ACC_WRITE:
+            if b == buf and k == (abi.ACC_WRITE if kind is None else kind):
                 out.append((lo, hi, t))
     return sorted(out)
 
@@ -39,24 +40,35 @@ def _partition(ranges, size):
 
 @pytest.mark.parametrize("name", list(si.CONFIGS))
 @pytest.mark.parametrize("n_sms", [148, 7])
-def test_real_lowerings_accepted_and_cover(name, n_sms):
+@pytest.mark.parametrize("fused", [2, -1])
+def test_real_lowerings_accepted_and_cover(name, n_sms, fused):
     cfg = si.get_config(name)
-    plan = amk.Plan(cfg, n_sms)
+    plan = amk.Plan(cfg, n_sms, amk.default_options(ffn_fused=fused))
     g = plan.graph()
     kinds, layers = plan.task_info()
     L, h, F = cfg.n_layers, cfg.hidden, cfg.ffn
-    # buffers: 6 per layer (qkv, part, xmid, xout, act, kvnew) + logits, key, key_next
+    is_fused = any(KIND[k] == "FFN" for k in kinds)
+    if fused < 0:
+        assert not is_fused
+    # buffers: 6 per layer (qkv, attention output, xmid, xout, act, kvnew) +
+    # logits, key, key_next
     assert len(g["buffers"]) == 6 * L + 3
     for l in range(L):
         _partition(_writes(g, 6 * l + 0), cfg.q_rows + 2 * cfg.kv_rows)   # QKV rows
         _partition(_writes(g, 6 * l + 2), h)                               # O rows
-        _partition(_writes(g, 6 * l + 3), h)                               # down rows
-        _partition(_writes(g, 6 * l + 4), F)                               # gate/up rows
+        # down rows, or (fused) the O rows that start the FFN's accumulator
+        _partition(_writes(g, 6 * l + 3), h)
+        if is_fused:
+            acc = _writes(g, 6 * l + 3, abi.ACC_ACCUM)
+            ffn = [t for t in range(len(kinds)) if KIND[kinds[t]] == "FFN" and layers[t] == l]
+            assert sorted(t for _, _, t in acc) == ffn
+            assert all((lo, hi) == (0, h) for lo, hi, _ in acc)
+        else:
+            _partition(_writes(g, 6 * l + 4), F)                           # gate/up rows
     _partition(_writes(g, 6 * L), cfg.vocab)                               # LM head rows
     # every SM runs its tasks level by level
     for q in g["queues"]:
-        seq = [(layers[t], ["QKV", "ATTN", "OPROJ", "GATEUP", "DOWN", "LMHEAD"].index(
-            KIND[kinds[t]])) for t in q]
+        seq = [(layers[t], ORDER.index(KIND[kinds[t]])) for t in q]
         assert seq == sorted(seq)
     n_att = sum(1 for k in kinds if KIND[k] == "ATTN")
     assert n_att % (L * cfg.n_kv_heads) == 0
@@ -64,6 +76,19 @@ def test_real_lowerings_accepted_and_cover(name, n_sms):
     # too); run it again on the exported graph
     ok, rule, msg = amk.validate_graph(g)
     assert ok, (rule, msg)
+
+
+def test_fused_ffn_slices_cover_ffn():
+    """The fused FFN level of each layer has about one slice per SM, each a
+    multiple of 16 bytes of a Wdown row, and the slices tile [0, ffn)."""
+    for name in ("tinyllama", "llama1b_w8", "llama7b", "smol135"):
+        cfg = si.get_config(name)
+        plan = amk.Plan(cfg, 148, amk.default_options(ffn_fused=2))
+        kinds, layers = plan.task_info()
+        n = sum(1 for k, l in zip(kinds, layers) if KIND[k] == "FFN" and l == 0)
+        esz = 1 if cfg.quant == "w8a16" else 2
+        w = -(-(cfg.ffn // (16 // esz)) // 148) * (16 // esz)
+        assert n == -(-cfg.ffn // w) and n <= 148, (name, n)
 
 
 def test_small_real_lowering_passes_brute_force():
@@ -76,11 +101,16 @@ def test_small_real_lowering_passes_brute_force():
 
 def test_balanced_tiles_on_148_sms():
     cfg = si.get_config("tinyllama")
-    plan = amk.Plan(cfg, 148)
+    plan = amk.Plan(cfg, 148, amk.default_options(ffn_fused=-1))
     g = plan.graph()
     kinds, layers = plan.task_info()
     per_sm_gateup = [sum(1 for t in q if kinds[t] == 4 and layers[t] == 0) for q in g["queues"]]
     assert max(per_sm_gateup) == 1 and min(per_sm_gateup) == 1
+    fused = amk.Plan(cfg, 148, amk.default_options(ffn_fused=2))
+    g = fused.graph()
+    kinds, layers = fused.task_info()
+    per_sm_ffn = [sum(1 for t in q if kinds[t] == 7 and layers[t] == 0) for q in g["queues"]]
+    assert max(per_sm_ffn) == 1
 
 
 @pytest.mark.parametrize("edit,status", [
