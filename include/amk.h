@@ -118,7 +118,10 @@ typedef struct {
                                  when the shape allows and hidden * element size <= 2 KB;
                                  2: whenever the shape allows; -1: separate gate/up and
                                  down levels */
-    int32_t reserved[5];
+    int32_t pos0_plan;        /* 1 (default): steps at position 0 run a second, validated
+                                 schedule without the attention level (softmax over one
+                                 key: each head's output is its KV head's V row); -1: off */
+    int32_t reserved[4];
 } amk_options;
 
 typedef struct amk_handle amk_handle;
@@ -219,6 +222,9 @@ AMK_API int amk_plan_graph(const amk_plan *p, amk_graph *out);
 /* Per-task kind and layer of a plan ([n_tasks] each; host memory, may be NULL). */
 AMK_API int amk_plan_task_info(const amk_plan *p, int32_t *kind, int32_t *layer);
 AMK_API void amk_plan_destroy(amk_plan *p);
+/* The schedule the plan's steps at position 0 run (amk_options.pos0_plan):
+ * validated with the plan, owned by it (not to be destroyed), or NULL. */
+AMK_API const amk_plan *amk_plan_pos0(const amk_plan *p);
 
 /* Creates a decoder: lowers, validates (rejection -> AMK_ERR_VALIDATION),
  * allocates the KV cache (bf16 [n_layers][2][n_kv_heads][max_ctx][head_dim],

@@ -150,10 +150,21 @@ class Plan:
         _check(abi.lib().amk_plan_task_info(self._p, kind, layer), "amk_plan_task_info")
         return list(kind[:n]), list(layer[:n])
 
+    def pos0(self) -> Optional["Plan"]:
+        """The schedule of steps at position 0 (a view owned by this plan), or
+        None when the plan was made with pos0_plan = -1."""
+        p = abi.lib().amk_plan_pos0(self._p)
+        if not p:
+            return None
+        view = Plan.__new__(Plan)
+        view._p = ctypes.c_void_p(p)
+        view._owner = self  # keeps the owning plan alive
+        return view
+
     def close(self):
-        if self._p:
+        if self._p and not hasattr(self, "_owner"):
             abi.lib().amk_plan_destroy(self._p)
-            self._p = ctypes.c_void_p()
+        self._p = ctypes.c_void_p()
 
     def __del__(self):
         try:

@@ -45,7 +45,8 @@ class Options(ctypes.Structure):
     _fields_ = [("ring_stages", c_i32), ("stage_bytes", c_i32), ("attn_splits", c_i32),
                 ("tasks_per_sm", c_i32), ("n_sms", c_i32), ("wait_timeout_us", c_u32),
                 ("debug_skip_signal_task", c_i32), ("profile", c_i32),
-                ("l2_prefetch_kb", c_i32), ("ffn_fused", c_i32), ("reserved", c_i32 * 5)]
+                ("l2_prefetch_kb", c_i32), ("ffn_fused", c_i32),
+                ("pos0_plan", c_i32), ("reserved", c_i32 * 4)]
 
 
 class GraphWait(ctypes.Structure):
@@ -112,6 +113,7 @@ SIGNATURES = {
     "amk_plan_graph": (ctypes.c_int, [c_vp, ctypes.POINTER(Graph)]),
     "amk_plan_task_info": (ctypes.c_int, [c_vp, ctypes.POINTER(c_i32), ctypes.POINTER(c_i32)]),
     "amk_plan_destroy": (None, [c_vp]),
+    "amk_plan_pos0": (c_vp, [c_vp]),
     "amk_create": (ctypes.c_int, [ctypes.POINTER(Config), ctypes.POINTER(Weights),
                                   ctypes.POINTER(Options), c_vp, ctypes.POINTER(c_vp)]),
     "amk_destroy": (None, [c_vp]),

@@ -82,6 +82,7 @@ extern "C" int amk_default_options(amk_options *o)
     o->wait_timeout_us = 1000000;  // 1 s
     o->debug_skip_signal_task = -1;
     o->ffn_fused = 1;
+    o->pos0_plan = 1;
     return AMK_OK;
 }
 
@@ -95,15 +96,24 @@ extern "C" int amk_plan_create(const amk_config *cfg, const amk_options *opt, in
     amk_plan *P = new (std::nothrow) amk_plan();
     if (!P)
         return amk_set_error(AMK_ERR_OOM, "amk_plan_create: out of host memory");
-    int rc = amk_lower(cfg, opt, n_sms, P);
-    if (rc == AMK_OK) {
-        amk_graph g;
-        amk_plan_view(P, &g);
-        amk_validation_report local;
-        rc = amk_validate_graph(&g, report ? report : &local);
-        if (rc != AMK_OK)
-            amk_set_error(rc, "lowered schedule rejected: %s",
-                          (report ? report : &local)->message);
+    auto lower_checked = [&](amk_plan *Q, int pos0) {
+        int r = amk_lower(cfg, opt, n_sms, Q, pos0);
+        if (r == AMK_OK) {
+            amk_graph g;
+            amk_plan_view(Q, &g);
+            amk_validation_report local;
+            r = amk_validate_graph(&g, report ? report : &local);
+            if (r != AMK_OK)
+                amk_set_error(r, "lowered %sschedule rejected: %s", pos0 ? "position-0 " : "",
+                              (report ? report : &local)->message);
+        }
+        return r;
+    };
+    int rc = lower_checked(P, 0);
+    if (rc == AMK_OK && P->opt.pos0_plan > 0) {
+        P->pos0 = new (std::nothrow) amk_plan();
+        rc = P->pos0 ? lower_checked(P->pos0, 1)
+                     : amk_set_error(AMK_ERR_OOM, "amk_plan_create: out of host memory");
     }
     if (rc != AMK_OK) {
         delete P;
@@ -112,6 +122,8 @@ extern "C" int amk_plan_create(const amk_config *cfg, const amk_options *opt, in
     *out = P;
     return AMK_OK;
 }
+
+extern "C" const amk_plan *amk_plan_pos0(const amk_plan *p) { return p ? p->pos0 : nullptr; }
 
 extern "C" int amk_plan_graph(const amk_plan *p, amk_graph *out)
 {
@@ -144,6 +156,11 @@ struct amk_handle {
     TaskDesc *d_tasks = nullptr;
     int32_t *d_qoff = nullptr;
     uint32_t *d_ctr = nullptr;
+    // the position-0 schedule (plan->pos0): its own tables and level counters
+    TaskDesc *d_tasks0 = nullptr;
+    int32_t *d_qoff0 = nullptr;
+    uint32_t *d_ctr0 = nullptr;
+    uint32_t epoch0 = 0;  // steps run with it since the last reset
     ErrorWord *d_err = nullptr;
     float *d_qkv = nullptr, *d_part = nullptr, *d_attn = nullptr, *d_xmid = nullptr,
           *d_xout = nullptr;
@@ -248,6 +265,9 @@ int zero_state(amk_handle *H)
     if (e == cudaSuccess)
         e = cudaMemsetAsync(H->d_ctr, 0, sizeof(uint32_t) * (size_t)(P->n_counters + P->n_arrive),
                             H->stream);
+    if (e == cudaSuccess && P->pos0)
+        e = cudaMemsetAsync(H->d_ctr0, 0, sizeof(uint32_t) * (size_t)P->pos0->n_counters,
+                            H->stream);
     if (e == cudaSuccess)
         e = cudaMemsetAsync(H->d_err, 0, sizeof(ErrorWord), H->stream);
     if (e == cudaSuccess)
@@ -257,6 +277,7 @@ int zero_state(amk_handle *H)
     if (e != cudaSuccess)
         return cuda_fail(e, "amk_reset_kv");
     H->epoch = 0;
+    H->epoch0 = 0;
     H->arrive_base = 0;
     H->poisoned = false;
     H->err_pending = false;
@@ -345,6 +366,10 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     if ((rc = dalloc(H, &H->d_tasks, sizeof(TaskDesc) * P->tasks.size())) ||
         (rc = dalloc(H, &H->d_qoff, sizeof(int32_t) * P->queue_off.size())) ||
         (rc = dalloc(H, &H->d_ctr, sizeof(uint32_t) * (size_t)(P->n_counters + P->n_arrive))) ||
+        (P->pos0 &&
+         ((rc = dalloc(H, &H->d_tasks0, sizeof(TaskDesc) * P->pos0->tasks.size())) ||
+          (rc = dalloc(H, &H->d_qoff0, sizeof(int32_t) * P->pos0->queue_off.size())) ||
+          (rc = dalloc(H, &H->d_ctr0, sizeof(uint32_t) * (size_t)P->pos0->n_counters)))) ||
         (rc = dalloc(H, &H->d_err, sizeof(ErrorWord))) ||
         (rc = dalloc(H, &act_block, H->act_bytes)) ||
         (rc = dalloc(H, &H->d_logits, sizeof(float) * (size_t)c.vocab)) ||
@@ -389,6 +414,18 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
         (e = cudaMemcpyAsync(H->d_qoff, P->queue_off.data(),
                              sizeof(int32_t) * P->queue_off.size(), cudaMemcpyHostToDevice,
                              H->stream)) != cudaSuccess) {
+        free_handle(H);
+        return cuda_fail(e, "upload schedule");
+    }
+    std::vector<TaskDesc> resolved0(P->pos0 ? P->pos0->tasks.size() : 0);
+    for (size_t t = 0; t < resolved0.size(); ++t)
+        amk_resolve_task(P->pos0, w, H->d_kv, (int)t, &resolved0[t]);
+    if (P->pos0 &&
+        ((e = cudaMemcpyAsync(H->d_tasks0, resolved0.data(), sizeof(TaskDesc) * resolved0.size(),
+                              cudaMemcpyHostToDevice, H->stream)) != cudaSuccess ||
+         (e = cudaMemcpyAsync(H->d_qoff0, P->pos0->queue_off.data(),
+                              sizeof(int32_t) * P->pos0->queue_off.size(),
+                              cudaMemcpyHostToDevice, H->stream)) != cudaSuccess)) {
         free_handle(H);
         return cuda_fail(e, "upload schedule");
     }
@@ -498,7 +535,15 @@ int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev,
     KParams k = H->kp;
     k.pos = pos;
     k.token = token_id;
-    k.epoch = H->epoch;
+    // counter epochs count the steps each schedule ran (parity counts all)
+    k.epoch = H->epoch - H->epoch0;
+    const bool at0 = pos == 0 && H->plan->pos0;
+    if (at0) {  // the position-0 schedule, with its own counters
+        k.tasks = H->d_tasks0;
+        k.queue_off = H->d_qoff0;
+        k.counters = H->d_ctr0;
+        k.epoch = H->epoch0;
+    }
     k.arrive_base = H->arrive_base;
     k.parity = (int32_t)(H->epoch & 1u);
     if (logits_dev)
@@ -519,6 +564,8 @@ int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev,
                              "cooperative launch: %s", cudaGetErrorString(e));
     }
     H->epoch += 1;
+    if (at0)
+        H->epoch0 += 1;
     {  // non-empty attention chunks of this step: each arrives once unless alone
         const int C = H->plan->opt.attn_splits, n = pos + 1;
         const int chunk = (n + C - 1) / C, nne = (n + chunk - 1) / chunk;

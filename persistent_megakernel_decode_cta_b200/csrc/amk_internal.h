@@ -53,6 +53,8 @@ enum TaskKind : uint8_t {
 
 enum TaskFlags : uint8_t {
     TF_RESET_ARGKEY = 1,  // this task clears the next step's argmax key
+    TF_POS0 = 2,          // O-projection of the position-0 schedule: head outputs = V rows,
+                          // and the task writes its share of KV-cache row 0
 };
 
 struct TaskDesc {           // 80 bytes, read-only for the kernel

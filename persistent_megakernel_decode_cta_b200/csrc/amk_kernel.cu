@@ -1365,6 +1365,49 @@ __device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
     return true;
 }
 
+// O-projection prologue of the position-0 schedule.  At position 0 the
+// softmax runs over the single key of this step, so every weight is 1 and the
+// attention output of head h is the V row of its KV head h / G as stored in
+// the cache (bf16), and RoPE at angle 0 is the identity.  Cache row 0 (K = k,
+// V = v, rounded to bf16) is written in shares: of its E = 2 nkv hd elements
+// (K of every head, then V), the tile of rows [r0, r1) writes
+// [r0 E / h, r1 E / h).
+__device__ void pos0_prologue(const KParams &p, const SmemLayout &s, const TaskDesc &d, int ct)
+{
+    const int l = d.layer, hd = p.head_dim, nh = p.n_heads, nkv = p.n_kv_heads, G = p.group;
+    const int N = nh * hd;
+    const float *qkv = p.qkv + (size_t)l * p.qkv_rows;
+    const float *vsrc = qkv + (size_t)(nh + nkv) * hd;
+    float v[kMaxPerThread];
+#pragma unroll
+    for (int j = 0; j < kMaxPerThread; ++j) {
+        const int i = ct + j * kConsumerThreads;
+        v[j] = 0.f;
+        if (i < N) {
+            const int h = i / hd;
+            v[j] = __ldcg(vsrc + (size_t)(h / G) * hd + (i - h * hd));
+        }
+    }
+    {
+        const int E = 2 * nkv * hd;
+        const int a = (int)((int64_t)d.r0 * E / p.hidden), b = (int)((int64_t)d.r1 * E / p.hidden);
+        const size_t blk = (size_t)p.max_ctx * hd;  // one (layer, K|V, head) block
+        for (int i = a + ct; i < b; i += kConsumerThreads) {
+            const int which = i / (nkv * hd), r = i - which * nkv * hd;  // 0: K, 1: V
+            const int g = r / hd, e = r - g * hd;
+            p.kv[(((size_t)l * 2 + which) * nkv + g) * blk + e] =
+                f_to_bf16(__ldcg(qkv + (size_t)nh * hd + i));
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxPerThread; ++j) {
+        const int i = ct + j * kConsumerThreads;
+        if (i < N)
+            s.vec[i] = bf16_to_f(f_to_bf16(v[j]));
+    }
+    consumer_bar();
+}
+
 // O-projection prologue: the merged attention output of layer l -> vec
 // (one L2 round trip).  n_heads * head_dim <= kMaxPerThread * 256.
 __device__ void attn_prologue(const KParams &p, const SmemLayout &s, int l, int ct)
@@ -1567,7 +1610,10 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
                                      gv, ct);
                 }
             } else if (d.kind == TK_OPROJ) {
-                attn_prologue(p, s, l, ct);
+                if (d.flags & TF_POS0)
+                    pos0_prologue(p, s, d, ct);
+                else
+                    attn_prologue(p, s, l, ct);
             } else if (d.kind == TK_GATEUP || d.kind == TK_FFN) {
                 rmsnorm_prologue(p, s, p.xmid + (size_t)l * p.hidden, nullptr, nullptr, gv, ct);
             } else if (d.kind == TK_DOWN) {

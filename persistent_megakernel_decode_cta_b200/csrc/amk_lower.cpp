@@ -72,7 +72,8 @@ struct Logical {
 
 }  // namespace
 
-int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_plan *P)
+int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_plan *P,
+              int pos0)
 {
     amk_options opt;
     amk_default_options(&opt);
@@ -86,6 +87,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         opt.profile = opt_in->profile;
         if (opt_in->l2_prefetch_kb > 0) opt.l2_prefetch_kb = opt_in->l2_prefetch_kb;
         if (opt_in->ffn_fused != 0) opt.ffn_fused = opt_in->ffn_fused;
+        if (opt_in->pos0_plan != 0) opt.pos0_plan = opt_in->pos0_plan;
         opt.n_sms = opt_in->n_sms;
     }
     const amk_config &c = *cfg;
@@ -221,8 +223,10 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     P->ffn_box_rows = fused ? box_rows : 0;
 
     // ---- logical tasks per level ---------------------------------------------
-    // unfused: QKV, ATTN, OPROJ, GATEUP, DOWN; fused: QKV, ATTN, OPROJ, FFN
-    const int LV_N = fused ? 4 : 5;
+    // unfused: QKV, ATTN, OPROJ, GATEUP, DOWN; fused: QKV, ATTN, OPROJ, FFN;
+    // the position-0 schedule has no ATTN level
+    P->is_pos0 = pos0 ? 1 : 0;
+    const int LV_N = (fused ? 4 : 5) - (pos0 ? 1 : 0);
     auto ctr_of = [&](int layer, int lv) { return layer * LV_N + lv; };
     const int n_ctr = L * LV_N;
     std::vector<std::vector<Logical>> levels;
@@ -269,13 +273,18 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
             gemv_level(amk::TK_QKV, l, rows3[m], h, esz, nt, amk::kMaxTaskRows, (uint8_t)m, qkv);
         }
         levels.push_back(std::move(qkv));
-        std::vector<Logical> att;
-        for (int g = 0; g < nkv; ++g)
-            for (int ci = 0; ci < C; ++ci)
-                att.push_back({mk(amk::TK_ATTN, l, g, ci), 0});
-        levels.push_back(std::move(att));
+        if (!pos0) {
+            std::vector<Logical> att;
+            for (int g = 0; g < nkv; ++g)
+                for (int ci = 0; ci < C; ++ci)
+                    att.push_back({mk(amk::TK_ATTN, l, g, ci), 0});
+            levels.push_back(std::move(att));
+        }
         std::vector<Logical> o, gu, dn;
         gemv_level(amk::TK_OPROJ, l, h, nh * hd, esz, target, amk::kMaxTaskRows, 0, o);
+        if (pos0)
+            for (auto &t : o)
+                t.d.flags |= amk::TF_POS0;
         levels.push_back(std::move(o));
         if (fused) {
             std::vector<Logical> ffn;
@@ -428,7 +437,16 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
                 break;
             }
             case amk::TK_OPROJ:
-                acc(B_ATTN(l), AMK_ACC_READ, 0, (int64_t)nh * hd);
+                if (d.flags & amk::TF_POS0) {
+                    // head outputs from the V rows; KV row 0 in shares: the tile
+                    // of rows [r0, r1) writes (K | V) elements [r0 E / h, r1 E / h)
+                    const int64_t E = (int64_t)2 * nkv * hd;
+                    acc(B_QKV(l), AMK_ACC_READ, (int64_t)nh * hd, (int64_t)(nh + 2 * nkv) * hd);
+                    if (d.r0 * E / h < d.r1 * E / h)
+                        acc(B_KVNEW(l), AMK_ACC_WRITE, d.r0 * E / h, d.r1 * E / h);
+                } else {
+                    acc(B_ATTN(l), AMK_ACC_READ, 0, (int64_t)nh * hd);
+                }
                 if (l > 0)
                     acc(B_XOUT(l - 1), AMK_ACC_READ, d.r0, d.r1);
                 else

@@ -18,10 +18,16 @@ struct amk_plan {
     std::vector<amk::TaskDesc> tasks;  // grouped by SM, queue order
     std::vector<int32_t> queue_off;    // [n_sms + 1]
     int n_counters = 0;  // level counters (the validator's graph)
-    int n_arrive = 0;
+    int n_arrive = 0;    // attention arrival counters, [L][nkv], after them
     int att_pg = 1;      // attention position groups per warp
     int ffn_fused = 0;   // 1: one FFN level per layer (gate/up + down column slice)
-    int ffn_box_rows = 0;  // rows of a Wdown TMA box (divides hidden)    // attention arrival counters, [L][nkv], after them
+    int ffn_box_rows = 0;  // rows of a Wdown TMA box (divides hidden)
+    int is_pos0 = 0;     // 1: the schedule of steps at position 0 (no attention level)
+    amk_plan *pos0 = nullptr;  // owned: that schedule, for a plan of all other steps
+    amk_plan() = default;
+    amk_plan(const amk_plan &) = delete;
+    amk_plan &operator=(const amk_plan &) = delete;
+    ~amk_plan() { delete pos0; }
     // the validator's view
     std::vector<amk_graph_task> gtasks;
     std::vector<amk_graph_wait> gwaits;
@@ -33,18 +39,21 @@ struct amk_plan {
     int64_t weight_bytes = 0, kv_row_bytes = 0;
 };
 
-// Lowers cfg for n_sms persistent CTAs into *P (no validation).
-int amk_lower(const amk_config *cfg, const amk_options *opt, int n_sms, amk_plan *P);
+// Lowers cfg for n_sms persistent CTAs into *P (no validation).  With pos0,
+// the schedule of a step at position 0: no attention level, the O-projection
+// takes each head's output from the V rows directly.
+int amk_lower(const amk_config *cfg, const amk_options *opt, int n_sms, amk_plan *P,
+              int pos0 = 0);
 // A non-owning amk_graph view of P's graph arrays.
 void amk_plan_view(const amk_plan *P, amk_graph *g);
-// Copies plan task t into *out with its device pointers resolved: weight
-// rows, row scales and norm gain from w, KV-cache blocks from kv (bf16
-// [L][2][nkv][max_ctx][hd]).  Host only; reads only host memory.
 // Tensor maps of the Wdown of layers [l0, l0 + n) for a fused FFN (128 bytes
 // each, to be copied to 64-byte aligned device memory): a 2-D [hidden][ffn]
 // view with boxes of 16 bytes x ffn_box_rows rows.  Returns an amk status.
 int amk_encode_down_maps(const amk_plan *P, const amk_weights *w, int l0, int n, void *out);
 
+// Copies plan task t into *out with its device pointers resolved: weight
+// rows, row scales and norm gain from w, KV-cache blocks from kv (bf16
+// [L][2][nkv][max_ctx][hd]).  Host only; reads only host memory.
 void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *kv, int t,
                       amk::TaskDesc *out);
 

@@ -126,6 +126,26 @@ def test_ffn_level_variants(name, ctx, fused):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("name", ["tinyllama", "llama1b_w8", "tiny"])
+def test_position0_schedule_matches_general(name):
+    """At position 0 the schedule without the attention level gives the same
+    logits, bit for bit, and the same KV-cache row 0 as the general one."""
+    cfg = si.get_config(name)
+    w = si.make_model(cfg, device="cuda")
+    tok = si.make_prompt(cfg, 1, seed=10)[0]
+    out = []
+    for pos0 in (1, -1):
+        dec = amk.Decoder(cfg, w, amk.default_options(pos0_plan=pos0))
+        lg = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+        am = dec.step(tok, 0, logits=lg)
+        kv0 = [torch.stack(dec.kv(l))[:, :, 0].clone() for l in range(cfg.n_layers)]
+        out.append((lg.clone(), am, kv0))
+        dec.close()
+    assert torch.equal(out[0][0], out[1][0]) and out[0][1] == out[1][1]
+    for a, b in zip(out[0][2], out[1][2]):
+        assert torch.equal(a, b)
+
+
 def test_smol_greedy_32_steps():
     cfg = si.get_config("smol135")
     pair = Pair(cfg)

@@ -78,6 +78,32 @@ def test_real_lowerings_accepted_and_cover(name, n_sms, fused):
     assert ok, (rule, msg)
 
 
+@pytest.mark.parametrize("name", list(si.CONFIGS))
+@pytest.mark.parametrize("fused", [2, -1])
+def test_position0_schedule(name, fused):
+    """The position-0 schedule has no attention level; its O-projection reads
+    the K/V rows, the O tiles write KV row 0 in shares that tile it, and the
+    validator accepts it."""
+    cfg = si.get_config(name)
+    plan = amk.Plan(cfg, 148, amk.default_options(ffn_fused=fused))
+    z = plan.pos0()
+    assert z is not None
+    g = z.graph()
+    kinds, layers = z.task_info()
+    assert not any(KIND[k] == "ATTN" for k in kinds)
+    L, nh, nkv, hd = cfg.n_layers, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    for l in range(L):
+        kvnew = _writes(g, 6 * l + 5)
+        _partition(kvnew, 2 * nkv * hd)
+        assert all(KIND[kinds[t]] == "OPROJ" for _, _, t in kvnew)
+    for q in g["queues"]:
+        seq = [(layers[t], ORDER.index(KIND[kinds[t]])) for t in q]
+        assert seq == sorted(seq)
+    ok, rule, msg = amk.validate_graph(g)
+    assert ok, (rule, msg)
+    assert amk.Plan(cfg, 148, amk.default_options(pos0_plan=-1)).pos0() is None
+
+
 def test_fused_ffn_slices_cover_ffn():
     """The fused FFN level of each layer has about one slice per SM, each a
     multiple of 16 bytes of a Wdown row, and the slices tile [0, ffn)."""
