@@ -375,6 +375,13 @@ __device__ __forceinline__ TaskDesc read_staged(uint32_t slot)
     return d;
 }
 
+// A GEMV's input vector in shared memory is padded by 16 bytes after every
+// 128 (element i at vidx(i)): a lane reads its E-element pieces of the
+// vector with 16-byte loads, and lanes 32 or 64 bytes apart would otherwise
+// share banks (8 lanes of a wavefront into 2 or 4 bank groups); with the
+// padding they fall into 8 distinct groups.
+__device__ __forceinline__ int vidx(int i) { return i + ((i >> 5) << 2); }
+
 // ------------------------------------------------------------- task geometry
 // Both the producer and the consumers derive a task's chunk stream from its
 // record with this function (no memory reads), so they agree on every chunk.
@@ -783,7 +790,7 @@ __device__ void rmsnorm_prologue(const KParams &p, const SmemLayout &s, const fl
     for (int j = 0; j < kMaxPerThread; ++j) {
         const int i = ct + j * kConsumerThreads;
         if (i < n)
-            s.vec[i] = gv[j] * (xv[j] * inv);
+            s.vec[vidx(i)] = gv[j] * (xv[j] * inv);
     }
     consumer_bar();
 }
@@ -809,25 +816,42 @@ __device__ __forceinline__ bool gemv_task(const KParams &p, const SmemLayout &s,
     const int vb = ks * VPS;
     const int ve = min(vb + VPS, NV);
     const int ni = (ve - vb - lane + 31) / 32;  // vectors this lane holds (may be <= 0)
+    // the lane's activations: 16-byte pieces of its vectors (8 bytes when a
+    // vector holds 2 elements), from the padded shared vector or from L2
     f2_t xp[NI][EP];
 #pragma unroll
     for (int i = 0; i < NI; ++i) {
         const int v = vb + lane + 32 * i;
+        if constexpr (E >= 4) {
 #pragma unroll
-        for (int e = 0; e < E; e += 2) {
+            for (int e = 0; e < E; e += 4) {
+                float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (i < ni) {
+                    if (xg) {
+                        t = __ldcg(reinterpret_cast<const float4 *>(xg + v * E + e));
+                    } else {
+                        const uint4 u = lds128(s.vec_a + (uint32_t)vidx(v * E + e) * 4);
+                        t = make_float4(__uint_as_float(u.x), __uint_as_float(u.y),
+                                        __uint_as_float(u.z), __uint_as_float(u.w));
+                    }
+                }
+                xp[i][e / 2] = pk2(t.x, t.y);
+                xp[i][e / 2 + 1] = pk2(t.z, t.w);
+            }
+        } else {
             float a = 0.f, b = 0.f;
             if (i < ni) {
                 if (xg) {
-                    const float2 t = __ldcg(reinterpret_cast<const float2 *>(xg + v * E + e));
+                    const float2 t = __ldcg(reinterpret_cast<const float2 *>(xg + v * E));
                     a = t.x;
                     b = t.y;
                 } else {
-                    const uint2 t = lds64(s.vec_a + (uint32_t)(v * E + e) * 4);
+                    const uint2 t = lds64(s.vec_a + (uint32_t)vidx(v * E) * 4);
                     a = __uint_as_float(t.x);
                     b = __uint_as_float(t.y);
                 }
             }
-            xp[i][e / 2] = pk2(a, b);
+            xp[i][0] = pk2(a, b);
         }
     }
     const uint32_t red_a = s.red_a + (uint32_t)warp * kMaxTaskRows * 4;
@@ -1403,7 +1427,7 @@ __device__ void pos0_prologue(const KParams &p, const SmemLayout &s, const TaskD
     for (int j = 0; j < kMaxPerThread; ++j) {
         const int i = ct + j * kConsumerThreads;
         if (i < N)
-            s.vec[i] = bf16_to_f(f_to_bf16(v[j]));
+            s.vec[vidx(i)] = bf16_to_f(f_to_bf16(v[j]));
     }
     consumer_bar();
 }
@@ -1424,7 +1448,7 @@ __device__ void attn_prologue(const KParams &p, const SmemLayout &s, int l, int 
     for (int j = 0; j < kMaxPerThread; ++j) {
         const int i = ct + j * kConsumerThreads;
         if (i < N)
-            s.vec[i] = v[j];
+            s.vec[vidx(i)] = v[j];
     }
     consumer_bar();
 }

@@ -161,11 +161,12 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     if (C <= 0)
         C = std::max(1, std::min(n_sms / nkv, 8));
     C = std::min(C, c.max_ctx);
-    // the shared vector holds a prologue's output: the normed hidden state,
-    // the combined attention output (+ per-(head, chunk) m / weight and l),
-    // or the attention tile's scratch; DOWN tiles read their activations
-    // from L2 directly
-    int vec = std::max({h, nh * hd + 2 * nh * C,
+    // the shared vector holds a prologue's output (the normed hidden state or
+    // the attention output, padded by 4 floats per 32 for conflict-free
+    // loads), a fused FFN slice's activations, or the attention tile's
+    // scratch; DOWN tiles read their activations from L2 directly
+    auto padded = [](int n) { return n + n / 32 * 4 + 4; };
+    int vec = std::max({padded(h), padded(nh * hd),
                         G * hd + 2 * hd + amk::kConsumerWarps * G * (hd + 2)});
     vec = (vec + 3) & ~3;
     int stages = opt.ring_stages;
