@@ -1399,35 +1399,36 @@ __device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
 __device__ void pos0_prologue(const KParams &p, const SmemLayout &s, const TaskDesc &d, int ct)
 {
     const int l = d.layer, hd = p.head_dim, nh = p.n_heads, nkv = p.n_kv_heads, G = p.group;
-    const int N = nh * hd;
+    const int KV = nkv * hd;  // elements of one of K, V
     const float *qkv = p.qkv + (size_t)l * p.qkv_rows;
-    const float *vsrc = qkv + (size_t)(nh + nkv) * hd;
+    const float *ksrc = qkv + (size_t)nh * hd, *vsrc = ksrc + KV;
+    // element r of V (KV head r / hd) is the output of the G heads of that
+    // group: thread t takes r = t + 256 j, one load and G stores each
     float v[kMaxPerThread];
 #pragma unroll
     for (int j = 0; j < kMaxPerThread; ++j) {
-        const int i = ct + j * kConsumerThreads;
-        v[j] = 0.f;
-        if (i < N) {
-            const int h = i / hd;
-            v[j] = __ldcg(vsrc + (size_t)(h / G) * hd + (i - h * hd));
-        }
+        const int r = ct + j * kConsumerThreads;
+        v[j] = r < KV ? __ldcg(vsrc + r) : 0.f;
     }
     {
-        const int E = 2 * nkv * hd;
+        const int E = 2 * KV;
         const int a = (int)((int64_t)d.r0 * E / p.hidden), b = (int)((int64_t)d.r1 * E / p.hidden);
         const size_t blk = (size_t)p.max_ctx * hd;  // one (layer, K|V, head) block
         for (int i = a + ct; i < b; i += kConsumerThreads) {
-            const int which = i / (nkv * hd), r = i - which * nkv * hd;  // 0: K, 1: V
+            const int which = i >= KV, r = i - which * KV;  // 0: K, 1: V
             const int g = r / hd, e = r - g * hd;
-            p.kv[(((size_t)l * 2 + which) * nkv + g) * blk + e] =
-                f_to_bf16(__ldcg(qkv + (size_t)nh * hd + i));
+            p.kv[(((size_t)l * 2 + which) * nkv + g) * blk + e] = f_to_bf16(__ldcg(ksrc + i));
         }
     }
 #pragma unroll
     for (int j = 0; j < kMaxPerThread; ++j) {
-        const int i = ct + j * kConsumerThreads;
-        if (i < N)
-            s.vec[vidx(i)] = bf16_to_f(f_to_bf16(v[j]));
+        const int r = ct + j * kConsumerThreads;
+        if (r < KV) {
+            const int g = r / hd, e = r - g * hd;
+            const float x = bf16_to_f(f_to_bf16(v[j]));
+            for (int hh = 0; hh < G; ++hh)
+                s.vec[vidx((g * G + hh) * hd + e)] = x;
+        }
     }
     consumer_bar();
 }
