@@ -146,6 +146,39 @@ def test_position0_schedule_matches_general(name):
         assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("edit", [
+    dict(n_kv_heads=1),                 # one KV head for every query head (G = 4)
+    dict(n_kv_heads=4),                 # plain multi-head attention (G = 1)
+    dict(head_dim=128, n_heads=4, n_kv_heads=2, hidden=128),  # wide heads, G = 2
+    dict(n_layers=3, ffn=256),          # FFN rows in 16-byte multiples: fused level
+])
+def test_tiny_shape_variants_to_the_last_cache_row(edit):
+    """Greedy decode through every position of the cache (0 .. max_ctx - 1,
+    the last row included) on variants of the tiny decoder, against the
+    oracle, teacher-forced where the top-2 margin is within the bound."""
+    cfg = si.get_config("tiny").with_(name="tiny_var", max_ctx=24, **edit)
+    pair = Pair(cfg, options=amk.default_options(ffn_fused=2))
+    prompt = si.make_prompt(cfg, 3)
+    worst, checked = greedy_teacher_forced(pair, prompt, cfg.max_ctx - len(prompt))
+    assert checked >= cfg.max_ctx // 2
+    with pytest.raises(amk.AmkError) as e:
+        pair.dec.step(1, cfg.max_ctx)
+    assert e.value.name == "AMK_ERR_POS_RANGE"
+
+
+def test_ragged_sm_count_full_size():
+    """A full-size shape on a prime number of CTAs (ragged tiles on every
+    level, several tasks per queue) against the oracle at a long context."""
+    cfg = si.get_config("tinyllama")
+    pair = Pair(cfg, options=amk.default_options(n_sms=37))
+    pair.fill_kv(300)
+    tok = si.make_prompt(cfg, 1, seed=10)[0]
+    g, am, ref, ref_am = pair.step(tok, 300)
+    compare(cfg, g, am, ref, ref_am, "tinyllama on 37 CTAs, ctx 300")
+    del pair
+    torch.cuda.empty_cache()
+
+
 def test_smol_greedy_32_steps():
     cfg = si.get_config("smol135")
     pair = Pair(cfg)
