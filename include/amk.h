@@ -121,7 +121,17 @@ typedef struct {
     int32_t pos0_plan;        /* 1 (default): steps at position 0 run a second, validated
                                  schedule without the attention level (softmax over one
                                  key: each head's output is its KV head's V row); -1: off */
-    int32_t reserved[4];
+    int32_t inflight_kb;      /* cap on the weight bytes each SM's bulk copies keep in flight
+                                 (KiB; 0 = default 64, < 0 = no cap).  Queued copies delay
+                                 every other memory access of the SM: with 192 KiB in flight
+                                 an L2 hit takes ~1.2 us and a grid-wide counter round ~12
+                                 us on B200, with 64 KiB ~0.6 us and ~3 us, while the stream
+                                 still reaches ~96% of its bandwidth */
+    int32_t copy_piece_kb;    /* largest piece a ring stage's copy is issued in, each piece
+                                 on its own mbarrier (KiB; 0 = default 64: one piece per
+                                 stage; smaller pieces let the cap bind more finely but cost
+                                 the producer more issue work) */
+    int32_t reserved[2];
 } amk_options;
 
 typedef struct amk_handle amk_handle;

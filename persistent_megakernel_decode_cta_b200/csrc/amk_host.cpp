@@ -484,6 +484,8 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     k.timeout_ns = (uint64_t)P->opt.wait_timeout_us * 1000ull;
     k.skip_signal_task = P->opt.debug_skip_signal_task;
     k.lookahead = (uint32_t)std::max(0, P->opt.l2_prefetch_kb) * 1024u;
+    k.inflight = amk_inflight_bytes(&P->opt);
+    k.piece = amk_piece_bytes(&P->opt);
     k.prof = H->d_prof;
     *out = H;
     return AMK_OK;

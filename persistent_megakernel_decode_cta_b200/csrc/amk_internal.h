@@ -35,6 +35,11 @@ static_assert(kProducerThreads * kProducerRegs + kConsumerThreads * kConsumerReg
                   kThreads * kLaunchRegs, "register split must equal the launch budget");
 constexpr int kMaxTaskRows = 256;   // output rows of one GEMV task (red buffer)
 constexpr int kMaxStages = 16;
+// A ring stage's copy goes out in up to kPieces pieces of about KParams::piece bytes,
+// each completing on its own mbarrier, so that the producer can keep a
+// bounded number of bytes in flight (KParams::inflight).
+constexpr int kPieces = 4;
+constexpr int kPieceQueue = 32;     // pieces the producer tracks at once
 
 // Task kinds (the instruction set: GEMV row tiles with fused prologues and
 // epilogues, and the split-K attention tile).
@@ -132,6 +137,8 @@ struct KParams {
     int32_t parity;             // epoch & 1
     uint64_t timeout_ns;
     uint32_t lookahead;         // L2 prefetch distance past the ring copies (bytes), 0 = off
+    uint32_t inflight;          // cap on bulk-copy bytes in flight per SM (0xffffffff: none)
+    uint32_t piece;             // bytes of a copy piece (multiple of 16)
     int32_t skip_signal_task;   // test hook, -1 = off
     unsigned long long *prof;   // [n_sms][kProfKinds][kProfFields] phase timers, or null
 };

@@ -68,6 +68,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
         : "memory");
     return ok != 0;
 }
+// Non-blocking test of the same phase completion (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
                                          uint32_t bar, uint64_t policy)
 {
@@ -308,11 +321,12 @@ struct SmemLayout {
     uint8_t *ring;        // ring_stages * stage_bytes
     float *vec;           // vec_floats: the task's input vector / scratch
     float *red;           // [kConsumerWarps][kMaxTaskRows]
-    uint64_t *full;       // [kMaxStages]
+    uint64_t *full;       // [kMaxStages][kPieces]: stage st, piece pc at st * kPieces + pc
     uint64_t *empty;      // [kMaxStages]
     int *flags;           // [0] abort
     float *scr;           // 64 floats of reduction scratch
     unsigned long long *wacc;  // [2] per-task sums over warps (profiling)
+    uint4 *pq;            // [kPieceQueue] producer's pieces in flight: (bar, parity, bytes, chunk)
     uint32_t ring_a, vec_a, red_a, full_a, empty_a;  // shared addresses
     uint32_t ptask_a, ctask_a;  // [2] staged task records of producer / consumers
 };
@@ -328,7 +342,7 @@ __device__ __forceinline__ SmemLayout smem_layout(uint8_t *base, const KParams &
     s.red = reinterpret_cast<float *>(base + off);
     off += (size_t)kConsumerWarps * kMaxTaskRows * 4;
     s.full = reinterpret_cast<uint64_t *>(base + off);
-    off += kMaxStages * 8;
+    off += kMaxStages * kPieces * 8;
     s.empty = reinterpret_cast<uint64_t *>(base + off);
     off += kMaxStages * 8;
     s.flags = reinterpret_cast<int *>(base + off);
@@ -337,6 +351,8 @@ __device__ __forceinline__ SmemLayout smem_layout(uint8_t *base, const KParams &
     off += 64 * 4;
     s.wacc = reinterpret_cast<unsigned long long *>(base + off);
     off += 16;
+    s.pq = reinterpret_cast<uint4 *>(base + off);
+    off += kPieceQueue * 16;
     s.ptask_a = smem_u32(base + off);
     off += 2 * sizeof(TaskDesc);
     s.ctask_a = smem_u32(base + off);
@@ -440,14 +456,22 @@ __device__ __forceinline__ Geom task_geom(const KParams &p, const TaskDesc &d)
     int rpc = p.stage_bytes / g.RB;
     rpc -= rpc % gran;
     // warp layout: each lane keeps at most 64 activations of its K-slice in
-    // registers; split K across more warps only when a row needs it, so that
-    // every warp reduces whole rows with as few shuffles as possible
+    // registers.  K is split across more warps when a row needs it, and also
+    // while that gives every warp fewer than four rows of a chunk (the GEMV
+    // takes rows four at a time) and still leaves each lane a whole vector
     g.VB = (g.RB % 16 == 0) ? 16 : ((g.RB % 8 == 0) ? 8 : 4);
     const int NV = g.RB / g.VB;
     const int max_vec = 64 / (g.VB / esz);  // vectors a lane may hold
+    const int rows = min(rpc, d.r1 - d.r0);
     int KS = 1;
-    while (KS < kConsumerWarps && (NV > KS * 32 * max_vec || kConsumerWarps / KS > rpc))
+    while (KS < kConsumerWarps) {
+        const int rgk = kConsumerWarps / KS;
+        const bool must = NV > KS * 32 * max_vec || rgk > rpc;
+        const bool more_rows = rgk * 4 > rows && NV >= 2 * KS * 32;
+        if (!must && !more_rows)
+            break;
         KS *= 2;
+    }
     g.KS = KS;
     g.RG = kConsumerWarps / KS;
     const int step = g.RG > gran ? g.RG : gran;  // rows per chunk: a multiple of both
@@ -547,6 +571,67 @@ __device__ __forceinline__ void lookahead_pump(const KParams &p, Lookahead &la, 
     }
 }
 
+// Bulk-copy bytes in flight.  Copies the producer has issued wait in the
+// SM's memory queues together with every other access of the SM, so the
+// more there are, the longer each L2 hit, counter poll and release takes
+// (on B200 an L2 hit goes from ~0.2 us idle to ~0.6 us with 64 KiB in
+// flight per SM and ~1.2 us with 192 KiB, while 64 KiB already draws ~96 %
+// of the stream bandwidth).  The producer therefore issues each chunk in
+// pieces on their own mbarriers and keeps at most p.inflight bytes
+// outstanding; the ring still fills completely while consumers wait.
+struct Flight {
+    uint32_t head, tail;  // queue positions (pieces issued: tail)
+    uint32_t bytes;       // bytes of the queued pieces
+};
+
+// Drops completed pieces from the front of the queue, and every piece of
+// a chunk below `done_below` (those are known complete: their stage has
+// been consumed).
+__device__ __forceinline__ void flight_retire(const SmemLayout &s, Flight &f, uint32_t done_below)
+{
+    while (f.head != f.tail) {
+        const uint4 e = s.pq[f.head % kPieceQueue];
+        if (e.w >= done_below && !mbar_test_wait(e.x, e.y))
+            break;
+        f.bytes -= e.z;
+        ++f.head;
+    }
+}
+
+// Waits (bounded) until `bytes` more fit under the cap; false on abort.
+__device__ bool flight_reserve(const KParams &p, const SmemLayout &s, Flight &f, uint32_t bytes,
+                               uint32_t done_below, uint64_t &prof_wait)
+{
+    flight_retire(s, f, done_below);
+    volatile int *abort_flag = s.flags;
+    uint32_t it = 0;
+    uint64_t t0 = 0;
+    while (f.head != f.tail && (f.bytes + bytes > p.inflight || f.tail - f.head >= kPieceQueue)) {
+        const uint4 e = s.pq[f.head % kPieceQueue];
+        if (mbar_try_wait(e.x, e.y)) {
+            f.bytes -= e.z;
+            ++f.head;
+            continue;
+        }
+        if (it == 0)
+            t0 = gtimer();
+        if ((++it & 255) == 0 &&
+            (*abort_flag || gtimer() - t0 > p.timeout_ns * 4 || it > (1u << 30)))
+            return false;
+    }
+    if (p.prof && it)
+        prof_wait += gtimer() - t0;
+    return true;
+}
+
+__device__ __forceinline__ void flight_push(const SmemLayout &s, Flight &f, uint32_t bar,
+                                            uint32_t par, uint32_t bytes, uint32_t chunk)
+{
+    s.pq[f.tail % kPieceQueue] = make_uint4(bar, par, bytes, chunk);
+    ++f.tail;
+    f.bytes += bytes;
+}
+
 // Lane 0 of the producer warpgroup streams every chunk of every task of this
 // SM's queue into the ring, one task record ahead.
 __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int qe)
@@ -561,6 +646,7 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
     Lookahead la{};
     la.ti = qb - 1;
     la.part = 2;
+    Flight fl{0u, 0u, 0u};
     if (qb < qe)
         stage_task(s.ptask_a, p.tasks + qb);
     for (int ti = qb; ti < qe && !stop; ++ti) {
@@ -575,6 +661,7 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
         const uint8_t *w1 = static_cast<const uint8_t *>(d.w1);
         for (int i = 0; i < g.nchunks; ++i, ++k) {
             const int st = k % NS;
+            const uint32_t done_below = k >= (uint32_t)NS ? k - NS + 1 : 0u;
             if (k >= (uint32_t)NS) {
                 const uint32_t par = ((k / NS) - 1) & 1;
                 uint32_t it = 0;
@@ -599,55 +686,100 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
                     prof_wait += gtimer() - t0;
             }
             const uint32_t dst = s.ring_a + (uint32_t)st * p.stage_bytes;
-            const uint32_t bar = s.full_a + 8 * st;
+            const uint32_t bar0 = s.full_a + 8 * (st * kPieces);
+            const uint32_t par = (k / NS) & 1;
             if (p.prof && i == 0)  // time from the task's start to its first copy
                 prof_setup += (gtimer() - ts) - (prof_wait - wait_before);
+            int used = 0;  // piece barriers armed for this chunk
             if (d.kind == TK_ATTN) {
+                // K rows on piece 0, V rows on piece 1
                 const int a = g.pa + i * g.P;
                 const int b = min(a + g.P, g.pb);
                 const uint32_t nb = (uint32_t)(b - a) * p.head_dim * 2;
-                mbar_arrive_expect_tx(bar, 2 * nb);
-                bulk_g2s_nohint(dst, w0 + (size_t)a * p.head_dim * 2, nb, bar);
-                bulk_g2s_nohint(dst + (uint32_t)g.P * p.head_dim * 2,
-                                w1 + (size_t)a * p.head_dim * 2, nb, bar);
+                for (int h = 0; h < 2 && !stop; ++h) {
+                    if (!flight_reserve(p, s, fl, nb, done_below, prof_wait)) {
+                        stop = true;
+                        break;
+                    }
+                    const uint32_t bar = bar0 + 8 * h;
+                    mbar_arrive_expect_tx(bar, nb);
+                    bulk_g2s_nohint(dst + (uint32_t)h * g.P * p.head_dim * 2,
+                                    (h ? w1 : w0) + (size_t)a * p.head_dim * 2, nb, bar);
+                    flight_push(s, fl, bar, par, nb, k);
+                    ++used;
+                }
                 prof_bytes += 2 * nb;
                 cpos += 2 * nb;
             } else if (i >= g.ngu) {
                 // fused FFN, Wdown part: rows [r0w, r0w + nrows) of the slice's
                 // 16-byte column groups jb, at (jb nrows + row) * 16 in the stage:
                 // one bulk copy per group from the packed copy, or TMA boxes of
-                // 16 bytes x br rows from the caller's Wdown
+                // 16 bytes x br rows from the caller's Wdown; all on piece 0
                 const int r0w = (i - g.ngu) * g.rpc2;
                 const int nrows = min(g.rpc2, p.hidden - r0w);
                 const uint32_t nb = (uint32_t)(nrows * g.ncb * 16);
-                mbar_arrive_expect_tx(bar, nb);
-                if (p.dpack) {
-                    const uint8_t *src = p.dpack + (size_t)d.layer * p.hidden * p.ffn * g.esz +
-                                         ((size_t)(d.r0 / (16 / g.esz)) * p.hidden + r0w) * 16;
-                    for (int jb = 0; jb < g.ncb; ++jb)
-                        bulk_g2s(dst + (uint32_t)(jb * nrows * 16),
-                                 src + (size_t)jb * p.hidden * 16, (uint32_t)nrows * 16, bar,
-                                 pol_w);
+                if (!flight_reserve(p, s, fl, nb, done_below, prof_wait)) {
+                    stop = true;
                 } else {
-                    const int br = p.ffn_box_rows;
-                    const void *tmap =
-                        static_cast<const uint8_t *>(p.dmaps) + (size_t)d.layer * 128;
-                    for (int ib = 0; ib < nrows / br; ++ib)
+                    mbar_arrive_expect_tx(bar0, nb);
+                    if (p.dpack) {
+                        const uint8_t *src = p.dpack +
+                                             (size_t)d.layer * p.hidden * p.ffn * g.esz +
+                                             ((size_t)(d.r0 / (16 / g.esz)) * p.hidden + r0w) * 16;
                         for (int jb = 0; jb < g.ncb; ++jb)
-                            tma_load_2d(dst + (uint32_t)((jb * nrows + ib * br) * 16), tmap,
-                                        d.r0 + jb * (16 / g.esz), r0w + ib * br, bar, pol_w);
+                            bulk_g2s(dst + (uint32_t)(jb * nrows * 16),
+                                     src + (size_t)jb * p.hidden * 16, (uint32_t)nrows * 16,
+                                     bar0, pol_w);
+                    } else {
+                        const int br = p.ffn_box_rows;
+                        const void *tmap =
+                            static_cast<const uint8_t *>(p.dmaps) + (size_t)d.layer * 128;
+                        for (int ib = 0; ib < nrows / br; ++ib)
+                            for (int jb = 0; jb < g.ncb; ++jb)
+                                tma_load_2d(dst + (uint32_t)((jb * nrows + ib * br) * 16), tmap,
+                                            d.r0 + jb * (16 / g.esz), r0w + ib * br, bar0,
+                                            pol_w);
+                    }
+                    flight_push(s, fl, bar0, par, nb, k);
+                    used = 1;
                 }
                 prof_bytes += nb;
                 cpos += nb;
             } else {
+                // GEMV rows: one contiguous range, split into up to kPieces
+                // pieces of about p.piece bytes (multiples of 16 bytes)
                 const int part = i / g.nck, c = i % g.nck;
                 const int r = c * g.rpc;
                 const int nr = min(g.rpc, g.R - r);
                 const uint32_t nb = (uint32_t)nr * g.RB;
-                mbar_arrive_expect_tx(bar, nb);
-                bulk_g2s(dst, (part ? w1 : w0) + (size_t)r * g.RB, nb, bar, pol_w);
+                const uint8_t *src = (part ? w1 : w0) + (size_t)r * g.RB;
+                const uint32_t np = max(1u, min((uint32_t)kPieces, (nb + p.piece - 1) / p.piece));
+                const uint32_t ps = ((nb + np - 1) / np + 15u) & ~15u;
+                for (uint32_t pc = 0; pc < np; ++pc) {
+                    const uint32_t off = pc * ps;
+                    if (off >= nb)
+                        break;
+                    const uint32_t len = min(ps, nb - off);
+                    if (!flight_reserve(p, s, fl, len, done_below, prof_wait)) {
+                        stop = true;
+                        break;
+                    }
+                    const uint32_t bar = bar0 + 8 * pc;
+                    mbar_arrive_expect_tx(bar, len);
+                    bulk_g2s(dst + off, src + off, len, bar, pol_w);
+                    flight_push(s, fl, bar, par, len, k);
+                    ++used;
+                }
                 prof_bytes += nb;
                 cpos += nb;
+            }
+            // the chunk's unused piece barriers complete this phase at once (on
+            // an abort too, so that the drain below can wait for the chunk)
+            for (int pc = used; pc < kPieces; ++pc)
+                mbar_arrive(bar0 + 8 * pc);
+            if (stop) {
+                ++k;
+                break;
             }
         }
     }
@@ -664,27 +796,31 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
     for (uint32_t j = first; j < k; ++j) {
         const int st = j % NS;
         const uint32_t par = (j / NS) & 1;
-        uint32_t it = 0;
-        const uint64_t t1 = gtimer();
-        while (!mbar_try_wait(s.full_a + 8 * st, par)) {
-            if ((++it & 255) == 0 && (gtimer() - t1 > p.timeout_ns || it > (1u << 30)))
-                break;
+        for (int pc = 0; pc < kPieces; ++pc) {
+            uint32_t it = 0;
+            const uint64_t t1 = gtimer();
+            while (!mbar_try_wait(s.full_a + 8 * (st * kPieces + pc), par)) {
+                if ((++it & 255) == 0 && (gtimer() - t1 > p.timeout_ns || it > (1u << 30)))
+                    break;
+            }
         }
     }
 }
 
 // ------------------------------------------------------------------ consumers
-// Waits (all lanes of a warp together) until the ring stage of chunk k is full.
-// All lanes of a warp poll the barrier together (one SIMT instruction).
+// Waits (all lanes of a warp together) until the ring stage of chunk k is full:
+// lane l polls piece l % kPieces of the stage, so one SIMT poll covers every
+// piece barrier.
 __device__ __forceinline__ bool wait_full(const KParams &p, const SmemLayout &s, uint32_t k)
 {
     const int st = k % p.ring_stages;
     const uint32_t par = (k / p.ring_stages) & 1;
+    const uint32_t bar = s.full_a + 8 * (st * kPieces + (threadIdx.x & (kPieces - 1)));
     volatile int *abort_flag = s.flags;
     uint32_t it = 0;
     uint64_t t0 = 0;
     while (true) {
-        const bool ok = mbar_try_wait(s.full_a + 8 * st, par);
+        const bool ok = mbar_try_wait(bar, par);
         if (__all_sync(0xffffffffu, ok))
             return true;
         if (it == 0)
@@ -919,6 +1055,271 @@ __device__ __forceinline__ bool gemv_task(const KParams &p, const SmemLayout &s,
     return true;
 }
 
+// Sums RW per-lane row partials over the warp with a transposed exchange:
+// the first log2(RW) steps trade halves of the rows between lane groups, so
+// four rows cost six shuffles and two rows five, instead of five per row.
+// Afterwards every lane of group l >> (5 - log2 RW) holds that row's total.
+template <int RW>
+__device__ __forceinline__ float warp_rows_sum(float (&s)[RW], int lane)
+{
+    constexpr unsigned FULL = 0xffffffffu;
+    if constexpr (RW == 4) {
+        const bool up = lane & 16;
+        s[0] = (up ? s[2] : s[0]) + __shfl_xor_sync(FULL, up ? s[0] : s[2], 16);
+        s[1] = (up ? s[3] : s[1]) + __shfl_xor_sync(FULL, up ? s[1] : s[3], 16);
+        const bool up8 = lane & 8;
+        s[0] = (up8 ? s[1] : s[0]) + __shfl_xor_sync(FULL, up8 ? s[0] : s[1], 8);
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1)
+            s[0] += __shfl_xor_sync(FULL, s[0], o);
+    } else if constexpr (RW == 2) {
+        const bool up = lane & 16;
+        s[0] = (up ? s[1] : s[0]) + __shfl_xor_sync(FULL, up ? s[0] : s[1], 16);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1)
+            s[0] += __shfl_xor_sync(FULL, s[0], o);
+    } else {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            s[0] += __shfl_xor_sync(FULL, s[0], o);
+    }
+    return s[0];
+}
+
+// int16 x int8 two-way dot products into an int32 accumulator: the 16-bit
+// halves of a times bytes 0, 1 (lo) or 2, 3 (hi) of b.
+__device__ __forceinline__ int dp2a_lo(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp2a.lo.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp2a.hi.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// The lane's activations for a GEMV with 16-byte weight vectors.  bf16
+// weights: f[i][e], element e of vector i as a float.  int8 weights: the
+// lane quantises its own activations to int16 with one scale (|error| <= half
+// a step = max|x| / 65534 per element) and packs them in pairs, q[i][k] =
+// elements 2k, 2k + 1 of vector i; the int8 x int16 products then add up
+// exactly in int32 (a lane's sum stays below 64 * 127 * 32767 < 2^31).
+template <int ESZ, int NI_>
+struct LaneX {
+    static constexpr int E = 16 / ESZ;   // elements per vector
+    static constexpr int NI = NI_;       // vectors per lane at most (NI E <= 64 activations)
+    float f[ESZ == 2 ? NI : 1][ESZ == 2 ? E : 1];
+    uint32_t q[ESZ == 1 ? NI : 1][8];
+    float scale;                         // int8: value of one int16 step
+};
+
+// Rows j0 + RG r (r < RW) of a ring chunk against the lane's activations;
+// each row's warp total goes to red[rowbase + row] (the warp's red slice).
+template <int ESZ, int NI, int RW>
+__device__ __forceinline__ void gemv_rows(const LaneX<ESZ, NI> &x, uint32_t lane_a, int RB, int RG,
+                                          int j0, int ni, uint32_t red_a, int rowbase, int lane)
+{
+    float sr[RW];
+    if constexpr (ESZ == 2) {
+        float acc[RW][4];
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                acc[r][q] = 0.f;
+#pragma unroll
+        for (int i = 0; i < NI; ++i) {
+            if (i < ni) {
+                uint4 w[RW];
+#pragma unroll
+                for (int r = 0; r < RW; ++r)
+                    w[r] = lds128(lane_a + (uint32_t)((j0 + r * RG) * RB + i * 512));
+#pragma unroll
+                for (int r = 0; r < RW; ++r) {
+                    const uint32_t A[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        acc[r][q] = fmaf(__uint_as_float(A[q] << 16), x.f[i][2 * q], acc[r][q]);
+                        acc[r][q] = fmaf(__uint_as_float(A[q] & 0xffff0000u), x.f[i][2 * q + 1],
+                                         acc[r][q]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+            sr[r] = (acc[r][0] + acc[r][1]) + (acc[r][2] + acc[r][3]);
+    } else {
+        int acc[RW][2];
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+            acc[r][0] = acc[r][1] = 0;
+#pragma unroll
+        for (int i = 0; i < NI; ++i) {
+            if (i < ni) {
+                uint4 w[RW];
+#pragma unroll
+                for (int r = 0; r < RW; ++r)
+                    w[r] = lds128(lane_a + (uint32_t)((j0 + r * RG) * RB + i * 512));
+#pragma unroll
+                for (int r = 0; r < RW; ++r) {
+                    const uint32_t A[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        acc[r][0] = dp2a_lo(x.q[i][2 * q], A[q], acc[r][0]);
+                        acc[r][1] = dp2a_hi(x.q[i][2 * q + 1], A[q], acc[r][1]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+            sr[r] = (float)(acc[r][0] + acc[r][1]) * x.scale;
+    }
+    const float tot = warp_rows_sum<RW>(sr, lane);
+    constexpr int SH = RW == 4 ? 3 : RW == 2 ? 4 : 5;
+    if ((lane & ((1 << SH) - 1)) == 0)
+        stsf(red_a + (uint32_t)(rowbase + j0 + (lane >> SH) * RG) * 4, tot);
+}
+
+// GEMV over a task's chunks with 16-byte weight vectors (every shape whose
+// rows are a multiple of 16 bytes).  Warp w = rg + RG ks owns K-slice ks of
+// the rows rg, rg + RG, ... of every chunk, and takes them four at a time
+// (then two, then one): four independent rows per weight-vector load and
+// four accumulators per row keep the FMA or dp2a pipes fed, and one
+// transposed shuffle reduction serves the four rows.  NI (vectors a lane
+// holds) is a template parameter so that the activation registers are sized
+// to the shape, not to the largest one.
+template <int ESZ, int NI>
+__device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &s, const Geom g,
+                                            uint32_t &kc, int warp, int lane, const float *xg,
+                                            uint64_t *wt)
+{
+    using LX = LaneX<ESZ, NI>;
+    constexpr int E = LX::E;
+    const int NV = g.RB / 16;
+    const int VPS = (NV + g.KS - 1) / g.KS;
+    const int RG = g.RG, RB = g.RB, rpc = g.rpc, R = g.R, nck = g.nck;
+    const int rg = warp % RG, ks = warp / RG;
+    const int vb = ks * VPS;
+    const int ve = min(vb + VPS, NV);
+    const int ni = (ve - vb - lane + 31) / 32;  // vectors this lane holds (may be <= 0)
+    LX x;
+    {
+        float xf[NI][E];
+#pragma unroll
+        for (int i = 0; i < NI; ++i) {
+            const int v = vb + lane + 32 * i;
+#pragma unroll
+            for (int e = 0; e < E; e += 4) {
+                float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (i < ni) {
+                    if (xg) {
+                        t = __ldcg(reinterpret_cast<const float4 *>(xg + v * E + e));
+                    } else {
+                        const uint4 u = lds128(s.vec_a + (uint32_t)vidx(v * E + e) * 4);
+                        t = make_float4(__uint_as_float(u.x), __uint_as_float(u.y),
+                                        __uint_as_float(u.z), __uint_as_float(u.w));
+                    }
+                }
+                xf[i][e] = t.x;
+                xf[i][e + 1] = t.y;
+                xf[i][e + 2] = t.z;
+                xf[i][e + 3] = t.w;
+            }
+        }
+        if constexpr (ESZ == 2) {
+#pragma unroll
+            for (int i = 0; i < NI; ++i)
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    x.f[i][e] = xf[i][e];
+            x.scale = 1.f;
+        } else {
+            float amax = 0.f;
+#pragma unroll
+            for (int i = 0; i < NI; ++i)
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    amax = fmaxf(amax, fabsf(xf[i][e]));
+            const float inv = amax > 0.f ? 32767.f / amax : 0.f;
+            x.scale = amax * (1.f / 32767.f);
+#pragma unroll
+            for (int i = 0; i < NI; ++i)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int a = max(-32767, min(32767, __float2int_rn(xf[i][2 * k] * inv)));
+                    const int b = max(-32767, min(32767, __float2int_rn(xf[i][2 * k + 1] * inv)));
+                    x.q[i][k] = ((uint32_t)a & 0xffffu) | ((uint32_t)b << 16);
+                }
+        }
+    }
+    const uint32_t red_a = s.red_a + (uint32_t)warp * kMaxTaskRows * 4;
+    const int NS = p.ring_stages, SB = p.stage_bytes;
+    uint64_t tA = 0, tB = 0;
+    for (int c = 0; c < g.ngu; ++c) {
+        if (wt)
+            tA = gtimer();
+        if (!wait_full(p, s, kc))
+            return false;
+        if (wt) {
+            tB = gtimer();
+            wt[0] += tB - tA;
+        }
+        const uint32_t stage_a = s.ring_a + (uint32_t)(kc % NS) * SB;
+        const int part = c / nck, cc = c - part * nck;
+        const int r0 = cc * rpc;
+        const int nr = min(rpc, R - r0);
+        const int rowbase = part * R + r0;
+        const uint32_t lane_a = stage_a + (uint32_t)(vb + lane) * 16;
+        const int nrw = nr > rg ? (nr - rg + RG - 1) / RG : 0;  // rows rg + RG m, m < nrw
+        int m = 0;
+        for (; m + 4 <= nrw; m += 4)
+            gemv_rows<ESZ, NI, 4>(x, lane_a, RB, RG, rg + RG * m, ni, red_a, rowbase, lane);
+        if (m + 2 <= nrw) {
+            gemv_rows<ESZ, NI, 2>(x, lane_a, RB, RG, rg + RG * m, ni, red_a, rowbase, lane);
+            m += 2;
+        }
+        if (m < nrw)
+            gemv_rows<ESZ, NI, 1>(x, lane_a, RB, RG, rg + RG * m, ni, red_a, rowbase, lane);
+        release_stage(p, s, kc, lane);
+        ++kc;
+        if (wt)
+            wt[1] += gtimer() - tB;
+    }
+    return true;
+}
+
+// Dispatch on the vectors a lane holds for this task's K-slice.
+template <int ESZ>
+__device__ __forceinline__ bool gemv16(const KParams &p, const SmemLayout &s, const Geom &g,
+                                       uint32_t &kc, int warp, int lane, const float *xg,
+                                       uint64_t *wt)
+{
+    const int vps = (g.RB / 16 + g.KS - 1) / g.KS;
+    const int nimax = (vps + 31) / 32;
+    if constexpr (ESZ == 2) {
+        if (nimax <= 2)
+            return gemv16_task<2, 2>(p, s, g, kc, warp, lane, xg, wt);
+        if (nimax <= 4)
+            return gemv16_task<2, 4>(p, s, g, kc, warp, lane, xg, wt);
+        if (nimax <= 6)
+            return gemv16_task<2, 6>(p, s, g, kc, warp, lane, xg, wt);
+        return gemv16_task<2, 8>(p, s, g, kc, warp, lane, xg, wt);
+    } else {
+        if (nimax <= 1)
+            return gemv16_task<1, 1>(p, s, g, kc, warp, lane, xg, wt);
+        if (nimax <= 2)
+            return gemv16_task<1, 2>(p, s, g, kc, warp, lane, xg, wt);
+        if (nimax <= 3)
+            return gemv16_task<1, 3>(p, s, g, kc, warp, lane, xg, wt);
+        return gemv16_task<1, 4>(p, s, g, kc, warp, lane, xg, wt);
+    }
+}
+
 // Fast instances (GENERIC = 0) only run 16-byte weight vectors in the
 // model's own format; the generic instance dispatches every variant at run
 // time (models with odd row widths, or a bf16 tied head on int8 layers).
@@ -929,19 +1330,19 @@ __device__ __forceinline__ bool run_gemv(const KParams &p, const SmemLayout &s, 
 {
     if constexpr (!GENERIC) {
         if constexpr (Q8)
-            return gemv_task<1, 16>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16<1>(p, s, g, kc, warp, lane, xg, wt);
         else
-            return gemv_task<2, 16>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16<2>(p, s, g, kc, warp, lane, xg, wt);
     } else {
         if (g.esz == 2) {
             if (g.VB == 16)
-                return gemv_task<2, 16>(p, s, g, kc, warp, lane, xg, wt);
+                return gemv16<2>(p, s, g, kc, warp, lane, xg, wt);
             if (g.VB == 8)
                 return gemv_task<2, 8>(p, s, g, kc, warp, lane, xg, wt);
             return gemv_task<2, 4>(p, s, g, kc, warp, lane, xg, wt);
         }
         if (g.VB == 16)
-            return gemv_task<1, 16>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16<1>(p, s, g, kc, warp, lane, xg, wt);
         if (g.VB == 8)
             return gemv_task<1, 8>(p, s, g, kc, warp, lane, xg, wt);
         return gemv_task<1, 4>(p, s, g, kc, warp, lane, xg, wt);
@@ -1783,7 +2184,8 @@ __global__ void __launch_bounds__(kThreads, 1) amk_decode_kernel(const __grid_co
 
     if (tid == 0) {
         for (int i = 0; i < p.ring_stages; ++i) {
-            mbar_init(s.full_a + 8 * i, 1);
+            for (int pc = 0; pc < kPieces; ++pc)
+                mbar_init(s.full_a + 8 * (i * kPieces + pc), 1);
             mbar_init(s.empty_a + 8 * i, kConsumerWarps);
         }
         // a failed earlier step poisons the device state: do no work until the
@@ -1825,7 +2227,8 @@ __global__ void amk_pack_down_kernel(const uint4 *wd, uint4 *out, int h, int ncg
 extern "C" int amk_kernel_smem_bytes(int ring_stages, int stage_bytes, int vec_floats)
 {
     return ring_stages * stage_bytes + vec_floats * 4 + kConsumerWarps * kMaxTaskRows * 4 +
-           2 * kMaxStages * 8 + 16 * 4 + 64 * 4 + 2 * 8 + 4 * (int)sizeof(TaskDesc);
+           (kPieces + 1) * kMaxStages * 8 + 16 * 4 + 64 * 4 + 2 * 8 + kPieceQueue * 16 +
+           4 * (int)sizeof(TaskDesc);
 }
 
 namespace {

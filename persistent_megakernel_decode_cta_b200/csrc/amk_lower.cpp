@@ -88,6 +88,8 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         if (opt_in->l2_prefetch_kb > 0) opt.l2_prefetch_kb = opt_in->l2_prefetch_kb;
         if (opt_in->ffn_fused != 0) opt.ffn_fused = opt_in->ffn_fused;
         if (opt_in->pos0_plan != 0) opt.pos0_plan = opt_in->pos0_plan;
+        if (opt_in->inflight_kb != 0) opt.inflight_kb = opt_in->inflight_kb;
+        if (opt_in->copy_piece_kb > 0) opt.copy_piece_kb = opt_in->copy_piece_kb;
         opt.n_sms = opt_in->n_sms;
     }
     const amk_config &c = *cfg;

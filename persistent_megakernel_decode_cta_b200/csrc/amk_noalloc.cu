@@ -243,6 +243,8 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     k.timeout_ns = (uint64_t)P.opt.wait_timeout_us * 1000ull;
     k.skip_signal_task = P.opt.debug_skip_signal_task;
     k.lookahead = (uint32_t)(P.opt.l2_prefetch_kb > 0 ? P.opt.l2_prefetch_kb : 0) * 1024u;
+    k.inflight = amk_inflight_bytes(&P.opt);
+    k.piece = amk_piece_bytes(&P.opt);
     e = amk_kernel_configure(P.smem_bytes, q8 ? 1 : 0, P.att_e, P.generic);
     if (e != cudaSuccess)
         return fail_cuda(e, "cudaFuncSetAttribute");

@@ -44,6 +44,21 @@ struct amk_plan {
 // takes each head's output from the V rows directly.
 int amk_lower(const amk_config *cfg, const amk_options *opt, int n_sms, amk_plan *P,
               int pos0 = 0);
+// The producer's cap on bulk-copy bytes in flight per SM for options o:
+// inflight_kb KiB, 64 KiB when 0, no cap when negative.
+inline uint32_t amk_inflight_bytes(const amk_options *o)
+{
+    if (o->inflight_kb < 0)
+        return 0xffffffffu;
+    return (uint32_t)(o->inflight_kb > 0 ? o->inflight_kb : 64) * 1024u;
+}
+
+// Bytes of one copy piece for options o: copy_piece_kb KiB, 64 KiB when 0.
+inline uint32_t amk_piece_bytes(const amk_options *o)
+{
+    return (uint32_t)(o->copy_piece_kb > 0 ? o->copy_piece_kb : 64) * 1024u;
+}
+
 // A non-owning amk_graph view of P's graph arrays.
 void amk_plan_view(const amk_plan *P, amk_graph *g);
 // Tensor maps of the Wdown of layers [l0, l0 + n) for a fused FFN (128 bytes

@@ -38,13 +38,17 @@ def test_tiny_greedy(variant, n_sms):
     worst, checked = greedy_teacher_forced(pair, prompt, 8)
     assert checked >= 6
     # the KV rows the kernel appended equal the oracle's (bf16 of nearly equal
-    # fp32/fp64 values: within one bf16 ulp)
+    # fp32/fp64 values: within one bf16 ulp).  The W8A16 GEMV takes its
+    # activations in int16 steps of max|x|/32767, so an element of k may move
+    # by up to sum_k |w_jk| * max|x| / 65534 (about 2e-4 on this model) before
+    # rounding: an absolute term of 1e-3 * max|K| covers it.
     for l in range(cfg.n_layers):
         k, v = pair.dec.kv(l)
         gk = k[:, :12].float().cpu().numpy()
         from oracle.brute import bf16_bits_to_f64
         rk = bf16_bits_to_f64(pair.orc.kv[l, 0, :, :12])
-        assert np.allclose(gk, rk, rtol=2 ** -7, atol=1e-6)
+        atol = 1e-3 * float(np.abs(rk).max()) if cfg.quant == "w8a16" else 1e-6
+        assert np.allclose(gk, rk, rtol=2 ** -7, atol=atol)
 
 
 def test_tiny_device_token_chaining():
