@@ -24,11 +24,12 @@ using amk::ErrorWord;
 using amk::KParams;
 using amk::TaskDesc;
 
-extern "C" cudaError_t amk_kernel_configure(int smem_bytes, int quant, int att_e, int generic);
+extern "C" cudaError_t amk_kernel_configure(int smem_bytes, int quant, int att_e, int generic,
+                                            int fused);
 extern "C" cudaError_t amk_pack_down(const void *wd, void *out, int h, int ffn, int esz,
                                      cudaStream_t stream);
 extern "C" cudaError_t amk_kernel_occupancy(int smem_bytes, int quant, int att_e, int generic,
-                                            int *blocks_per_sm);
+                                            int fused, int *blocks_per_sm);
 namespace amk {
 extern "C" cudaError_t amk_kernel_launch(const KParams *p, int n_ctas, int smem_bytes,
                                          cudaStream_t stream);
@@ -340,13 +341,13 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     }
     const amk_plan *P = H->plan;
     const int q8 = P->cfg.quant == AMK_QUANT_W8A16 ? 1 : 0;
-    cudaError_t e = amk_kernel_configure(P->smem_bytes, q8, P->att_e, P->generic);
+    cudaError_t e = amk_kernel_configure(P->smem_bytes, q8, P->att_e, P->generic, P->ffn_fused);
     if (e != cudaSuccess) {
         free_handle(H);
         return cuda_fail(e, "cudaFuncSetAttribute");
     }
     int per_sm = 0;
-    e = amk_kernel_occupancy(P->smem_bytes, q8, P->att_e, P->generic, &per_sm);
+    e = amk_kernel_occupancy(P->smem_bytes, q8, P->att_e, P->generic, P->ffn_fused, &per_sm);
     if (e != cudaSuccess || per_sm < 1) {
         free_handle(H);
         return amk_set_error(AMK_ERR_LAUNCH, "kernel does not fit one SM (smem %d B)",

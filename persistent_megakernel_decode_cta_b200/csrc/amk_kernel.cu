@@ -1877,30 +1877,29 @@ __device__ int resolve_token(const KParams &p)
     return t;
 }
 
-// Fused FFN, after its gate/up GEMV: the slice's SwiGLU activations
-// act[j] = silu(gate_j) up_j go to vec[0, R); then the slice's columns of
-// Wdown stream through the ring, 16-byte column group jb of chunk row lr at
-// (jb nrows + lr) * 16 of the stage.  Thread t owns the rows t + 256 k of
-// each chunk: it forms sum_j W[row][r0 + j] act[j] (times the row's int8
-// scale, loaded before the chunk's ring wait) and adds it into the layer's
-// fixed-point residual.  The 16-byte pieces a warp reads at once are
-// consecutive: free of bank conflicts.
-template <int ESZ>
-__device__ __forceinline__ bool ffn_down_part(const KParams &p, const SmemLayout &s,
+// Fused FFN, after its gate/up GEMV: the slice's R SwiGLU activations
+// act[j] = silu(gate_j) up_j are in vec[0, R) (int8 weights: also as int16
+// pairs at byte kQOff of vec, with one scale for the slice in scr[8]); then
+// the slice's columns of Wdown stream through the ring, 16-byte column group
+// jb of chunk row lr at (jb nrows + lr) * 16 of the stage.  Thread t owns the
+// rows t + 256 k of each chunk: it forms sum_j W[row][r0 + j] act[j] (times
+// the row's int8 scale, loaded before the chunk's ring wait) and adds it
+// into the layer's fixed-point residual.  The 16-byte pieces a warp reads at
+// once are consecutive: free of bank conflicts.
+constexpr int kQOff = 1024;  // byte offset of the int16 activation copy in vec
+
+// bf16 weights: the activations stay in shared memory (broadcast loads),
+// which measured faster than register copies for the narrow slices of the
+// models that fuse the level
+__device__ __forceinline__ bool ffn_down_bf16(const KParams &p, const SmemLayout &s,
                                               const Geom &g, const TaskDesc &d, uint32_t &kc,
                                               int ct, int lane)
 {
-    constexpr int E = 16 / ESZ;  // elements per box row
+    constexpr int E = 8;  // bf16 elements per box row
     const int ncb = g.ncb, h = p.hidden;
     long long *acc_out = p.xacc + (size_t)d.layer * h;
     for (int c2 = 0; c2 < g.nck2; ++c2) {
         const int r0w = c2 * g.rpc2, nrows = min(g.rpc2, h - r0w);
-        float scl[16];  // rows per thread per chunk <= stage / (16 B * 256)
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const int lr = ct + kConsumerThreads * k;
-            scl[k] = (d.s2 && lr < nrows) ? fp16_to_f(__ldg(d.s2 + r0w + lr)) : 1.f;
-        }
         if (!wait_full(p, s, kc))
             return false;
         const uint32_t st_a = s.ring_a + (uint32_t)(kc % p.ring_stages) * p.stage_bytes;
@@ -1917,9 +1916,9 @@ __device__ __forceinline__ bool ffn_down_part(const KParams &p, const SmemLayout
                         const uint2 t = lds64(s.vec_a + (uint32_t)(jb * E + 2 * u) * 4);
                         x[u] = pk2(__uint_as_float(t.x), __uint_as_float(t.y));
                     }
-                    acc = vdot2<ESZ, 16>(w, x, acc);
+                    acc = vdot2<2, 16>(w, x, acc);
                 }
-                red_add_fix(acc_out + r0w + lr, to_fix(sum2(acc) * scl[k]));
+                red_add_fix(acc_out + r0w + lr, to_fix(sum2(acc)));
             }
         }
         release_stage(p, s, kc, lane);
@@ -1928,26 +1927,123 @@ __device__ __forceinline__ bool ffn_down_part(const KParams &p, const SmemLayout
     return true;
 }
 
+// int8 weights: every thread holds the slice's activations as int16 pairs
+// (NCB >= ncb column groups of 16) and multiplies them with dp2a
+template <int NCB>
+__device__ __forceinline__ bool ffn_down_i8(const KParams &p, const SmemLayout &s, const Geom &g,
+                                            const TaskDesc &d, uint32_t &kc, int ct, int lane)
+{
+    const int ncb = g.ncb, h = p.hidden;
+    long long *acc_out = p.xacc + (size_t)d.layer * h;
+    uint32_t xq[NCB * 8];
+#pragma unroll
+    for (int jb = 0; jb < NCB; ++jb)
+#pragma unroll
+        for (int k = 0; k < 8; k += 4) {
+            uint4 u = make_uint4(0u, 0u, 0u, 0u);
+            if (jb < ncb)
+                u = lds128(s.vec_a + kQOff + (uint32_t)(jb * 8 + k) * 4);
+            xq[jb * 8 + k] = u.x;
+            xq[jb * 8 + k + 1] = u.y;
+            xq[jb * 8 + k + 2] = u.z;
+            xq[jb * 8 + k + 3] = u.w;
+        }
+    const float xs = s.scr[8];
+    for (int c2 = 0; c2 < g.nck2; ++c2) {
+        const int r0w = c2 * g.rpc2, nrows = min(g.rpc2, h - r0w);
+        float scl[16];  // rows per thread per chunk <= stage / (16 B * 256)
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int lr = ct + kConsumerThreads * k;
+            scl[k] = (d.s2 && lr < nrows) ? fp16_to_f(__ldg(d.s2 + r0w + lr)) : 1.f;
+        }
+        if (!wait_full(p, s, kc))
+            return false;
+        const uint32_t st_a = s.ring_a + (uint32_t)(kc % p.ring_stages) * p.stage_bytes;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int lr = ct + kConsumerThreads * k;
+            if (lr < nrows) {
+                int acc[2] = {0, 0};
+#pragma unroll
+                for (int jb = 0; jb < NCB; ++jb) {
+                    if (jb < ncb) {
+                        const uint4 w = lds128(st_a + (uint32_t)((jb * nrows + lr) * 16));
+                        const uint32_t A[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            acc[0] = dp2a_lo(xq[jb * 8 + 2 * q], A[q], acc[0]);
+                            acc[1] = dp2a_hi(xq[jb * 8 + 2 * q + 1], A[q], acc[1]);
+                        }
+                    }
+                }
+                const float sum = (float)(acc[0] + acc[1]) * xs;
+                red_add_fix(acc_out + r0w + lr, to_fix(sum * scl[k]));
+            }
+        }
+        release_stage(p, s, kc, lane);
+        ++kc;
+    }
+    return true;
+}
+
+// The slice's activations into vec[0, R); for int8 weights also as int16
+// pairs at vec + kQOff with their step in scr[8] (one scale for the slice:
+// the largest |act| over 32767), then the dispatch on the column groups.
 template <int Q8, int GENERIC>
 __device__ __forceinline__ bool ffn_down(const KParams &p, const SmemLayout &s, const Geom &g,
                                          const TaskDesc &d, uint32_t &kc, int ct, int lane,
                                          float sc0, float sc1)
 {
+    float a = 0.f;
     if (ct < g.R) {
         const float gt = row_total(s, g, ct) * sc0;
         const float up = row_total(s, g, g.R + ct) * sc1;
-        s.vec[ct] = gt / (1.f + __expf(-gt)) * up;
+        a = gt / (1.f + __expf(-gt)) * up;
+        s.vec[ct] = a;
+    }
+    const bool q8 = GENERIC ? g.esz == 1 : Q8 != 0;
+    if (q8) {
+        float m = fabsf(a);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if ((ct & 31) == 0)
+            s.scr[ct >> 5] = m;
     }
     consumer_bar();
-    if constexpr (GENERIC)
-        return g.esz == 1 ? ffn_down_part<1>(p, s, g, d, kc, ct, lane)
-                          : ffn_down_part<2>(p, s, g, d, kc, ct, lane);
-    else
-        return ffn_down_part<Q8 ? 1 : 2>(p, s, g, d, kc, ct, lane);
+    if (q8) {
+        float m = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w)
+            m = fmaxf(m, s.scr[w]);
+        const float inv = m > 0.f ? 32767.f / m : 0.f;
+        if (ct < g.R) {
+            const int q = max(-32767, min(32767, __float2int_rn(a * inv)));
+            reinterpret_cast<short *>(reinterpret_cast<uint8_t *>(s.vec) + kQOff)[ct] = (short)q;
+        }
+        if (ct == 0)
+            s.scr[8] = m * (1.f / 32767.f);
+        consumer_bar();
+    }
+    const int ncb = g.ncb;
+    if (g.esz == 1) {
+        if constexpr (GENERIC || Q8) {
+            if (ncb <= 2)
+                return ffn_down_i8<2>(p, s, g, d, kc, ct, lane);
+            if (ncb <= 4)
+                return ffn_down_i8<4>(p, s, g, d, kc, ct, lane);
+            return ffn_down_i8<8>(p, s, g, d, kc, ct, lane);
+        }
+    } else {
+        if constexpr (GENERIC || !Q8)
+            return ffn_down_bf16(p, s, g, d, kc, ct, lane);
+    }
+    return false;
 }
 
 // ---------------------------------------------------------- consumer loop
-template <int Q8, int ATT_E, int GENERIC>
+template <int Q8, int ATT_E, int GENERIC, int FUSED>
 __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout &s, int qb,
                                               int qe, int ct)
 {
@@ -2101,7 +2197,8 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
                             p.xacc[(size_t)l * p.hidden + d.r0 + ct] = to_fix(v);
                     }
                 } else if (d.kind == TK_FFN) {
-                    ok = ffn_down<Q8, GENERIC>(p, s, g, d, kc, ct, lane, sc0, sc1);
+                    if constexpr (FUSED || GENERIC)
+                        ok = ffn_down<Q8, GENERIC>(p, s, g, d, kc, ct, lane, sc0, sc1);
                 } else if (d.kind == TK_GATEUP) {
                     for (int t = ct; t < g.R; t += kConsumerThreads) {
                         const float gt = row_total(s, g, t) * sc0;
@@ -2174,7 +2271,7 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
 // ------------------------------------------------------------------- kernel
 // One fast instance per (weight format, attention lane width), holding only
 // the paths its models use, plus one generic instance for the rest.
-template <int Q8, int ATT_E, int GENERIC>
+template <int Q8, int ATT_E, int GENERIC, int FUSED>
 __global__ void __launch_bounds__(kThreads, 1) amk_decode_kernel(const __grid_constant__ KParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -2204,7 +2301,7 @@ __global__ void __launch_bounds__(kThreads, 1) amk_decode_kernel(const __grid_co
         return;
     }
     setmaxnreg_inc<kConsumerRegs>();
-    consumer_loop<Q8, ATT_E, GENERIC>(p, s, qb, qe, tid - kProducerThreads);
+    consumer_loop<Q8, ATT_E, GENERIC, FUSED>(p, s, qb, qe, tid - kProducerThreads);
     // On abort the producer notices the flag, drains its copies and returns.
 }
 
@@ -2232,34 +2329,36 @@ extern "C" int amk_kernel_smem_bytes(int ring_stages, int stage_bytes, int vec_f
 }
 
 namespace {
-const void *kernel_for(int quant, int att_e, int generic)
+const void *kernel_for(int quant, int att_e, int generic, int fused)
 {
     if (generic)
-        return reinterpret_cast<const void *>(amk_decode_kernel<0, 0, 1>);
-#define AMK_K(Q, E) reinterpret_cast<const void *>(amk_decode_kernel<Q, E, 0>)
-    static const void *const table[2][5] = {
-        {AMK_K(0, 1), AMK_K(0, 2), AMK_K(0, 4), AMK_K(0, 8), AMK_K(0, 16)},
-        {AMK_K(1, 1), AMK_K(1, 2), AMK_K(1, 4), AMK_K(1, 8), AMK_K(1, 16)}};
+        return reinterpret_cast<const void *>(amk_decode_kernel<0, 0, 1, 1>);
+#define AMK_K(F, Q, E) reinterpret_cast<const void *>(amk_decode_kernel<Q, E, 0, F>)
+    static const void *const table[2][2][5] = {
+        {{AMK_K(0, 0, 1), AMK_K(0, 0, 2), AMK_K(0, 0, 4), AMK_K(0, 0, 8), AMK_K(0, 0, 16)},
+         {AMK_K(0, 1, 1), AMK_K(0, 1, 2), AMK_K(0, 1, 4), AMK_K(0, 1, 8), AMK_K(0, 1, 16)}},
+        {{AMK_K(1, 0, 1), AMK_K(1, 0, 2), AMK_K(1, 0, 4), AMK_K(1, 0, 8), AMK_K(1, 0, 16)},
+         {AMK_K(1, 1, 1), AMK_K(1, 1, 2), AMK_K(1, 1, 4), AMK_K(1, 1, 8), AMK_K(1, 1, 16)}}};
 #undef AMK_K
     int e = 0;
     while (e < 4 && (1 << e) < att_e)
         ++e;
-    return table[quant ? 1 : 0][e];
+    return table[fused ? 1 : 0][quant ? 1 : 0][e];
 }
 }  // namespace
 
-extern "C" cudaError_t amk_kernel_configure(int smem_bytes, int quant, int att_e, int generic)
+extern "C" cudaError_t amk_kernel_configure(int smem_bytes, int quant, int att_e, int generic,
+                                            int fused)
 {
-    return cudaFuncSetAttribute(kernel_for(quant, att_e, generic),
+    return cudaFuncSetAttribute(kernel_for(quant, att_e, generic, fused),
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
 }
 
 extern "C" cudaError_t amk_kernel_occupancy(int smem_bytes, int quant, int att_e, int generic,
-                                            int *blocks_per_sm)
+                                            int fused, int *blocks_per_sm)
 {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm,
-                                                         kernel_for(quant, att_e, generic),
-                                                         kThreads, smem_bytes);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        blocks_per_sm, kernel_for(quant, att_e, generic, fused), kThreads, smem_bytes);
 }
 
 extern "C" cudaError_t amk_pack_down(const void *wd, void *out, int h, int ffn, int esz,
@@ -2276,7 +2375,8 @@ extern "C" cudaError_t amk_kernel_launch(const KParams *p, int n_ctas, int smem_
                                          cudaStream_t stream)
 {
     void *args[] = {const_cast<KParams *>(p)};
-    return cudaLaunchCooperativeKernel(kernel_for(p->quant, p->att_e, p->generic), dim3(n_ctas),
+    return cudaLaunchCooperativeKernel(kernel_for(p->quant, p->att_e, p->generic, p->ffn_fused),
+                                       dim3(n_ctas),
                                        dim3(kThreads), args, (size_t)smem_bytes, stream);
 }
 

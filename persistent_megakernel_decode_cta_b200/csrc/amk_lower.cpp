@@ -168,8 +168,10 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     // loads), a fused FFN slice's activations, or the attention tile's
     // scratch; DOWN tiles read their activations from L2 directly
     auto padded = [](int n) { return n + n / 32 * 4 + 4; };
+    // (and, for a fused FFN slice of int8 weights, its activations as int16
+    // pairs at byte 1024: at least 320 floats)
     int vec = std::max({padded(h), padded(nh * hd),
-                        G * hd + 2 * hd + amk::kConsumerWarps * G * (hd + 2)});
+                        G * hd + 2 * hd + amk::kConsumerWarps * G * (hd + 2), 320});
     vec = (vec + 3) & ~3;
     int stages = opt.ring_stages;
     while (stages > 2 && amk_kernel_smem_bytes(stages, opt.stage_bytes, vec) > kMaxSmem)

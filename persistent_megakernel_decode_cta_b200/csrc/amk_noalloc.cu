@@ -21,7 +21,8 @@
 #include "amk_plan.h"
 
 extern "C" int amk_kernel_smem_bytes(int ring_stages, int stage_bytes, int vec_floats);
-extern "C" cudaError_t amk_kernel_configure(int smem_bytes, int quant, int att_e, int generic);
+extern "C" cudaError_t amk_kernel_configure(int smem_bytes, int quant, int att_e, int generic,
+                                            int fused);
 namespace amk {
 extern "C" cudaError_t amk_kernel_launch(const KParams *p, int n_ctas, int smem_bytes,
                                          cudaStream_t stream);
@@ -245,7 +246,7 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     k.lookahead = (uint32_t)(P.opt.l2_prefetch_kb > 0 ? P.opt.l2_prefetch_kb : 0) * 1024u;
     k.inflight = amk_inflight_bytes(&P.opt);
     k.piece = amk_piece_bytes(&P.opt);
-    e = amk_kernel_configure(P.smem_bytes, q8 ? 1 : 0, P.att_e, P.generic);
+    e = amk_kernel_configure(P.smem_bytes, q8 ? 1 : 0, P.att_e, P.generic, P.ffn_fused);
     if (e != cudaSuccess)
         return fail_cuda(e, "cudaFuncSetAttribute");
     e = amk::amk_kernel_launch(&k, P.n_sms, P.smem_bytes, st);
