@@ -115,7 +115,7 @@ typedef struct {
                                  Wdown columns in one task, the slices' down projections
                                  summed into the residual in 64-bit fixed point (amk_create
                                  keeps a packed copy of every Wdown for it).  1 (default):
-                                 when the shape allows and hidden * element size <= 2 KB;
+                                 when the shape allows and hidden * element size <= 1.5 KB;
                                  2: whenever the shape allows; -1: separate gate/up and
                                  down levels */
     int32_t pos0_plan;        /* 1 (default): steps at position 0 run a second, validated

@@ -214,16 +214,16 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     const int64_t ffn_fit = box_rows ? (int64_t)opt.stage_bytes /
                                            ((int64_t)ffn_w * esz * box_rows) * box_rows
                                      : 0;
-    // default (ffn_fused = 1): fuse when a residual row is at most 2 KB.  The
+    // default (ffn_fused = 1): fuse when a residual row is at most 1.5 KB.  The
     // fused level adds every slice's partial down projection into the same
     // hidden-sized accumulator with 64-bit atomics, whose contention grows with
-    // the width; measured on B200 it gains 23% (SmolLM2 shape, 1152 B) and 5%
-    // (Llama-1B W8A16, 2 KB) but loses 3% (TinyLlama, 4 KB) and 8% (Llama-7B,
-    // 8 KB).  ffn_fused = 2 fuses whenever the shape allows.
+    // the width; measured on B200 it gains 3% on the SmolLM2 shape (1152 B) but
+    // loses 2% on Llama-1B W8A16 (2 KB), 4% on Llama-7B and 10% on TinyLlama.
+    // ffn_fused = 2 fuses whenever the shape allows.
     const bool shape_ok = F % ffn_gran == 0 && box_rows > 0 && ((int64_t)F * esz) % 16 == 0 &&
                           (ffn_fit >= h || ffn_fit >= 256);
     const bool fused = shape_ok && (opt.ffn_fused >= 2 ||
-                                    (opt.ffn_fused == 1 && (int64_t)h * esz <= 2048));
+                                    (opt.ffn_fused == 1 && (int64_t)h * esz <= 1536));
     P->ffn_fused = fused ? 1 : 0;
     P->ffn_box_rows = fused ? box_rows : 0;
 

@@ -113,7 +113,7 @@ def test_full_size_single_steps(name, ctxs):
     ("tinyllama", 256, 2),     # the fused FFN level where the default keeps it split
     ("llama7b_w8", 0, 2),
     ("smol135", 128, -1),      # split levels where the default fuses
-    ("llama1b_w8", 512, -1),
+    ("llama1b_w8", 512, 2),    # the fused int8 level (dp2a column loop), split by default
 ])
 def test_ffn_level_variants(name, ctx, fused):
     """Both FFN schedules (one fused level with fixed-point accumulation of
