@@ -571,7 +571,7 @@ int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev,
         H->epoch0 += 1;
     {  // non-empty attention chunks of this step: each arrives once unless alone
         const int C = H->plan->opt.attn_splits, n = pos + 1;
-        const int chunk = (n + C - 1) / C, nne = (n + chunk - 1) / chunk;
+        const int chunk = amk::attn_chunk_len(n, C), nne = (n + chunk - 1) / chunk;
         if (nne > 1)
             H->arrive_base += (uint32_t)nne;
     }

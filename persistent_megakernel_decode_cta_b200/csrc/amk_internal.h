@@ -6,6 +6,8 @@
 
 #include <stdint.h>
 
+#include <cuda_runtime.h>
+
 #include "amk.h"
 
 #ifdef __cplusplus
@@ -34,6 +36,15 @@ constexpr int kConsumerRegs = 224;
 static_assert(kProducerThreads * kProducerRegs + kConsumerThreads * kConsumerRegs ==
                   kThreads * kLaunchRegs, "register split must equal the launch budget");
 constexpr int kMaxTaskRows = 256;   // output rows of one GEMV task (red buffer)
+// Positions of a split-K attention chunk: ceil(n / attn_splits) for n
+// positions, but at least kMinAttnChunk, so that short contexts use fewer,
+// longer chunks (the kernel and the host's arrival count both use this).
+constexpr int kMinAttnChunk = 32;
+inline __host__ __device__ int attn_chunk_len(int n, int splits)
+{
+    const int c = (n + splits - 1) / splits;
+    return c > kMinAttnChunk ? c : kMinAttnChunk;
+}
 constexpr int kMaxStages = 16;
 // A ring stage's copy goes out in up to kPieces pieces of about KParams::piece bytes,
 // each completing on its own mbarrier, so that the producer can keep a

@@ -429,7 +429,7 @@ __device__ __forceinline__ Geom task_geom(const KParams &p, const TaskDesc &d)
     if (d.kind == TK_ATTN) {
         const int c = d.r1, hd = p.head_dim;
         const int n = p.pos + 1;
-        const int chunk = (n + p.attn_splits - 1) / p.attn_splits;
+        const int chunk = attn_chunk_len(n, p.attn_splits);
         g.j0 = c * chunk;
         g.j1 = min(g.j0 + chunk, n);
         if (g.j1 < g.j0)
@@ -1770,7 +1770,7 @@ __device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
         return false;
     const int l = d.layer, gi = d.r0, C = p.attn_splits;
     const int n = p.pos + 1;
-    const int chunk = (n + C - 1) / C;
+    const int chunk = attn_chunk_len(n, C);
     const int nne = (n + chunk - 1) / chunk;  // non-empty chunks: 0 .. nne-1
     if (nne == 1 || g.j1 <= g.j0)
         return true;  // written directly, or empty
