@@ -101,8 +101,10 @@ typedef struct {
  * pipelining depth; README "two autoresearch loops").  Zero fields take the
  * defaults from amk_default_options. */
 typedef struct {
-    int32_t ring_stages;      /* shared-memory weight ring depth (>= 2) */
-    int32_t stage_bytes;      /* bytes per ring stage (multiple of 1024) */
+    int32_t ring_stages;      /* shared-memory weight ring depth (>= 2); 0 = auto:
+                                 192 KiB / stage_bytes */
+    int32_t stage_bytes;      /* bytes per ring stage (multiple of 1024); 0 = auto:
+                                 48 KiB for W8A16 weights, 64 KiB for bf16 */
     int32_t attn_splits;      /* split-K chunks per KV head; 0 = auto */
     int32_t tasks_per_sm;     /* GEMV row tiles per SM per level; 0 = auto */
     int32_t n_sms;            /* persistent CTAs; 0 = all SMs of the device */

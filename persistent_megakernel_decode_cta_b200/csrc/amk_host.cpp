@@ -75,8 +75,8 @@ extern "C" int amk_default_options(amk_options *o)
     if (!o)
         return amk_set_error(AMK_ERR_INVALID_ARG, "amk_default_options: NULL");
     memset(o, 0, sizeof *o);
-    o->ring_stages = 3;
-    o->stage_bytes = 65536;
+    o->ring_stages = 0;  // ring shape resolved by the lowering from the weight format
+    o->stage_bytes = 0;
     o->attn_splits = 0;
     o->tasks_per_sm = 1;
     o->n_sms = 0;

@@ -34,6 +34,8 @@ def test_tiny_greedy(variant, n_sms):
         cfg = cfg.with_(quant="w8a16", name="tiny_w8")
     opts = amk.default_options(n_sms=n_sms) if n_sms else None
     pair = Pair(cfg, options=opts)
+    st = pair.dec.stats()  # the ring shape resolved from the weight format
+    assert (st.ring_stages, st.stage_bytes) == ((4, 49152) if cfg.quant == "w8a16" else (3, 65536))
     prompt = si.make_prompt(cfg, 4)
     worst, checked = greedy_teacher_forced(pair, prompt, 8)
     assert checked >= 6
