@@ -99,12 +99,13 @@ def _ptr(a: np.ndarray, typ=None):
 
 
 def to_numpy_bits(t) -> np.ndarray:
-    """A torch bf16/fp16 tensor -> its uint16 bits; int8 -> int8 (CPU)."""
+    """A torch bf16/fp16 tensor -> its uint16 bits; int8 -> int8 and packed
+    int4 (uint8) -> uint8 (CPU)."""
     import torch
     t = t.detach().to("cpu").contiguous()
     if t.dtype in (torch.bfloat16, torch.float16):
         return t.view(torch.int16).numpy().view(np.uint16)
-    if t.dtype == torch.int8:
+    if t.dtype in (torch.int8, torch.uint8):
         return t.numpy()
     raise TypeError(f"unexpected weight dtype {t.dtype}")
 
@@ -133,15 +134,20 @@ def rmsnorm(x, g_bits, eps: float, lib=None) -> np.ndarray:
 
 
 def matvec(W, x, scale_bits=None, lib=None) -> np.ndarray:
-    """W: uint16 bf16 bits [rows, cols], or int8 [rows, cols] with fp16 bits
-    ``scale_bits`` [rows]."""
+    """W: uint16 bf16 bits [rows, cols], int8 [rows, cols] with fp16 bits
+    ``scale_bits`` [rows], or packed int4 uint8 [rows, cols / 2] with fp16
+    bits ``scale_bits`` [rows, ceil(cols / 128)] (cols = len(x))."""
     W = np.ascontiguousarray(W)
     x = _f64(x)
     rows, cols = W.shape
     y = np.zeros(rows, dtype=np.float64)
-    quant = 1 if W.dtype == np.int8 else 0
-    if quant == 0 and W.dtype != np.uint16:
+    quant = {np.dtype(np.uint16): 0, np.dtype(np.int8): 1, np.dtype(np.uint8): 2}.get(W.dtype)
+    if quant is None:
         raise TypeError("bf16 weights are passed as uint16 bits")
+    if quant == 2:
+        cols = len(x)
+        if W.shape[1] * 2 != cols:
+            raise ValueError("packed int4 rows hold len(x) / 2 bytes")
     s = None
     if quant:
         s = np.ascontiguousarray(scale_bits, dtype=np.uint16)
@@ -201,7 +207,7 @@ class OracleModel:
         c.max_ctx = cfg.max_ctx
         c.rms_eps, c.rope_theta = cfg.rms_eps, cfg.rope_theta
         c.tied = 1 if cfg.tied else 0
-        c.quant = 1 if cfg.quant == "w8a16" else 0
+        c.quant = {"bf16": 0, "w8a16": 1, "w4a16": 2}[cfg.quant]
         self._c = c
         self._keep = []  # keeps numpy buffers alive for the C side
 

@@ -16,12 +16,18 @@
  *   dequant).
  *   Same README, results section: W8A16 int8 weights (per output channel),
  *   correctness gated on an exact argmax.
+ *   gist.science technical summary of the paper, "Belangrijkste Bijdragen"
+ *   (the quantised-megakernels item): int8 and int4 weight-only kernels from
+ *   the same IR path.  The pages give no int4 format; the one
+ *   read here is symmetric 4-bit codes with one fp16 scale per group of 128
+ *   consecutive inputs of a row (the last group shorter when the row length
+ *   is not a multiple of 128), two codes per byte, input 2i in the low nibble.
  * Where the pages leave a step open, the HuggingFace Llama definition is used
  * (the pages reproduce HF greedy generate token for token): RoPE is HF
  * rotate_half, GQA maps query head h to KV head h / (n_heads / n_kv_heads),
  * the softmax is the max-subtracted form over positions 0..pos inclusive.
  *
- * Precision: weights arrive as the exact bf16 (or int8 + fp16 scale) bytes the
+ * Precision: weights arrive as the exact bf16 (or int8/int4 + fp16 scale) bytes the
  * GPU consumes and are widened to double; everything else is double.  The KV
  * cache is stored as bf16 (round to nearest even), which is how the workload
  * defines the cache ("bf16 activations/KV"); every K and V row is rounded
@@ -43,14 +49,15 @@ typedef struct {
     int32_t hidden, n_layers, n_heads, n_kv_heads, head_dim, ffn, vocab, max_ctx;
     double rms_eps, rope_theta;
     int32_t tied;  /* 1: the LM head is the embedding table */
-    int32_t quant; /* 0: bf16 linear weights; 1: int8 + fp16 row scales */
+    int32_t quant; /* 0: bf16 linear weights; 1: int8 + fp16 row scales;
+                      2: packed int4 + fp16 scales per 128-input group */
 } orc_config;
 
 typedef struct {
     const uint16_t *embed;      /* bf16 [vocab][hidden] */
     const uint16_t *final_norm; /* bf16 [hidden] */
-    const void *lm_head;        /* bf16 or int8 [vocab][hidden]; unused if tied */
-    const uint16_t *lm_head_scale; /* fp16 [vocab] (int8, untied) */
+    const void *lm_head;        /* bf16, int8 or packed int4 [vocab][hidden]; unused if tied */
+    const uint16_t *lm_head_scale; /* fp16 [vocab] (int8) or [vocab][groups] (int4), untied */
     const uint16_t *const *attn_norm; /* [n_layers] -> bf16 [hidden] */
     const uint16_t *const *ffn_norm;
     const void *const *wq, *const *wk, *const *wv, *const *wo;
@@ -122,8 +129,20 @@ void orc_rmsnorm(const double *x, const uint16_t *g, int32_t n, double eps,
         out[i] = orc_bf16_to_double(g[i]) * (x[i] * inv);
 }
 
+#define ORC_INT4_GROUP 128
+
+/* The signed value of input k's 4-bit code in a packed int4 row: byte k / 2,
+ * low nibble for even k, high nibble for odd k, two's complement. */
+static int orc_int4_code(const uint8_t *row, int32_t k)
+{
+    int nib = (row[k >> 1] >> ((k & 1) * 4)) & 0xF;
+    return nib >= 8 ? nib - 16 : nib;
+}
+
 /* y = W x for row-major W [rows][cols].  quant 0: W is bf16.  quant 1: W is
- * int8 and row j's weights are scale_j * q_jk, so y_j = scale_j * sum_k q_jk x_k. */
+ * int8 and row j's weights are scale_j * q_jk, so y_j = scale_j * sum_k q_jk x_k.
+ * quant 2: W is packed int4 (cols / 2 bytes per row) and weight (j, k) is
+ * scale[j][k / 128] * q_jk, the scales fp16 [rows][ceil(cols / 128)]. */
 void orc_matvec(const void *W, const uint16_t *scale, int32_t quant,
                 int32_t rows, int32_t cols, const double *x, double *y)
 {
@@ -135,11 +154,18 @@ void orc_matvec(const void *W, const uint16_t *scale, int32_t quant,
             for (int32_t k = 0; k < cols; ++k)
                 acc += orc_bf16_to_double(w[k]) * x[k];
             y[j] = acc;
-        } else {
+        } else if (quant == 1) {
             const int8_t *w = (const int8_t *)W + (size_t)j * cols;
             for (int32_t k = 0; k < cols; ++k)
                 acc += (double)w[k] * x[k];
             y[j] = orc_fp16_to_double(scale[j]) * acc;
+        } else {
+            const uint8_t *w = (const uint8_t *)W + (size_t)j * (cols / 2);
+            const int32_t ng = (cols + ORC_INT4_GROUP - 1) / ORC_INT4_GROUP;
+            const uint16_t *sj = scale + (size_t)j * ng;
+            for (int32_t k = 0; k < cols; ++k)
+                acc += orc_fp16_to_double(sj[k / ORC_INT4_GROUP]) * orc_int4_code(w, k) * x[k];
+            y[j] = acc;
         }
     }
 }
@@ -229,8 +255,10 @@ int32_t orc_decode_step(const orc_config *c, const orc_weights *w,
     const int32_t h = c->hidden, nh = c->n_heads, nkv = c->n_kv_heads;
     const int32_t hd = c->head_dim, F = c->ffn;
     if (token < 0 || token >= c->vocab || pos < 0 || pos >= c->max_ctx ||
-        nkv <= 0 || nh % nkv != 0 || (hd & 1))
+        nkv <= 0 || nh % nkv != 0 || (hd & 1) || c->quant < 0 || c->quant > 2)
         return -1;
+    if (c->quant == 2 && ((h & 1) || ((nh * hd) & 1) || (F & 1)))
+        return -1; /* packed int4 rows hold whole bytes */
     const int32_t group = nh / nkv;
     const int32_t qr = nh * hd, kr = nkv * hd;
 

@@ -36,15 +36,24 @@ def round_to_bf16(v) -> np.ndarray:
 
 
 def dequant(weights: Dict[str, object], key: str, layer=None) -> np.ndarray:
-    """A weight matrix as float64: bf16 bits widened, or int8 times its fp16
-    row scale."""
+    """A weight matrix as float64: bf16 bits widened, int8 times its fp16
+    row scale, or packed int4 (uint8, two 4-bit two's-complement codes per
+    byte, the even input in the low nibble) times the fp16 scale of its group
+    of 128 inputs."""
     from . import to_numpy_bits
     t = weights[key] if layer is None else weights[key][layer]
     a = to_numpy_bits(t)
-    if a.dtype == np.int8:
+    if a.dtype in (np.int8, np.uint8):
         skey = "lm_head_scale" if key == "lm_head" else "s" + key[1:]
         s = weights[skey] if layer is None else weights[skey][layer]
-        return a.astype(np.float64) * fp16_bits_to_f64(to_numpy_bits(s))[:, None]
+        sc = fp16_bits_to_f64(to_numpy_bits(s))
+        if a.dtype == np.int8:
+            return a.astype(np.float64) * sc[:, None]
+        nib = np.stack([a & 0xF, a >> 4], axis=-1).reshape(a.shape[0], -1).astype(np.int64)
+        codes = np.where(nib >= 8, nib - 16, nib)
+        cols = codes.shape[1]
+        per_input = np.repeat(sc, 128, axis=1)[:, :cols]
+        return codes.astype(np.float64) * per_input
     return bf16_bits_to_f64(a)
 
 

@@ -16,6 +16,13 @@ weights are needed or used):
   per output row, ``s = fp16(max|w_row| / 127)`` and
   ``q = clamp(round_half_even(w / s), -127, 127)`` (a row of zeros gets s = 1,
   q = 0).  The decode step consumes q and s; neither side re-quantises;
+* W4A16 weights: from the same masters, one symmetric scale per group of
+  ``INT4_GROUP`` consecutive inputs of a row (the last group of a row is
+  shorter when the row length is not a multiple of it),
+  ``s = fp16(max|w_group| / 7)`` and ``q = clamp(round_half_even(w / s), -7, 7)``
+  (an all-zero group gets s = 1, q = 0).  Codes are packed two per byte in
+  4-bit two's complement, input 2i in the low nibble of byte i and input
+  2i + 1 in the high nibble; scales are fp16 [rows][ceil(cols / INT4_GROUP)];
 * prompt token ids: uniform in [0, vocab);
 * synthetic KV-cache fill for long contexts: N(0, 1) rounded to bf16.
 
@@ -59,7 +66,7 @@ class ModelConfig:
     rms_eps: float = 1e-5
     rope_theta: float = 1e4
     tied: bool = False
-    quant: str = "bf16"  # "bf16" or "w8a16"
+    quant: str = "bf16"  # "bf16", "w8a16" or "w4a16"
 
     @property
     def q_rows(self) -> int:
@@ -133,31 +140,60 @@ def _int8_rows(shape, device, seed, name):
     return q.to(torch.int8), s
 
 
+INT4_GROUP = 128  # inputs per W4A16 scale
+
+
+def _int4_groups(shape, device, seed, name):
+    """Per-group symmetric int4 weights from N(0, 0.02) fp32 masters, packed
+    two codes per byte (even input in the low nibble)."""
+    rows, cols = shape
+    if cols % 2:
+        raise ValueError("W4A16 rows need an even number of inputs")
+    w = _normal(shape, 0.02, device, seed, name)
+    ng = (cols + INT4_GROUP - 1) // INT4_GROUP
+    pad = ng * INT4_GROUP - cols
+    wp = torch.nn.functional.pad(w, (0, pad)).view(rows, ng, INT4_GROUP)
+    amax = wp.abs().amax(dim=2)
+    s = (amax / 7.0).to(torch.float16)
+    s = torch.where(amax == 0, torch.ones_like(s), s)
+    q = torch.round(wp / s.to(torch.float32)[:, :, None]).clamp_(-7, 7)
+    q = torch.where((amax == 0)[:, :, None], torch.zeros_like(q), q)
+    q = q.view(rows, ng * INT4_GROUP)[:, :cols].to(torch.int16)
+    del w, wp
+    nib = q & 0xF  # 4-bit two's complement
+    packed = (nib[:, 0::2] | (nib[:, 1::2] << 4)).to(torch.uint8)
+    return packed, s
+
+
 def make_model(cfg, seed: int = 0, device="cpu") -> Dict[str, object]:
     """Random-init weights of ``cfg``'s shape.
 
     Returns a dict with tensors on ``device``:
       embed [vocab, hidden] bf16; final_norm [hidden] bf16;
-      lm_head [vocab, hidden] bf16 or int8 (None when tied);
-      lm_head_scale [vocab] fp16 (W8A16 and untied only, else None);
+      lm_head [vocab, hidden] bf16 or int8, or packed int4 [vocab, hidden/2]
+      (None when tied);
+      lm_head_scale [vocab] fp16 (W8A16), [vocab, groups] fp16 (W4A16), or
+      None (bf16 or tied);
       per-layer lists attn_norm, ffn_norm [hidden] bf16;
       wq [nh*hd, hidden], wk/wv [nkv*hd, hidden], wo [hidden, nh*hd],
-      wgate/wup [ffn, hidden], wdown [hidden, ffn] (bf16, or int8), and for
-      W8A16 the fp16 row scales sq, sk, sv, so, sgate, sup, sdown.
+      wgate/wup [ffn, hidden], wdown [hidden, ffn] (bf16, int8, or packed
+      int4 uint8 [out, in/2]), and for W8A16 the fp16 row scales sq, sk, sv,
+      so, sgate, sup, sdown ([out]; W4A16: group scales [out, groups]).
     All weights are row-major [out, in].
     """
     cfg = get_config(cfg)
     h, L = cfg.hidden, cfg.n_layers
-    q8 = cfg.quant == "w8a16"
+    if cfg.quant not in ("bf16", "w8a16", "w4a16"):
+        raise ValueError(f"unknown quant {cfg.quant!r}")
+    qfn = {"w8a16": _int8_rows, "w4a16": _int4_groups}.get(cfg.quant)
     m: Dict[str, object] = {}
     m["embed"] = _bf16_normal((cfg.vocab, h), 0.02, device, seed, "embed")
     m["final_norm"] = _gain(h, device, seed, "final_norm")
     m["lm_head"] = None
     m["lm_head_scale"] = None
     if not cfg.tied:
-        if q8:
-            m["lm_head"], m["lm_head_scale"] = _int8_rows(
-                (cfg.vocab, h), device, seed, "lm_head")
+        if qfn:
+            m["lm_head"], m["lm_head_scale"] = qfn((cfg.vocab, h), device, seed, "lm_head")
         else:
             m["lm_head"] = _bf16_normal((cfg.vocab, h), 0.02, device, seed,
                                         "lm_head")
@@ -173,14 +209,14 @@ def make_model(cfg, seed: int = 0, device="cpu") -> Dict[str, object]:
     for key in ("attn_norm", "ffn_norm", *shapes):
         m[key] = []
     for key in shapes:
-        m["s" + key[1:]] = [] if q8 else None
+        m["s" + key[1:]] = [] if qfn else None
     for layer in range(L):
         m["attn_norm"].append(_gain(h, device, seed, f"l{layer}.attn_norm"))
         m["ffn_norm"].append(_gain(h, device, seed, f"l{layer}.ffn_norm"))
         for key, shp in shapes.items():
             name = f"l{layer}.{key}"
-            if q8:
-                q, s = _int8_rows(shp, device, seed, name)
+            if qfn:
+                q, s = qfn(shp, device, seed, name)
                 m[key].append(q)
                 m["s" + key[1:]].append(s)
             else:
@@ -210,14 +246,20 @@ def model_bytes(cfg) -> Dict[str, int]:
     """Byte counts of the stored weights (for roofline bookkeeping)."""
     cfg = get_config(cfg)
     h, L = cfg.hidden, cfg.n_layers
-    wb = 1 if cfg.quant == "w8a16" else 2
-    per_layer_params = (cfg.q_rows * h + 2 * cfg.kv_rows * h + h * cfg.q_rows
-                        + 3 * cfg.ffn * h)
-    per_layer_rows = (cfg.q_rows + 2 * cfg.kv_rows + h + 2 * cfg.ffn + h)
-    linear = L * per_layer_params * wb
-    scales = L * per_layer_rows * 2 if wb == 1 else 0
-    head = 0 if cfg.tied else cfg.vocab * h * wb
-    head_scales = cfg.vocab * 2 if (wb == 1 and not cfg.tied) else 0
+    # (rows, inputs) of every linear weight of one layer
+    mats = [(cfg.q_rows, h), (cfg.kv_rows, h), (cfg.kv_rows, h), (h, cfg.q_rows),
+            (cfg.ffn, h), (cfg.ffn, h), (h, cfg.ffn)]
+
+    def wbytes(rows, cols):  # (weight bytes, scale bytes) of one matrix
+        if cfg.quant == "w8a16":
+            return rows * cols, rows * 2
+        if cfg.quant == "w4a16":
+            return rows * cols // 2, rows * ((cols + INT4_GROUP - 1) // INT4_GROUP) * 2
+        return rows * cols * 2, 0
+
+    linear = L * sum(wbytes(r, k)[0] for r, k in mats)
+    scales = L * sum(wbytes(r, k)[1] for r, k in mats)
+    head, head_scales = (0, 0) if cfg.tied else wbytes(cfg.vocab, h)
     norms = (2 * L + 1) * h * 2
     return {
         "linear": linear, "scales": scales + head_scales, "head": head,
@@ -228,7 +270,7 @@ def model_bytes(cfg) -> Dict[str, int]:
 
 def streamed_weight_bytes(cfg) -> int:
     """Weight bytes one decode step reads: every linear weight (and int8 row
-    scale) once, the LM head -- the whole embedding table when tied --, the
+    or int4 group scale) once, the LM head -- the whole embedding table when tied --, the
     norm gains and the one embedding row of the input token."""
     b = model_bytes(cfg)
     head = b["embed_table"] if get_config(cfg).tied else b["head"]

@@ -29,8 +29,19 @@ def test_int8_byte_ratio_matches_published():
     assert abs(ratio - float(g["ratio"])) <= float(g["abs_tolerance"]), ratio
 
 
+def test_int4_byte_ratio_matches_published():
+    """The W4A16 reading (symmetric int4, one fp16 scale per 128 inputs of a
+    row, tied head in bf16) against the pages' 2.42x weight-traffic cut; one
+    scale per row (2.44x) or per 64 inputs (2.38x) falls outside."""
+    g = _golden("int4_byte_ratio.txt")
+    cfg = si.get_config(g["model"])
+    ratio = (si.streamed_weight_bytes(cfg.with_(quant="bf16"))
+             / si.streamed_weight_bytes(cfg.with_(quant="w4a16")))
+    assert abs(ratio - float(g["ratio"])) <= float(g["abs_tolerance"]), ratio
+
+
 @pytest.mark.parametrize("tied", [False, True])
-@pytest.mark.parametrize("quant", ["bf16", "w8a16"])
+@pytest.mark.parametrize("quant", ["bf16", "w8a16", "w4a16"])
 def test_byte_accounting_matches_generated_tensors(tied, quant):
     """model_bytes / streamed_weight_bytes count exactly the tensors that
     make_model produces (so the byte ratio above is about real weights)."""

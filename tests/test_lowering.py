@@ -145,6 +145,7 @@ def test_balanced_tiles_on_148_sms():
     (dict(ffn=12290), "AMK_ERR_UNSUPPORTED"),            # down K above the register slice
     (dict(hidden=0), "AMK_ERR_INVALID_ARG"),
     (dict(ffn=171), "AMK_ERR_UNSUPPORTED"),              # odd bf16 K: row not 4-byte aligned
+    (dict(quant="w4a16"), "AMK_ERR_UNSUPPORTED"),        # int4: oracle only, no kernel
 ])
 def test_unsupported_shapes_rejected(edit, status):
     cfg = si.get_config("tiny").with_(**edit)

@@ -1,5 +1,5 @@
 """Pins the oracle's incremental decode (KV cache, positions, GQA mapping,
-tied head, W8A16 dequant) against the non-incremental full-sequence forward
+tied head, W8A16 and W4A16 dequant) against the non-incremental full-sequence forward
 in ``oracle.brute``.
 
 "RightNow-AI/AutoMegaKernel" README (bittide mirror), "What is built and
@@ -51,6 +51,11 @@ def test_tiny_tied_head():
 
 def test_tiny_w8a16():
     _check(si.get_config("tiny").with_(quant="w8a16", name="tiny_w8"))
+
+
+def test_tiny_w4a16():
+    # the down projection's 172 inputs end in a ragged group of 44
+    _check(si.get_config("tiny").with_(quant="w4a16", name="tiny_w4"))
 
 
 def test_gqa_group_sizes():

@@ -40,6 +40,13 @@ MUTANTS = [
     ("silu_is_sigmoid", [("return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));")]),
     ("swiglu_swapped", [("a[j] = orc_silu(gt[j]) * up[j];", "a[j] = orc_silu(up[j]) * gt[j];")]),
     ("int8_scale_dropped", [("y[j] = orc_fp16_to_double(scale[j]) * acc;", "y[j] = acc;")]),
+    ("int4_nibbles_swapped", [("int nib = (row[k >> 1] >> ((k & 1) * 4)) & 0xF;",
+                               "int nib = (row[k >> 1] >> ((~k & 1) * 4)) & 0xF;")]),
+    ("int4_unsigned_codes", [("return nib >= 8 ? nib - 16 : nib;", "return nib;")]),
+    ("int4_offset_binary", [("return nib >= 8 ? nib - 16 : nib;", "return nib - 8;")]),
+    ("int4_group_of_64", [("sj[k / ORC_INT4_GROUP]", "sj[k / 64]")]),
+    ("int4_row_stride_bytes", [("(const uint8_t *)W + (size_t)j * (cols / 2);",
+                                "(const uint8_t *)W + (size_t)j * cols;")]),
     ("matvec_transposed", [("acc += orc_bf16_to_double(w[k]) * x[k];",
                             "acc += orc_bf16_to_double(((const uint16_t *)W)[(size_t)k * rows + j]) * x[k];")]),
     ("embed_row_index", [("w->embed[(size_t)token * h + i]", "w->embed[(size_t)token + i]")]),
@@ -55,6 +62,7 @@ BATTERY = [getattr(tp, n) for n in dir(tp) if n.startswith("test_")] + [
     tb.test_tiny_full_sequence_12_positions,
     tb.test_tiny_tied_head,
     tb.test_tiny_w8a16,
+    tb.test_tiny_w4a16,
     tb.test_gqa_head_to_group_mapping_at_pos0,
 ]
 

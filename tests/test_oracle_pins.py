@@ -137,6 +137,39 @@ def test_matvec_int8_row_scales():
     assert y[1] == 2.0 * (127 - 254)
 
 
+def test_matvec_int4_nibble_order_and_sign():
+    """Packed int4 row, scale 1.0 (fp16 0x3C00): input 2i sits in the low
+    nibble of byte i, input 2i + 1 in the high nibble, 4-bit two's
+    complement.  Bytes 0x8F, 0x70, 0x21 hold the codes -1, -8, 0, 7, 1, 2,
+    read off one by one with one-hot inputs."""
+    W = np.array([[0x8F, 0x70, 0x21]], dtype=np.uint8)
+    s = np.array([[0x3C00]], dtype=np.uint16)
+    want = [-1, -8, 0, 7, 1, 2]
+    for k, v in enumerate(want):
+        e = np.zeros(6)
+        e[k] = 1.0
+        assert orc.matvec(W, e, scale_bits=s)[0] == v
+
+
+def test_matvec_int4_group_scales_ragged_closed_form():
+    """576 inputs = four groups of 128 and a last group of 64.  Every code 1
+    (byte 0x11) in row 0 and -1 (0xFF) in row 1, group g scaled by 2**g
+    (fp16 1, 2, 4, 8, 16), x all ones: y = +-(128 (1 + 2 + 4 + 8) + 64 * 16)
+    = +-2944.  A scale indexed per 64 inputs, or the last group taken as
+    full, gives another sum."""
+    W = np.empty((2, 288), dtype=np.uint8)
+    W[0] = 0x11
+    W[1] = 0xFF
+    s = np.array([[0x3C00, 0x4000, 0x4400, 0x4800, 0x4C00]] * 2, dtype=np.uint16)
+    y = orc.matvec(W, np.ones(576), scale_bits=s)
+    assert y[0] == 2944.0 and y[1] == -2944.0
+    # one input at a time: its group's scale times its code
+    for k in (0, 127, 128, 511, 512, 575):
+        e = np.zeros(576)
+        e[k] = 3.0
+        assert orc.matvec(W, e, scale_bits=s)[0] == 3.0 * 2 ** (k // 128)
+
+
 # ---- RoPE --------------------------------------------------------------------
 
 def test_rope_position_zero_is_identity():
