@@ -160,18 +160,30 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(rows)}
 
 
-def dist_setup(n_gpus: int):
+def dist_env(n_gpus: int):
+    """(world, rank, local rank) from the launcher's environment; the world
+    size must equal --gpus."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world != n_gpus:
         raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+def dist_setup(n_gpus: int, backend: str = "nccl"):
+    """One rank per GPU.  The process group carries only the barriers and the
+    max-over-ranks reductions of the timing (replicas share no data)."""
+    world, rank, local = dist_env(n_gpus)
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -187,9 +199,16 @@ def max_over_ranks(world, value: float) -> float:
     if world == 1:
         return value
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_us_per_token(elapsed_ms: float, steps: int, world: int) -> float:
+    """Whole-job time per token: `world` replicas each decode `steps` tokens
+    within the slowest rank's `elapsed_ms`."""
+    return elapsed_ms * 1e3 / (steps * world)
 
 
 def oracle_steps(cfg, weights, ctx, kv_fill, budget_s: float, max_steps: int):
@@ -217,7 +236,8 @@ def oracle_steps(cfg, weights, ctx, kv_fill, budget_s: float, max_steps: int):
 
 
 def run_reference(args):
-    world, rank, _ = dist_setup(args.gpus)
+    # rank 0 alone times the oracle; no process group is needed for that
+    world, rank, _ = dist_env(args.gpus)
     if rank != 0:
         return
     name = args.workload
@@ -354,7 +374,7 @@ def run_ours(args):
     nbytes = algorithmic_bytes(cfg, ctx)
     peak, peak_kind = measured_peak()
     achieved = nbytes / (kernel_ms * 1e-3) / 1e9
-    value = elapsed_ms * 1e3 / (K * world)
+    value = job_us_per_token(elapsed_ms, K, world)
     st = dec.stats()
     if rank == 0:
         line = {
@@ -372,7 +392,7 @@ def run_ours(args):
                          "kernel_us_per_launch": kernel_ms * 1e3},
             "achieved_gbs": achieved,
             "cpu_baseline": cpu_base,
-            "e2e": {"value": e2e_s * 1e6 / (K_e2e * world), "unit": UNIT,
+            "e2e": {"value": job_us_per_token(e2e_s * 1e3, K_e2e, world), "unit": UNIT,
                     "h2d_bytes_per_step": 4, "d2h_bytes_per_step": cfg.vocab * 4 + 8 + 32,
                     "steps": K_e2e},
             "gpu_launches": K,
