@@ -132,6 +132,30 @@ def test_ffn_level_variants(name, ctx, fused):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("name,ctx,stages,stage_bytes", [
+    ("llama1b_w8", 512, 3, 65536),   # the bf16 ring shape on int8 weights
+    ("tinyllama", 256, 4, 49152),    # the int8 ring shape on bf16 weights
+    ("smol135", 128, 6, 32768),      # small stages: more chunks per task
+    ("tinyllama", 0, 2, 98304),      # two large stages
+])
+def test_ring_shapes(name, ctx, stages, stage_bytes):
+    """Ring shapes other than the weight format's default change the rows per
+    chunk, the K split of the GEMV warps and the positions per attention
+    chunk; every one must still match the oracle."""
+    cfg = si.get_config(name)
+    opts = amk.default_options(ring_stages=stages, stage_bytes=stage_bytes)
+    pair = Pair(cfg, options=opts)
+    st = pair.dec.stats()
+    assert (st.ring_stages, st.stage_bytes) == (stages, stage_bytes)
+    if ctx:
+        pair.fill_kv(ctx)
+    tok = si.make_prompt(cfg, 1, seed=10 + ctx)[0]
+    g, am, ref, ref_am = pair.step(tok, ctx)
+    compare(cfg, g, am, ref, ref_am, what=f"{name} ctx {ctx} ring {stages} x {stage_bytes}")
+    del pair
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("name", ["tinyllama", "llama1b_w8", "tiny"])
 def test_position0_schedule_matches_general(name):
     """At position 0 the schedule without the attention level gives the same
