@@ -287,6 +287,10 @@ typedef struct {
     int64_t epoch;          /* decode steps since the last reset */
 } amk_plan_stats;
 AMK_API int amk_get_stats(amk_handle *h, amk_plan_stats *out);
+/* The same figures for a host plan (amk_plan_create), with the resolved
+ * schedule knobs (ring shape, attention splits); epoch is 0.  Host only: no
+ * device is touched.  AMK_ERR_INVALID_ARG on a NULL argument. */
+AMK_API int amk_plan_get_stats(const amk_plan *p, amk_plan_stats *out);
 
 /* Introspection for tests: device pointers (owned by the handle) to the
  * fp32 activations the last step left, per layer l:

@@ -145,6 +145,12 @@ class Plan:
                  "pair": G.buffers[b].pair} for b in range(G.n_buffers)]
         return {"n_counters": G.n_counters, "buffers": bufs, "tasks": tasks, "queues": queues}
 
+    def stats(self) -> abi.PlanStats:
+        """Task and counter counts, resolved schedule knobs, streamed bytes."""
+        st = abi.PlanStats()
+        _check(abi.lib().amk_plan_get_stats(self._p, ctypes.byref(st)), "amk_plan_get_stats")
+        return st
+
     def task_info(self) -> Tuple[List[int], List[int]]:
         G = abi.Graph()
         _check(abi.lib().amk_plan_graph(self._p, ctypes.byref(G)), "amk_plan_graph")

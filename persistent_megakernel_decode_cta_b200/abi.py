@@ -123,6 +123,7 @@ SIGNATURES = {
     "amk_get_kv": (ctypes.c_int, [c_vp, c_i32, ctypes.POINTER(c_vp), ctypes.POINTER(c_vp)]),
     "amk_get_logits": (ctypes.c_int, [c_vp, ctypes.POINTER(c_vp)]),
     "amk_get_stats": (ctypes.c_int, [c_vp, ctypes.POINTER(PlanStats)]),
+    "amk_plan_get_stats": (ctypes.c_int, [c_vp, ctypes.POINTER(PlanStats)]),
     "amk_get_error_info": (ctypes.c_int, [c_vp, ctypes.POINTER(ErrorInfo)]),
     "amk_get_workspace": (ctypes.c_int, [c_vp, ctypes.POINTER(Workspace)]),
     "amk_get_profile": (ctypes.c_int, [c_vp, ctypes.POINTER(ctypes.c_uint64), c_i64]),

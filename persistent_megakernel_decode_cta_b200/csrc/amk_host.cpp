@@ -658,11 +658,10 @@ extern "C" int amk_get_logits(amk_handle *h, float **logits_dev)
     return AMK_OK;
 }
 
-extern "C" int amk_get_stats(amk_handle *h, amk_plan_stats *o)
+extern "C" int amk_plan_get_stats(const amk_plan *P, amk_plan_stats *o)
 {
-    if (!h || !o)
-        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_get_stats: NULL argument");
-    const amk_plan *P = h->plan;
+    if (!P || !o)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_plan_get_stats: NULL argument");
     memset(o, 0, sizeof *o);
     o->n_tasks = (int32_t)P->tasks.size();
     o->n_counters = P->n_counters;
@@ -674,8 +673,17 @@ extern "C" int amk_get_stats(amk_handle *h, amk_plan_stats *o)
     o->threads_per_cta = amk::kThreads;
     o->weight_bytes = P->weight_bytes;
     o->kv_row_bytes = P->kv_row_bytes;
-    o->epoch = h->epoch;
     return AMK_OK;
+}
+
+extern "C" int amk_get_stats(amk_handle *h, amk_plan_stats *o)
+{
+    if (!h || !o)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_get_stats: NULL argument");
+    const int rc = amk_plan_get_stats(h->plan, o);
+    if (rc == AMK_OK)
+        o->epoch = h->epoch;
+    return rc;
 }
 
 extern "C" int amk_get_workspace(amk_handle *h, amk_workspace *out)

@@ -159,3 +159,19 @@ def test_bad_options_rejected():
     with pytest.raises(amk.AmkError) as e:
         amk.Plan(cfg, 4, amk.default_options(stage_bytes=1000))
     assert e.value.name == "AMK_ERR_INVALID_ARG"
+
+
+@pytest.mark.parametrize("name", ["tiny", "smol135", "tinyllama", "llama1b_w8", "llama7b",
+                                  "llama7b_w8"])
+def test_ring_shape_resolved_per_weight_format(name):
+    """Left at 0, the ring takes 48 KiB stages for int8 weights and 64 KiB for
+    bf16, as many as make 192 KiB; explicit values are kept."""
+    cfg = si.get_config(name)
+    st = amk.Plan(cfg, 148).stats()
+    want = (4, 48 * 1024) if cfg.quant == "w8a16" else (3, 64 * 1024)
+    assert (st.ring_stages, st.stage_bytes) == want
+    assert st.n_tasks > 0 and st.epoch == 0 and st.smem_bytes <= 227 * 1024
+    st = amk.Plan(cfg, 148, amk.default_options(stage_bytes=32768)).stats()
+    assert (st.ring_stages, st.stage_bytes) == (6, 32768)
+    st = amk.Plan(cfg, 148, amk.default_options(ring_stages=2, stage_bytes=65536)).stats()
+    assert (st.ring_stages, st.stage_bytes) == (2, 65536)
