@@ -25,7 +25,7 @@ from typing import Dict, Iterable, List, Optional, Tuple
 from . import Decoder, AmkError, default_options
 
 DEFAULT_SPACE: Dict[str, List[int]] = {
-    "ring_stages": [2, 3],
+    "ring_stages": [0, 2],  # 0: as many stages as make 192 KiB (6 x 32, 4 x 48, 3 x 64 KiB)
     "stage_bytes": [32768, 49152, 65536],
     "attn_splits": [0, 2, 4],
     "ffn_fused": [1, 2, -1],
