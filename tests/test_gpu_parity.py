@@ -196,6 +196,22 @@ def test_tiny_shape_variants_to_the_last_cache_row(edit):
     assert e.value.name == "AMK_ERR_POS_RANGE"
 
 
+@pytest.mark.parametrize("name", ["tinyllama", "llama1b_w8"])
+def test_last_cache_row_full_size(name):
+    """A full-size step at the last position the cache holds (max_ctx - 1,
+    every earlier row filled): the longest split-K attention chunks and the
+    last KV row, against the oracle."""
+    cfg = si.get_config(name)
+    pos = cfg.max_ctx - 1
+    pair = Pair(cfg)
+    pair.fill_kv(pos)
+    tok = si.make_prompt(cfg, 1, seed=10)[0]
+    g, am, ref, ref_am = pair.step(tok, pos)
+    compare(cfg, g, am, ref, ref_am, f"{name} at the last cache row {pos}")
+    del pair
+    torch.cuda.empty_cache()
+
+
 def test_ragged_sm_count_full_size():
     """A full-size shape on a prime number of CTAs (ragged tiles on every
     level, several tasks per queue) against the oracle at a long context."""
