@@ -59,7 +59,7 @@ WORKLOADS = {
     "tiny-ctx4": ("tiny", 4),
 }
 DEFAULT_WORKLOAD = "llama7b-ctx2048"
-KERNEL_SOURCES = ["persistent_megakernel_decode_cta_b200/csrc/amk_kernel.cu",
+KERNEL_SOURCES = ["persistent_megakernel_decode_cta_b200/csrc/amk_kernel_body.cuh",
                   "persistent_megakernel_decode_cta_b200/csrc/amk_internal.h"]
 
 

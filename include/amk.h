@@ -352,12 +352,17 @@ AMK_API int amk_get_error_info(amk_handle *h, amk_error_info *out);
  *              device errors are not reported.
  * Returns AMK_ERR_UNSUPPORTED, without touching the GPU, when the model's
  * scratch would exceed AMK_NOALLOC_SCRATCH_BYTES (amk_last_error says how
- * much it needs).  The first call on each device looks up the static array's
- * device address (cudaGetSymbolAddress); make that first call before any
- * stream capture.  Every call re-uploads the schedule and clears the
- * counters in the shared array, which keeps the last call's contents: calls
- * that can overlap on the GPU (other streams, other host threads) race on
- * it and must be serialised by the caller. */
+ * much it needs), and when cuda_stream is capturing (the schedule uploads
+ * read host stack memory).  AMK_ERR_INVALID_ARG for the position-0 schedule
+ * (amk_plan_pos0) at any pos other than 0.  The first call on each device is
+ * the set-up: it looks up the static array's device address
+ * (cudaGetSymbolAddress, which may load the library's device code), so make
+ * that first call before any stream capture; later calls look the address
+ * up again, so it stays right after a cudaDeviceReset.  Every call
+ * re-uploads the schedule and clears the counters in the shared array, which
+ * keeps the last call's contents: calls that can overlap on the GPU (other
+ * streams, other host threads) race on it and must be serialised by the
+ * caller. */
 #define AMK_NOALLOC_SCRATCH_BYTES (16u << 20)
 AMK_API int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *w, void *kv_cache,
                                     int32_t token_id, int32_t pos, float *logits_dev,

@@ -14,7 +14,6 @@
 
 #include <cstdint>
 #include <cstring>
-#include <mutex>
 
 #include "amk.h"
 #include "amk_internal.h"
@@ -32,10 +31,6 @@ namespace {
 
 constexpr size_t kScratchBytes = AMK_NOALLOC_SCRATCH_BYTES;
 __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
-
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void *g_scratch_addr[kMaxDevices];  // device address of g_scratch, per device
 
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -72,27 +67,21 @@ Layout layout_of(const amk_plan &P)
     return o;
 }
 
-// Device address of g_scratch for the current device, looked up on the first
-// call for that device.
+// Device address of g_scratch on the current device.  In host code the name
+// g_scratch is only a host-side stand-in, so the kernel gets the address the
+// runtime reports.  The first call on a device is the set-up (it loads the
+// library's device code there if that has not happened yet); every call looks
+// the address up again, a host-side query, so that it stays right after the
+// device's context has been reset (which reloads the device code, possibly
+// at another address).
 int scratch_address(unsigned char **out)
 {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
-        return amk_set_error(AMK_ERR_NO_DEVICE, "amk_decode_step_noalloc: %s",
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
+    if (e != cudaSuccess || !p)
+        return amk_set_error(AMK_ERR_CUDA, "cudaGetSymbolAddress(g_scratch): %s",
                              cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDevices)
-        return amk_set_error(AMK_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_scratch);
-        if (e != cudaSuccess || !p)
-            return amk_set_error(AMK_ERR_CUDA, "cudaGetSymbolAddress(g_scratch): %s",
-                                 cudaGetErrorString(e));
-        g_scratch_addr[dev] = p;
-    }
-    *out = static_cast<unsigned char *>(g_scratch_addr[dev]);
+    *out = static_cast<unsigned char *>(p);
     return AMK_OK;
 }
 
@@ -134,9 +123,29 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
                              "amk_decode_step_noalloc: this model needs %zu bytes of scratch, "
                              "more than the %zu-byte static array; use amk_create",
                              lay.total, kScratchBytes);
+    if (P.is_pos0 && pos != 0)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_decode_step_noalloc: the position-0 "
+                             "schedule runs only steps at position 0 (pos %d)", pos);
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    {
+        // the schedule uploads below read host stack buffers; a captured
+        // graph would keep pointers to them
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        const cudaError_t ce = cudaStreamIsCapturing(st, &cs);
+        if (ce != cudaSuccess)
+            return fail_cuda(ce, "cudaStreamIsCapturing");
+        if (cs != cudaStreamCaptureStatusNone)
+            return amk_set_error(AMK_ERR_UNSUPPORTED, "amk_decode_step_noalloc: the stream is "
+                                 "capturing; the call uploads its schedule from host stack "
+                                 "memory and does nothing under capture");
+    }
     int dev = 0, sms = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t de = cudaGetDevice(&dev);
+    if (de == cudaSuccess)
+        de = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (de != cudaSuccess)
+        return amk_set_error(AMK_ERR_NO_DEVICE, "amk_decode_step_noalloc: %s",
+                             cudaGetErrorString(de));
     if (P.n_sms > sms)
         return amk_set_error(AMK_ERR_INVALID_ARG, "plan made for %d SMs, device has %d",
                              P.n_sms, sms);
@@ -144,7 +153,6 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     int rc = scratch_address(&base);
     if (rc != AMK_OK)
         return rc;
-    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     cudaError_t e;
     // per-layer pointers must all be present before any task is resolved
     for (int l = 0; l < c.n_layers; ++l) {
