@@ -211,13 +211,23 @@ def job_us_per_token(elapsed_ms: float, steps: int, world: int) -> float:
     return elapsed_ms * 1e3 / (steps * world)
 
 
-def oracle_steps(cfg, weights, ctx, kv_fill, budget_s: float, max_steps: int):
+def cpu_model() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_steps(cfg, weights, ctx, kv_fill, budget_s: float, max_steps: int, threads: int = 0):
     """Times full fp64 oracle decode steps at position ctx (as many as fit the
-    budget, at least one).  Returns (us per token, steps, threads, logits of
-    the first step)."""
+    budget, at least one) on `threads` OpenMP threads (0: all host cores).
+    Returns (us per token, steps, threads, logits of the first step)."""
     import oracle
     m = oracle.OracleModel(cfg, weights)
-    threads = oracle.set_threads(0)
+    threads = oracle.set_threads(threads if threads > 0 else (os.cpu_count() or 1))
     if kv_fill is not None:
         m.fill_kv(kv_fill)
     tok = si.make_prompt(cfg, 1, seed=10 + ctx)[0]
@@ -233,6 +243,45 @@ def oracle_steps(cfg, weights, ctx, kv_fill, budget_s: float, max_steps: int):
         if time.perf_counter() - t_all > budget_s:
             break
     return statistics.median(times) * 1e6, len(times), threads, first
+
+
+KINDS = {1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead", 7: "ffn"}
+
+
+def phase_shares(P):
+    """Where the consumers' time goes, from the kernel's phase timers of one
+    step (uint64 [n_sms, kinds, fields]; amk_get_profile): shares of the
+    consumer warpgroups' time from kernel start to their end, summed over
+    SMs, and the producer lane's share of time stalled on a full ring or the
+    in-flight cap."""
+    P = P.astype(np.float64)
+    total = float((P[:, 0, 1] - P[:, 0, 0]).sum())
+    prod = float((P[:, 0, 3] - P[:, 0, 0]).sum())
+    wait = float(P[:, 1:, 1].sum())
+    prologue = float(P[:, 1:, 2].sum())
+    ring = float(P[:, 1:, 6].sum()) / 8.0
+    compute = float(P[:, 1:, 7].sum()) / 8.0
+    run = float(P[:, 1:, 4].sum())
+    epi = float(P[:, 1:, 5].sum())
+    per_kind = {}
+    for k, name in KINDS.items():
+        n = float(P[:, k, 0].sum())
+        if n == 0:
+            continue
+        f = P[:, k, :].sum(axis=0) / n / 1e3
+        per_kind[name] = {"tasks": int(n), "counter_wait_us": f[1], "prologue_us": f[2],
+                          "ring_wait_us": f[6] / 8.0, "gemv_or_attention_us": f[7] / 8.0,
+                          "epilogue_release_us": f[5], "run_us": f[4]}
+    return {
+        "counter_wait": wait / total, "prologue": prologue / total,
+        "ring_wait": ring / total, "gemv_or_attention": compute / total,
+        "epilogue_release": epi / total,
+        "other": max(0.0, 1.0 - (wait + run) / total),
+        "producer_stalled": float(P[:, 0, 2].sum()) / prod if prod > 0 else None,
+        "per_task_kind_us": per_kind,
+        "how": "phase timers (globaltimer) of one profiled step after the timed region; "
+               "shares of the consumer warpgroups' time, summed over SMs",
+    }
 
 
 def run_reference(args):
@@ -319,9 +368,13 @@ def run_ours(args):
         parity = {"verdict": "PASS" if err <= tol else "FAIL", "max_abs_dlogit": err,
                   "tolerance": tol, "max_abs_logit": scale,
                   "argmax_match": int(np.argmax(g)) == int(np.argmax(ref))}
+        us1, n1, _, _ = oracle_steps(cfg, w, ctx, kv, 0.0, 1, threads=1)
         cpu_base = {"value": us, "unit": UNIT, "cores": threads, "kind": "oracle",
                     "sample": f"{n} full fp64 decode steps of {name} at position {ctx} "
-                              f"(~{budget:.0f} s budget), median"}
+                              f"(~{budget:.0f} s budget), median",
+                    "cpu_model": cpu_model(), "host_cores": os.cpu_count(),
+                    "one_core": {"value": us1, "unit": UNIT, "cores": 1,
+                                 "sample": f"{n1} full fp64 decode step on one thread"}}
 
     # ---- device timing --------------------------------------------------------
     def step():
@@ -354,6 +407,7 @@ def run_ours(args):
     per_launch = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     elapsed_ms = max_over_ranks(world, elapsed_ms)
     kernel_ms = max_over_ranks(world, statistics.mean(per_launch))
+    qs = np.percentile(np.array(per_launch) * 1e3, [10, 50, 90])
 
     # ---- end to end: host token in, host logits + token out, every step ------
     host_logits = torch.empty(cfg.vocab, dtype=torch.float32).pin_memory()
@@ -371,6 +425,25 @@ def run_ours(args):
             tok = dec.step_host(tok, ctx, hl)
     e2e_s = max_over_ranks(world, time.perf_counter() - t0)
 
+    # ---- phase timers of one profiled step (outside the timed region) -------
+    phases = None
+    if rank == 0 and not args.no_phases:
+        popts = amk.default_options()
+        popts.profile = 1
+        with torch.cuda.stream(stream):
+            pdec = amk.Decoder(cfg, w, popts, stream=stream.cuda_stream)
+            if kv is not None:
+                for l in range(cfg.n_layers):
+                    k, v = pdec.kv(l)
+                    k[:, :ctx].copy_(kv[l, 0])
+                    v[:, :ctx].copy_(kv[l, 1])
+            pdec.step(tok0, ctx, want_argmax=False)
+            for _ in range(3):
+                pdec.step(-1, ctx, want_argmax=False)
+        torch.cuda.synchronize()
+        phases = phase_shares(pdec.profile())
+        pdec.close()
+
     nbytes = algorithmic_bytes(cfg, ctx)
     peak, peak_kind = measured_peak()
     achieved = nbytes / (kernel_ms * 1e-3) / 1e9
@@ -380,7 +453,9 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": ("int8 weights x int16 activations, i32 then f32 accumulate"
+                      if cfg.quant == "w8a16" else "bf16 weights x f32 activations, f32 accumulate"),
             "data": "synthetic (seeded random-init weights and KV cache)",
             "config": dict(workload_config(name, cfg, ctx),
                            parallelism=f"replicas{world}" if world > 1 else "single"),
@@ -395,6 +470,9 @@ def run_ours(args):
             "e2e": {"value": job_us_per_token(e2e_s * 1e3, K_e2e, world), "unit": UNIT,
                     "h2d_bytes_per_step": 4, "d2h_bytes_per_step": cfg.vocab * 4 + 8 + 32,
                     "steps": K_e2e},
+            "per_step_us": {"p10": float(qs[0]), "p50": float(qs[1]), "p90": float(qs[2]),
+                            "mean": kernel_ms * 1e3, "steps": K},
+            "phases": phases,
             "gpu_launches": K,
             "clocks": clocks.summary(),
             "schedule": {"tasks": st.n_tasks, "ctas": st.n_sms, "ring_stages": st.ring_stages,
@@ -418,6 +496,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-phases", action="store_true",
+                    help="skip the profiled step that reports the phase-timer shares")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

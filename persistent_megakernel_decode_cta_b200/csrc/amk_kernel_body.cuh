@@ -651,6 +651,8 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
     const uint64_t pol_w = evict_first_policy();  // weights: streamed once per step
     const int NS = p.ring_stages;
     uint32_t k = 0;  // chunks issued
+    int pst = 0;          // stage of chunk k (k % NS)
+    uint32_t ppar = 0u;   // phase of chunk k's full barriers ((k / NS) & 1)
     volatile int *abort_flag = s.flags;
     bool stop = false;
     uint64_t prof_wait = 0, prof_bytes = 0, prof_setup = 0;
@@ -679,10 +681,10 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
         const uint8_t *w0 = static_cast<const uint8_t *>(d.w0);
         const uint8_t *w1 = static_cast<const uint8_t *>(d.w1);
         for (int i = 0; i < g.nchunks; ++i, ++k) {
-            const int st = k % NS;
+            const int st = pst;
             const uint32_t done_below = k >= (uint32_t)NS ? k - NS + 1 : 0u;
             if (k >= (uint32_t)NS) {
-                const uint32_t par = ((k / NS) - 1) & 1;
+                const uint32_t par = ppar ^ 1u;  // the stage's previous use
                 uint32_t it = 0;
                 uint64_t t0 = 0;
                 while (!mbar_try_wait(s.empty_a + 8 * st, par)) {
@@ -706,7 +708,11 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
             }
             const uint32_t dst = s.ring_a + (uint32_t)st * p.stage_bytes;
             const uint32_t bar0 = s.full_a + 8 * (st * kPieces);
-            const uint32_t par = (k / NS) & 1;
+            const uint32_t par = ppar;
+            if (++pst == NS) {  // the stage and phase of the next chunk
+                pst = 0;
+                ppar ^= 1u;
+            }
             if (p.prof && i == 0)  // time from the task's start to its first copy
                 prof_setup += (gtimer() - ts) - (prof_wait - wait_before);
             int used = 0;  // piece barriers armed for this chunk
@@ -827,13 +833,31 @@ __device__ void producer_loop(const KParams &p, const SmemLayout &s, int qb, int
 }
 
 // ------------------------------------------------------------------ consumers
-// Waits (all lanes of a warp together) until the ring stage of chunk k is full:
-// lane l polls piece l % kPieces of the stage, so one SIMT poll covers every
-// piece barrier.
-__device__ __forceinline__ bool wait_full(const KParams &p, const SmemLayout &s, uint32_t k)
+// The consumers' position in the ring: chunk k sits in stage st = k % stages,
+// whose full barrier completes phase par = (k / stages) & 1 for it.  Advanced
+// one chunk at a time, so that no chunk pays for a division by the run-time
+// stage count.
+struct RingPos {
+    uint32_t k;
+    int st;
+    uint32_t par;
+    __device__ __forceinline__ void advance(int stages)
+    {
+        ++k;
+        if (++st == stages) {
+            st = 0;
+            par ^= 1u;
+        }
+    }
+};
+
+// Waits (all lanes of a warp together) until the ring stage of chunk kc is
+// full: lane l polls piece l % kPieces of the stage, so one SIMT poll covers
+// every piece barrier.
+__device__ __forceinline__ bool wait_full(const KParams &p, const SmemLayout &s, const RingPos &kc)
 {
-    const int st = k % p.ring_stages;
-    const uint32_t par = (k / p.ring_stages) & 1;
+    const int st = kc.st;
+    const uint32_t par = kc.par;
     const uint32_t bar = s.full_a + 8 * (st * kPieces + (threadIdx.x & (kPieces - 1)));
     volatile int *abort_flag = s.flags;
     uint32_t it = 0;
@@ -854,11 +878,11 @@ __device__ __forceinline__ bool wait_full(const KParams &p, const SmemLayout &s,
 }
 
 __device__ __forceinline__ void release_stage(const KParams &p, const SmemLayout &s,
-                                              uint32_t k, int lane)
+                                              const RingPos &kc, int lane)
 {
     __syncwarp();
     if (lane == 0)
-        mbar_arrive(s.empty_a + 8 * (k % p.ring_stages));
+        mbar_arrive(s.empty_a + 8 * kc.st);
 }
 
 __device__ void record_error(const KParams &p, uint32_t code, int task, int ctr, uint32_t seen,
@@ -958,7 +982,7 @@ __device__ void rmsnorm_prologue(const KParams &p, const SmemLayout &s, const fl
 // shared vector (prologue output) or, when xg is set, straight from L2.
 template <int ESZ, int VB>
 __device__ __forceinline__ bool gemv_task(const KParams &p, const SmemLayout &s, const Geom g,
-                                          uint32_t &kc, int warp, int lane, const float *xg,
+                                          RingPos &kc, int warp, int lane, const float *xg,
                                           uint64_t *wt)
 {
     constexpr int E = VB / ESZ;   // elements per vector (even)
@@ -1010,7 +1034,7 @@ __device__ __forceinline__ bool gemv_task(const KParams &p, const SmemLayout &s,
         }
     }
     const uint32_t red_a = s.red_a + (uint32_t)warp * kMaxTaskRows * 4;
-    const int NS = p.ring_stages, SB = p.stage_bytes;
+    const int SB = p.stage_bytes;
     uint64_t tA = 0, tB = 0;
     for (int i = 0; i < g.ngu; ++i) {
         if (wt)
@@ -1021,7 +1045,7 @@ __device__ __forceinline__ bool gemv_task(const KParams &p, const SmemLayout &s,
             tB = gtimer();
             wt[0] += tB - tA;
         }
-        const uint32_t stage_a = s.ring_a + (uint32_t)(kc % NS) * SB;
+        const uint32_t stage_a = s.ring_a + (uint32_t)kc.st * SB;
         const int part = i / nck, c = i - part * nck;
         const int r = c * rpc;
         const int nr = min(rpc, R - r);
@@ -1067,7 +1091,7 @@ __device__ __forceinline__ bool gemv_task(const KParams &p, const SmemLayout &s,
             }
         }
         release_stage(p, s, kc, lane);
-        ++kc;
+        kc.advance(p.ring_stages);
         if (wt)
             wt[1] += gtimer() - tB;
     }
@@ -1137,11 +1161,20 @@ struct LaneX {
 
 // Rows j0 + RG r (r < RW) of a ring chunk against the lane's activations;
 // each row's warp total goes to red[rowbase + row] (the warp's red slice).
+// The lane reads vector i of a row at byte voff[i] of it: every lane takes
+// all NI vectors, with no guard in the loop (a lane's vectors past the end of
+// its K-slice re-read a vector of the slice and meet zero activations), so
+// that the compiler can issue the loads of all RW rows ahead of the math.
 template <int ESZ, int NI, int RW>
-__device__ __forceinline__ void gemv_rows(const LaneX<ESZ, NI> &x, uint32_t lane_a, int RB, int RG,
-                                          int j0, int ni, uint32_t red_a, int rowbase, int lane)
+__device__ __forceinline__ void gemv_rows(const LaneX<ESZ, NI> &x, uint32_t stage_a,
+                                          const uint32_t (&voff)[NI], int RB, int RG, int j0,
+                                          uint32_t red_a, int rowbase, int lane)
 {
     float sr[RW];
+    uint32_t ra[RW];
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+        ra[r] = stage_a + (uint32_t)((j0 + r * RG) * RB);
     if constexpr (ESZ == 2) {
         float acc[RW][4];
 #pragma unroll
@@ -1151,20 +1184,18 @@ __device__ __forceinline__ void gemv_rows(const LaneX<ESZ, NI> &x, uint32_t lane
                 acc[r][q] = 0.f;
 #pragma unroll
         for (int i = 0; i < NI; ++i) {
-            if (i < ni) {
-                uint4 w[RW];
+            uint4 w[RW];
 #pragma unroll
-                for (int r = 0; r < RW; ++r)
-                    w[r] = lds128(lane_a + (uint32_t)((j0 + r * RG) * RB + i * 512));
+            for (int r = 0; r < RW; ++r)
+                w[r] = lds128(ra[r] + voff[i]);
 #pragma unroll
-                for (int r = 0; r < RW; ++r) {
-                    const uint32_t A[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+            for (int r = 0; r < RW; ++r) {
+                const uint32_t A[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        acc[r][q] = fmaf(__uint_as_float(A[q] << 16), x.f[i][2 * q], acc[r][q]);
-                        acc[r][q] = fmaf(__uint_as_float(A[q] & 0xffff0000u), x.f[i][2 * q + 1],
-                                         acc[r][q]);
-                    }
+                for (int q = 0; q < 4; ++q) {
+                    acc[r][q] = fmaf(__uint_as_float(A[q] << 16), x.f[i][2 * q], acc[r][q]);
+                    acc[r][q] = fmaf(__uint_as_float(A[q] & 0xffff0000u), x.f[i][2 * q + 1],
+                                     acc[r][q]);
                 }
             }
         }
@@ -1178,19 +1209,17 @@ __device__ __forceinline__ void gemv_rows(const LaneX<ESZ, NI> &x, uint32_t lane
             acc[r][0] = acc[r][1] = 0;
 #pragma unroll
         for (int i = 0; i < NI; ++i) {
-            if (i < ni) {
-                uint4 w[RW];
+            uint4 w[RW];
 #pragma unroll
-                for (int r = 0; r < RW; ++r)
-                    w[r] = lds128(lane_a + (uint32_t)((j0 + r * RG) * RB + i * 512));
+            for (int r = 0; r < RW; ++r)
+                w[r] = lds128(ra[r] + voff[i]);
 #pragma unroll
-                for (int r = 0; r < RW; ++r) {
-                    const uint32_t A[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+            for (int r = 0; r < RW; ++r) {
+                const uint32_t A[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        acc[r][0] = dp2a_lo(x.q[i][2 * q], A[q], acc[r][0]);
-                        acc[r][1] = dp2a_hi(x.q[i][2 * q + 1], A[q], acc[r][1]);
-                    }
+                for (int q = 0; q < 4; ++q) {
+                    acc[r][0] = dp2a_lo(x.q[i][2 * q], A[q], acc[r][0]);
+                    acc[r][1] = dp2a_hi(x.q[i][2 * q + 1], A[q], acc[r][1]);
                 }
             }
         }
@@ -1214,7 +1243,7 @@ __device__ __forceinline__ void gemv_rows(const LaneX<ESZ, NI> &x, uint32_t lane
 // to the shape, not to the largest one.
 template <int ESZ, int NI>
 __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &s, const Geom g,
-                                            uint32_t &kc, int warp, int lane, const float *xg,
+                                            RingPos &kc, int warp, int lane, const float *xg,
                                             uint64_t *wt)
 {
     using LX = LaneX<ESZ, NI>;
@@ -1276,9 +1305,20 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
                 }
         }
     }
+    // byte offset in a row of the lane's vector i: its own while i < ni,
+    // else (zero activations) one that the slice surely holds
+    uint32_t voff[NI];
+#pragma unroll
+    for (int i = 0; i < NI; ++i)
+        voff[i] = (uint32_t)(i < ni ? vb + lane + 32 * i : ni > 0 ? vb + lane : min(vb, NV - 1)) *
+                  16;
     const uint32_t red_a = s.red_a + (uint32_t)warp * kMaxTaskRows * 4;
-    const int NS = p.ring_stages, SB = p.stage_bytes;
+    const int SB = p.stage_bytes;
+    // rows rg + RG m (m < nrw) of a chunk are this warp's: rpc / RG of a full
+    // chunk (rpc is a multiple of RG); the last chunk of a part may hold fewer
+    const int nrw_full = rpc / RG;
     uint64_t tA = 0, tB = 0;
+    int part = 0, cc = 0;  // chunk c = part * nck + cc, advanced without divisions
     for (int c = 0; c < g.ngu; ++c) {
         if (wt)
             tA = gtimer();
@@ -1288,24 +1328,26 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
             tB = gtimer();
             wt[0] += tB - tA;
         }
-        const uint32_t stage_a = s.ring_a + (uint32_t)(kc % NS) * SB;
-        const int part = c / nck, cc = c - part * nck;
+        const uint32_t stage_a = s.ring_a + (uint32_t)kc.st * SB;
         const int r0 = cc * rpc;
         const int nr = min(rpc, R - r0);
         const int rowbase = part * R + r0;
-        const uint32_t lane_a = stage_a + (uint32_t)(vb + lane) * 16;
-        const int nrw = nr > rg ? (nr - rg + RG - 1) / RG : 0;  // rows rg + RG m, m < nrw
+        const int nrw = nr == rpc ? nrw_full : nr > rg ? (nr - rg + RG - 1) / RG : 0;
+        if (++cc == nck) {
+            cc = 0;
+            ++part;
+        }
         int m = 0;
         for (; m + 4 <= nrw; m += 4)
-            gemv_rows<ESZ, NI, 4>(x, lane_a, RB, RG, rg + RG * m, ni, red_a, rowbase, lane);
+            gemv_rows<ESZ, NI, 4>(x, stage_a, voff, RB, RG, rg + RG * m, red_a, rowbase, lane);
         if (m + 2 <= nrw) {
-            gemv_rows<ESZ, NI, 2>(x, lane_a, RB, RG, rg + RG * m, ni, red_a, rowbase, lane);
+            gemv_rows<ESZ, NI, 2>(x, stage_a, voff, RB, RG, rg + RG * m, red_a, rowbase, lane);
             m += 2;
         }
         if (m < nrw)
-            gemv_rows<ESZ, NI, 1>(x, lane_a, RB, RG, rg + RG * m, ni, red_a, rowbase, lane);
+            gemv_rows<ESZ, NI, 1>(x, stage_a, voff, RB, RG, rg + RG * m, red_a, rowbase, lane);
         release_stage(p, s, kc, lane);
-        ++kc;
+        kc.advance(p.ring_stages);
         if (wt)
             wt[1] += gtimer() - tB;
     }
@@ -1315,7 +1357,7 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
 // Dispatch on the vectors a lane holds for this task's K-slice.
 template <int ESZ>
 __device__ __forceinline__ bool gemv16(const KParams &p, const SmemLayout &s, const Geom &g,
-                                       uint32_t &kc, int warp, int lane, const float *xg,
+                                       RingPos &kc, int warp, int lane, const float *xg,
                                        uint64_t *wt)
 {
     const int vps = (g.RB / 16 + g.KS - 1) / g.KS;
@@ -1344,7 +1386,7 @@ __device__ __forceinline__ bool gemv16(const KParams &p, const SmemLayout &s, co
 // time (models with odd row widths, or a bf16 tied head on int8 layers).
 template <int Q8, int GENERIC>
 __device__ __forceinline__ bool run_gemv(const KParams &p, const SmemLayout &s, const Geom &g,
-                                         uint32_t &kc, int warp, int lane, const float *xg,
+                                         RingPos &kc, int warp, int lane, const float *xg,
                                          uint64_t *wt)
 {
     if constexpr (!GENERIC) {
@@ -1431,7 +1473,7 @@ __device__ __forceinline__ void lds_bf16(uint32_t a, float (&out)[E])
 // writes (m, l, o[hd]) per query head of the group, unnormalised.
 template <int E>
 __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s,
-                                          const TaskDesc &d, const Geom &g, uint32_t &kc,
+                                          const TaskDesc &d, const Geom &g, RingPos &kc,
                                           int ct, int warp, int lane, uint64_t *wt)
 {
     const int l = d.layer, gi = d.r0, c = d.r1;
@@ -1527,7 +1569,7 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
             tB = gtimer();
             wt[0] += tB - tA;
         }
-        const uint32_t ka = s.ring_a + (uint32_t)(kc % p.ring_stages) * p.stage_bytes;
+        const uint32_t ka = s.ring_a + (uint32_t)kc.st * p.stage_bytes;
         const uint32_t va = ka + (uint32_t)g.P * hd * 2;
         const int a = g.pa + i * g.P;
         const int n = min(g.P, g.pb - a);
@@ -1585,7 +1627,7 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
             m = mn;
         }
         release_stage(p, s, kc, lane);
-        ++kc;
+        kc.advance(p.ring_stages);
         if (wt)
             wt[1] += gtimer() - tB;
     }
@@ -1782,7 +1824,7 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v)
 
 template <int E>
 __device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
-                                          const TaskDesc &d, const Geom &g, uint32_t &kc,
+                                          const TaskDesc &d, const Geom &g, RingPos &kc,
                                           int ct, int warp, int lane, uint64_t *wt)
 {
     if (!attn_chunk<E>(p, s, d, g, kc, ct, warp, lane, wt))
@@ -1911,7 +1953,7 @@ constexpr int kQOff = 1024;  // byte offset of the int16 activation copy in vec
 // which measured faster than register copies for the narrow slices of the
 // models that fuse the level
 __device__ __forceinline__ bool ffn_down_bf16(const KParams &p, const SmemLayout &s,
-                                              const Geom &g, const TaskDesc &d, uint32_t &kc,
+                                              const Geom &g, const TaskDesc &d, RingPos &kc,
                                               int ct, int lane)
 {
     constexpr int E = 8;  // bf16 elements per box row
@@ -1921,7 +1963,7 @@ __device__ __forceinline__ bool ffn_down_bf16(const KParams &p, const SmemLayout
         const int r0w = c2 * g.rpc2, nrows = min(g.rpc2, h - r0w);
         if (!wait_full(p, s, kc))
             return false;
-        const uint32_t st_a = s.ring_a + (uint32_t)(kc % p.ring_stages) * p.stage_bytes;
+        const uint32_t st_a = s.ring_a + (uint32_t)kc.st * p.stage_bytes;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             const int lr = ct + kConsumerThreads * k;
@@ -1941,7 +1983,7 @@ __device__ __forceinline__ bool ffn_down_bf16(const KParams &p, const SmemLayout
             }
         }
         release_stage(p, s, kc, lane);
-        ++kc;
+        kc.advance(p.ring_stages);
     }
     return true;
 }
@@ -1950,7 +1992,7 @@ __device__ __forceinline__ bool ffn_down_bf16(const KParams &p, const SmemLayout
 // (NCB >= ncb column groups of 16) and multiplies them with dp2a
 template <int NCB>
 __device__ __forceinline__ bool ffn_down_i8(const KParams &p, const SmemLayout &s, const Geom &g,
-                                            const TaskDesc &d, uint32_t &kc, int ct, int lane)
+                                            const TaskDesc &d, RingPos &kc, int ct, int lane)
 {
     const int ncb = g.ncb, h = p.hidden;
     long long *acc_out = p.xacc + (size_t)d.layer * h;
@@ -1978,7 +2020,7 @@ __device__ __forceinline__ bool ffn_down_i8(const KParams &p, const SmemLayout &
         }
         if (!wait_full(p, s, kc))
             return false;
-        const uint32_t st_a = s.ring_a + (uint32_t)(kc % p.ring_stages) * p.stage_bytes;
+        const uint32_t st_a = s.ring_a + (uint32_t)kc.st * p.stage_bytes;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             const int lr = ct + kConsumerThreads * k;
@@ -2001,7 +2043,7 @@ __device__ __forceinline__ bool ffn_down_i8(const KParams &p, const SmemLayout &
             }
         }
         release_stage(p, s, kc, lane);
-        ++kc;
+        kc.advance(p.ring_stages);
     }
     return true;
 }
@@ -2011,7 +2053,7 @@ __device__ __forceinline__ bool ffn_down_i8(const KParams &p, const SmemLayout &
 // the largest |act| over 32767), then the dispatch on the column groups.
 template <int Q8, int GENERIC>
 __device__ __forceinline__ bool ffn_down(const KParams &p, const SmemLayout &s, const Geom &g,
-                                         const TaskDesc &d, uint32_t &kc, int ct, int lane,
+                                         const TaskDesc &d, RingPos &kc, int ct, int lane,
                                          float sc0, float sc1)
 {
     float a = 0.f;
@@ -2074,7 +2116,7 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
     const bool wprof = p.prof != nullptr && lane == 0;
     uint64_t wt_store[2] = {0, 0};
     uint64_t *wt = wprof ? wt_store : nullptr;
-    uint32_t kc = 0;  // chunks consumed
+    RingPos kc{0u, 0, 0u};  // chunks consumed
     int token = -1;
     if (ct == 0 && qb < qe)
         stage_task(s.ctask_a, p.tasks + qb);

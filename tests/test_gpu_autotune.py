@@ -8,6 +8,7 @@ import torch
 import persistent_megakernel_decode_cta_b200 as amk
 from persistent_megakernel_decode_cta_b200 import autotune, build
 import synth_inputs as si
+from parity_helpers import Pair, compare
 
 pytestmark = pytest.mark.gpu
 
@@ -31,11 +32,18 @@ def test_tune_keeps_fastest_passing_schedule():
     fastest = min(ok, key=lambda r: r["us"])
     for k, v in fastest["knobs"].items():
         assert getattr(best, k) == v
-    # the chosen options decode like the default ones
-    dec = amk.Decoder(cfg, w, best)
-    a = dec.step(7, 0)
-    dec.close()
-    dec = amk.Decoder(cfg, w)
-    assert dec.step(7, 0) == a
-    dec.close()
+    # every schedule that passed the gate, the chosen one included, against
+    # the fp64 oracle on the same bytes (the gate itself compares with the
+    # default schedule, since the product has no oracle)
+    for r in ok:
+        pair = Pair(cfg, options=amk.default_options(**r["knobs"]), weights=w)
+        pair.fill_kv(64)
+        g, am, ref, ref_am = pair.step(7, 64)
+        compare(cfg, g, am, ref, ref_am, what=f"tuned knobs {r['knobs']}")
+        del pair
+    pair = Pair(cfg, options=best, weights=w)
+    pair.fill_kv(64)
+    g, am, ref, ref_am = pair.step(7, 64)
+    compare(cfg, g, am, ref, ref_am, what="chosen options")
+    del pair
     torch.cuda.empty_cache()

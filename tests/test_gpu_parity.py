@@ -232,6 +232,26 @@ def test_smol_greedy_32_steps():
     assert checked >= 16
 
 
+@pytest.mark.parametrize("name,prompt_len,n_new", [
+    ("smol135", 128, 32),      # 32 greedy steps at KV context 128 (seeded 128-token prompt)
+    ("tinyllama", 1, 32),      # 32 greedy steps from KV context 0
+    ("llama1b_w8", 1, 32),     # the int8 path over many steps
+])
+def test_greedy_32_steps_full_size(name, prompt_len, n_new):
+    """Greedy generation with the persistent KV cache at full size: the prompt
+    is decoded through the real path (every step compared with the oracle),
+    then n_new greedy steps, each token fed back; logits within the bound at
+    every step and tokens exact wherever the oracle's top-2 margin exceeds
+    it (teacher-forced past a near-tie)."""
+    cfg = si.get_config(name)
+    pair = Pair(cfg)
+    prompt = si.make_prompt(cfg, prompt_len)
+    worst, checked = greedy_teacher_forced(pair, prompt, n_new - 1)
+    assert checked >= (prompt_len + n_new) // 2
+    del pair
+    torch.cuda.empty_cache()
+
+
 def test_bad_arguments():
     cfg = si.get_config("tiny")
     pair = Pair(cfg)
