@@ -400,7 +400,7 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     }
     std::vector<TaskDesc> resolved(P->tasks.size());
     for (size_t t = 0; t < resolved.size(); ++t)
-        amk_resolve_task(P, w, H->d_kv, (int)t, &resolved[t]);
+        amk_resolve_task(P, w, H->d_kv, (int)t, &resolved[t], P->ffn_fused ? 1 : 0);
     // fused FFN: the handle's packed copy of every layer's Wdown
     for (int l = 0; P->ffn_fused && l < L; ++l) {
         const size_t lb = (size_t)c.hidden * c.ffn * (q8 ? 1 : 2);
@@ -420,7 +420,7 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     }
     std::vector<TaskDesc> resolved0(P->pos0 ? P->pos0->tasks.size() : 0);
     for (size_t t = 0; t < resolved0.size(); ++t)
-        amk_resolve_task(P->pos0, w, H->d_kv, (int)t, &resolved0[t]);
+        amk_resolve_task(P->pos0, w, H->d_kv, (int)t, &resolved0[t], P->pos0->ffn_fused ? 1 : 0);
     if (P->pos0 &&
         ((e = cudaMemcpyAsync(H->d_tasks0, resolved0.data(), sizeof(TaskDesc) * resolved0.size(),
                               cudaMemcpyHostToDevice, H->stream)) != cudaSuccess ||
@@ -538,6 +538,8 @@ int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev,
     KParams k = H->kp;
     k.pos = pos;
     k.token = token_id;
+    k.att_chunk = amk::attn_chunk_len(pos + 1, H->plan->opt.attn_splits);
+    k.att_P = H->plan->opt.stage_bytes / (4 * c.head_dim);
     // counter epochs count the steps each schedule ran (parity counts all)
     k.epoch = H->epoch - H->epoch0;
     const bool at0 = pos == 0 && H->plan->pos0;

@@ -73,7 +73,7 @@ enum TaskFlags : uint8_t {
                           // and the task writes its share of KV-cache row 0
 };
 
-struct TaskDesc {           // 80 bytes, read-only for the kernel
+struct TaskDesc {           // 96 bytes, read-only for the kernel
     uint8_t kind, mat, flags, pad;
     int32_t layer;
     int32_t wait_ctr;       // -1: no wait
@@ -87,8 +87,19 @@ struct TaskDesc {           // 80 bytes, read-only for the kernel
     const uint16_t *s0, *s1;  // fp16 row scales at row r0 (W8A16), or null
     const uint16_t *gain;     // RMSNorm gain of the prologue, or null
     const uint16_t *s2;       // TK_FFN: fp16 row scales of Wdown [hidden] (W8A16), or null
+    // ring geometry of a GEMV task (zero for ATTN), computed by the host when it
+    // resolves the task (amk_task_geometry), so that neither the producer nor
+    // the consumers divide by run-time values at a task boundary:
+    uint16_t nchunks;         // ring chunks: the row GEMV's, then a fused FFN's Wdown ones
+    uint16_t ngu;             // chunks of the row GEMV (of all its parts)
+    uint16_t rpc;             // rows per chunk (a multiple of the row groups and of the
+                              //   16-byte granule of the row length)
+    uint16_t nck;             // chunks per part (gate and up are two parts)
+    uint16_t rpc2, nck2;      // fused FFN Wdown: rows per chunk, chunks
+    uint16_t ncb;             // fused FFN Wdown: 16-byte column groups of the slice
+    uint8_t ks_log2, rg_log2; // the 8 consumer warps: 2^ks K-slices x 2^rg row groups
 };
-static_assert(sizeof(TaskDesc) == 80, "TaskDesc is 80 bytes");
+static_assert(sizeof(TaskDesc) == 96, "TaskDesc is 96 bytes (six 16-byte pieces)");
 
 // Per-layer weight pointers (device copies of the caller's pointers).
 struct LayerPtrs {
@@ -150,6 +161,8 @@ struct KParams {
     uint32_t lookahead;         // L2 prefetch distance past the ring copies (bytes), 0 = off
     uint32_t inflight;          // cap on bulk-copy bytes in flight per SM (0xffffffff: none)
     uint32_t piece;             // bytes of a copy piece (multiple of 16)
+    int32_t att_chunk;          // positions per split-K attention chunk at this step
+    int32_t att_P;              // KV positions per ring stage (stage_bytes / (4 head_dim))
     int32_t skip_signal_task;   // test hook, -1 = off
     unsigned long long *prof;   // [n_sms][kProfKinds][kProfFields] phase timers, or null
 };

@@ -377,13 +377,13 @@ __device__ __forceinline__ SmemLayout smem_layout(uint8_t *base, const KParams &
 }
 
 // Copies a task record into a shared-memory slot asynchronously (cp.async,
-// five 16-byte pieces, one commit group), holding no registers; the issuing
+// six 16-byte pieces, one commit group), holding no registers; the issuing
 // thread waits for it with stage_task_wait before anyone reads the slot.
 __device__ __forceinline__ void stage_task(uint32_t slot, const TaskDesc *t)
 {
     const uint8_t *src = reinterpret_cast<const uint8_t *>(t);
 #pragma unroll
-    for (int i = 0; i < 5; ++i)
+    for (int i = 0; i < (int)sizeof(TaskDesc) / 16; ++i)
         asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(slot + 16 * i),
                      "l"(src + 16 * i)
                      : "memory");
@@ -398,7 +398,7 @@ __device__ __forceinline__ TaskDesc read_staged(uint32_t slot)
     TaskDesc d;
     uint4 *dst = reinterpret_cast<uint4 *>(&d);
 #pragma unroll
-    for (int i = 0; i < 5; ++i)
+    for (int i = 0; i < (int)sizeof(TaskDesc) / 16; ++i)
         dst[i] = lds128(slot + 16 * i);
     return d;
 }
@@ -423,89 +423,53 @@ struct Geom {
     // or all of h
     int ncb, rpc2, nck2;
     int VB, KS, RG;  // vector bytes; warps split K into KS slices x RG row groups
+    int ks_log2, rg_log2;
     // attention tiles
     int j0, j1, pa, pb, P;
 };
-
-__device__ __forceinline__ int gcd16(int v)
-{
-    int g = 16;
-    while (v % g)
-        g >>= 1;
-    return g;
-}
 
 __device__ __forceinline__ Geom task_geom(const KParams &p, const TaskDesc &d)
 {
     Geom g{};
     if (d.kind == TK_ATTN) {
-        const int c = d.r1, hd = p.head_dim;
+        const int c = d.r1;
         const int n = p.pos + 1;
-        const int chunk = attn_chunk_len(n, p.attn_splits);
+        const int chunk = p.att_chunk;  // positions per chunk at this step
         g.j0 = c * chunk;
         g.j1 = min(g.j0 + chunk, n);
         if (g.j1 < g.j0)
             g.j1 = g.j0;
         g.pa = g.j0;
         g.pb = max(g.pa, min(g.j1, p.pos));
-        g.P = p.stage_bytes / (4 * hd);
+        g.P = p.att_P;
         g.nchunks = (g.pb - g.pa + g.P - 1) / g.P;
         return g;
     }
-    int K = p.hidden, esz = p.quant ? 1 : 2, parts = 1;
+    // GEMV tiles: the chunk stream and warp layout come with the record
+    // (the host computed them when it resolved the task)
+    int K = p.hidden, esz = p.quant ? 1 : 2;
     if (d.kind == TK_OPROJ)
         K = p.n_heads * p.head_dim;
     else if (d.kind == TK_DOWN)
         K = p.ffn;
-    else if (d.kind == TK_GATEUP || d.kind == TK_FFN)
-        parts = 2;
     else if (d.kind == TK_LMHEAD && p.tied)
         esz = 2;
     g.K = K;
     g.esz = esz;
     g.RB = K * esz;
-    const int gran = 16 / gcd16(g.RB);
-    int rpc = p.stage_bytes / g.RB;
-    rpc -= rpc % gran;
-    // warp layout: each lane keeps at most 64 activations of its K-slice in
-    // registers.  K is split across more warps when a row needs it, and also
-    // while that gives every warp fewer than four rows of a chunk (the GEMV
-    // takes rows four at a time) and still leaves each lane a whole vector
-    g.VB = (g.RB % 16 == 0) ? 16 : ((g.RB % 8 == 0) ? 8 : 4);
-    const int NV = g.RB / g.VB;
-    const int max_vec = 64 / (g.VB / esz);  // vectors a lane may hold
-    const int rows = min(rpc, d.r1 - d.r0);
-    int KS = 1;
-    while (KS < kConsumerWarps) {
-        const int rgk = kConsumerWarps / KS;
-        const bool must = NV > KS * 32 * max_vec || rgk > rpc;
-        const bool more_rows = rgk * 4 > rows && NV >= 2 * KS * 32;
-        if (!must && !more_rows)
-            break;
-        KS *= 2;
-    }
-    g.KS = KS;
-    g.RG = kConsumerWarps / KS;
-    const int step = g.RG > gran ? g.RG : gran;  // rows per chunk: a multiple of both
-    if (rpc >= step)
-        rpc -= rpc % step;
-    g.rpc = rpc;
+    g.VB = (g.RB & 15) == 0 ? 16 : ((g.RB & 7) == 0 ? 8 : 4);
     g.R = d.r1 - d.r0;
-    g.nck = (g.R + rpc - 1) / rpc;
-    g.nchunks = g.nck * parts;
-    g.ngu = g.nchunks;
-    if (d.kind == TK_FFN) {
-        const int row_bytes = g.R * esz, br = p.ffn_box_rows;
-        g.ncb = row_bytes / 16;
-        if (p.dpack) {  // contiguous column groups: any row count per chunk
-            g.rpc2 = min(p.hidden, p.stage_bytes / row_bytes);
-        } else {        // TMA boxes of br rows
-            const int fit = (p.stage_bytes / (row_bytes * br)) * br;  // rows per stage
-            g.rpc2 = fit >= p.hidden ? p.hidden : fit / 256 * 256;
-        }
-        g.nck2 = (p.hidden + g.rpc2 - 1) / g.rpc2;
-        g.nchunks += g.nck2;
-    }
+    g.rpc = d.rpc;
+    g.nck = d.nck;
+    g.ngu = d.ngu;
+    g.nchunks = d.nchunks;
+    g.ncb = d.ncb;
+    g.rpc2 = d.rpc2;
+    g.nck2 = d.nck2;
+    g.ks_log2 = d.ks_log2;
+    g.rg_log2 = d.rg_log2;
+    g.KS = 1 << d.ks_log2;
+    g.RG = 1 << d.rg_log2;
     return g;
 }
 
@@ -535,6 +499,9 @@ __device__ __forceinline__ void lookahead_load(const KParams &p, Lookahead &la)
     const longlong2 w = __ldg(reinterpret_cast<const longlong2 *>(rec + 32));  // w0, w1
     d.r0 = q.z;
     d.r1 = q.w;
+    // the geometry fields (the record's last 16 bytes)
+    const int4 gq = __ldg(reinterpret_cast<const int4 *>(rec + 80));
+    memcpy(reinterpret_cast<uint8_t *>(&d) + 80, &gq, 16);
     const Geom g = task_geom(p, d);
     const uint8_t *w0 = reinterpret_cast<const uint8_t *>(w.x);
     const uint8_t *w1 = reinterpret_cast<const uint8_t *>(w.y);
@@ -924,18 +891,19 @@ __device__ bool wait_counter(const KParams &p, const TaskDesc &d, int ti)
     }
 }
 
-// Block-wide sum over the 256 consumer threads (uses s.scr).
+// Block-wide sum over the 256 consumer threads, through s.scr[16 .. 24),
+// which nothing else uses: one barrier (the next call comes after the
+// caller's own barriers, so the slots are free again by then).
 __device__ float block_sum(float v, const SmemLayout &s, int ct)
 {
     v = warp_sum(v);
     if ((ct & 31) == 0)
-        s.scr[ct >> 5] = v;
+        s.scr[16 + (ct >> 5)] = v;
     consumer_bar();
     float t = 0.f;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w)
-        t += s.scr[w];
-    consumer_bar();
+        t += s.scr[16 + w];
     return t;
 }
 
@@ -1248,13 +1216,13 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
 {
     using LX = LaneX<ESZ, NI>;
     constexpr int E = LX::E;
-    const int NV = g.RB / 16;
-    const int VPS = (NV + g.KS - 1) / g.KS;
+    const int NV = g.RB >> 4;
+    const int VPS = (NV + g.KS - 1) >> g.ks_log2;
     const int RG = g.RG, RB = g.RB, rpc = g.rpc, R = g.R, nck = g.nck;
-    const int rg = warp % RG, ks = warp / RG;
+    const int rg = warp & (RG - 1), ks = warp >> g.rg_log2;
     const int vb = ks * VPS;
     const int ve = min(vb + VPS, NV);
-    const int ni = (ve - vb - lane + 31) / 32;  // vectors this lane holds (may be <= 0)
+    const int ni = (ve - vb - lane + 31) >> 5;  // vectors this lane holds (may be <= 0)
     LX x;
     {
         float xf[NI][E];
@@ -1316,7 +1284,7 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
     const int SB = p.stage_bytes;
     // rows rg + RG m (m < nrw) of a chunk are this warp's: rpc / RG of a full
     // chunk (rpc is a multiple of RG); the last chunk of a part may hold fewer
-    const int nrw_full = rpc / RG;
+    const int nrw_full = rpc >> g.rg_log2;
     uint64_t tA = 0, tB = 0;
     int part = 0, cc = 0;  // chunk c = part * nck + cc, advanced without divisions
     for (int c = 0; c < g.ngu; ++c) {
@@ -1332,7 +1300,7 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
         const int r0 = cc * rpc;
         const int nr = min(rpc, R - r0);
         const int rowbase = part * R + r0;
-        const int nrw = nr == rpc ? nrw_full : nr > rg ? (nr - rg + RG - 1) / RG : 0;
+        const int nrw = nr == rpc ? nrw_full : nr > rg ? (nr - rg + RG - 1) >> g.rg_log2 : 0;
         if (++cc == nck) {
             cc = 0;
             ++part;
@@ -1360,8 +1328,8 @@ __device__ __forceinline__ bool gemv16(const KParams &p, const SmemLayout &s, co
                                        RingPos &kc, int warp, int lane, const float *xg,
                                        uint64_t *wt)
 {
-    const int vps = (g.RB / 16 + g.KS - 1) / g.KS;
-    const int nimax = (vps + 31) / 32;
+    const int vps = ((g.RB >> 4) + g.KS - 1) >> g.ks_log2;
+    const int nimax = (vps + 31) >> 5;
     if constexpr (ESZ == 2) {
         if (nimax <= 2)
             return gemv16_task<2, 2>(p, s, g, kc, warp, lane, xg, wt);
@@ -1414,7 +1382,8 @@ __device__ __forceinline__ bool run_gemv(const KParams &p, const SmemLayout &s, 
 // included): the warps rg + RG * ks with rg = (row within its chunk) % RG.
 __device__ __forceinline__ float row_total(const SmemLayout &s, const Geom &g, int t)
 {
-    const int rg = (t % g.R) % g.RG;  // chunks start at multiples of RG
+    const int tr = t >= g.R ? t - g.R : t;  // the row within its part (at most two parts)
+    const int rg = tr & (g.RG - 1);          // chunks start at multiples of RG
     float y = 0.f;
     for (int ks = 0; ks < g.KS; ++ks)
         y += s.red[(rg + g.RG * ks) * kMaxTaskRows + t];
@@ -1831,7 +1800,7 @@ __device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
         return false;
     const int l = d.layer, gi = d.r0, C = p.attn_splits;
     const int n = p.pos + 1;
-    const int chunk = attn_chunk_len(n, C);
+    const int chunk = p.att_chunk;
     const int nne = (n + chunk - 1) / chunk;  // non-empty chunks: 0 .. nne-1
     if (nne == 1 || g.j1 <= g.j0)
         return true;  // written directly, or empty

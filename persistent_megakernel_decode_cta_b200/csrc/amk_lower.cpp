@@ -532,8 +532,78 @@ void amk_plan_view(const amk_plan *P, amk_graph *g)
     g->queue_tasks = P->gqueue.data();
 }
 
+void amk_task_geometry(const amk_plan *P, amk::TaskDesc *dp, int packed_down)
+{
+    amk::TaskDesc &d = *dp;
+    d.nchunks = d.ngu = d.rpc = d.nck = d.rpc2 = d.nck2 = d.ncb = 0;
+    d.ks_log2 = d.rg_log2 = 0;
+    if (d.kind == amk::TK_ATTN)
+        return;
+    const amk_config &c = P->cfg;
+    const int stage = P->opt.stage_bytes;
+    constexpr int W = amk::kConsumerWarps;
+    int K = c.hidden, esz = c.quant == AMK_QUANT_W8A16 ? 1 : 2, parts = 1;
+    if (d.kind == amk::TK_OPROJ)
+        K = c.n_heads * c.head_dim;
+    else if (d.kind == amk::TK_DOWN)
+        K = c.ffn;
+    else if (d.kind == amk::TK_GATEUP || d.kind == amk::TK_FFN)
+        parts = 2;
+    else if (d.kind == amk::TK_LMHEAD && c.tied_embeddings)
+        esz = 2;
+    const int RB = K * esz, R = d.r1 - d.r0;
+    const int gran = gran_rows(RB);
+    int rpc = stage / RB;
+    rpc -= rpc % gran;
+    // warp layout: each lane keeps at most 64 activations of its K-slice in
+    // registers.  K is split across more warps when a row needs it, and also
+    // while that gives every warp fewer than four rows of a chunk (the GEMV
+    // takes rows four at a time) and still leaves each lane a whole vector
+    const int VB = (RB % 16 == 0) ? 16 : ((RB % 8 == 0) ? 8 : 4);
+    const int NV = RB / VB;
+    const int max_vec = 64 / (VB / esz);
+    const int rows = std::min(rpc, R);
+    int KS = 1, ks_log2 = 0;
+    while (KS < W) {
+        const int rgk = W / KS;
+        const bool must = NV > KS * 32 * max_vec || rgk > rpc;
+        const bool more_rows = rgk * 4 > rows && NV >= 2 * KS * 32;
+        if (!must && !more_rows)
+            break;
+        KS *= 2;
+        ++ks_log2;
+    }
+    const int RG = W / KS;
+    const int step = std::max(RG, gran);  // rows per chunk: a multiple of both
+    if (rpc >= step)
+        rpc -= rpc % step;
+    const int nck = (R + rpc - 1) / rpc;
+    int nchunks = nck * parts;
+    d.ngu = (uint16_t)nchunks;
+    if (d.kind == amk::TK_FFN) {
+        const int row_bytes = R * esz, br = P->ffn_box_rows;
+        int rpc2;
+        if (packed_down) {  // contiguous column groups: any row count per chunk
+            rpc2 = std::min(c.hidden, stage / row_bytes);
+        } else {            // TMA boxes of br rows
+            const int fit = (stage / (row_bytes * br)) * br;  // rows per stage
+            rpc2 = fit >= c.hidden ? c.hidden : fit / 256 * 256;
+        }
+        d.ncb = (uint16_t)(row_bytes / 16);
+        d.rpc2 = (uint16_t)rpc2;
+        d.nck2 = (uint16_t)((c.hidden + rpc2 - 1) / rpc2);
+        nchunks += d.nck2;
+    }
+    d.nchunks = (uint16_t)nchunks;
+    d.rpc = (uint16_t)rpc;
+    d.nck = (uint16_t)nck;
+    d.ks_log2 = (uint8_t)ks_log2;
+    d.rg_log2 = (uint8_t)(3 - ks_log2);
+    static_assert(amk::kConsumerWarps == 8, "the row-group log assumes 8 consumer warps");
+}
+
 void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *kv, int t,
-                      amk::TaskDesc *out)
+                      amk::TaskDesc *out, int packed_down)
 {
     const amk_config &c = P->cfg;
     amk::TaskDesc d = P->tasks[t];
@@ -595,6 +665,7 @@ void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *k
         break;
     }
     }
+    amk_task_geometry(P, &d, packed_down);
     *out = d;
 }
 

@@ -175,7 +175,7 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     for (int t0 = 0; t0 < T; t0 += 64) {
         const int n = T - t0 < 64 ? T - t0 : 64;
         for (int i = 0; i < n; ++i)
-            amk_resolve_task(&P, w, kv, t0 + i, &batch[i]);
+            amk_resolve_task(&P, w, kv, t0 + i, &batch[i], 0);
         e = cudaMemcpyAsync(base + lay.tasks + sizeof(amk::TaskDesc) * (size_t)t0, batch,
                             sizeof(amk::TaskDesc) * (size_t)n, cudaMemcpyHostToDevice, st);
         if (e != cudaSuccess)
@@ -246,6 +246,8 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     k.generic = P.generic;
     k.pos = pos;
     k.token = token_id;
+    k.att_chunk = amk::attn_chunk_len(pos + 1, P.opt.attn_splits);
+    k.att_P = P.opt.stage_bytes / (4 * c.head_dim);
     k.epoch = 0;   // counters were cleared above
     k.arrive_base = 0;
     k.parity = 0;

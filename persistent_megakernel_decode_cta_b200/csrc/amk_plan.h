@@ -68,8 +68,14 @@ int amk_encode_down_maps(const amk_plan *P, const amk_weights *w, int l0, int n,
 
 // Copies plan task t into *out with its device pointers resolved: weight
 // rows, row scales and norm gain from w, KV-cache blocks from kv (bf16
-// [L][2][nkv][max_ctx][hd]).  Host only; reads only host memory.
+// [L][2][nkv][max_ctx][hd]), and its ring geometry (amk_task_geometry).
+// packed_down: the handle keeps a packed copy of every Wdown (fused FFN
+// slices then stream contiguous column groups; else 2-D tensor-map boxes).
+// Host only; reads only host memory.
 void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *kv, int t,
-                      amk::TaskDesc *out);
+                      amk::TaskDesc *out, int packed_down);
+// The ring geometry of GEMV task d of plan P (the chunk stream its producer
+// issues and the warp layout of its consumers); attention tasks get zeros.
+void amk_task_geometry(const amk_plan *P, amk::TaskDesc *d, int packed_down);
 
 #endif
