@@ -54,6 +54,8 @@ WORKLOADS = {
     "tinyllama-ctx1024": ("tinyllama", 1024),
     "llama1b_w8-ctx0": ("llama1b_w8", 0),
     "llama1b_w8-ctx512": ("llama1b_w8", 512),
+    "smol135_w4-ctx0": ("smol135_w4", 0),
+    "llama7b_w4-ctx2048": ("llama7b_w4", 2048),
     "smol135-ctx0": ("smol135", 0),
     "smol135-ctx128": ("smol135", 128),
     "tiny-ctx4": ("tiny", 4),
@@ -364,7 +366,7 @@ def run_ours(args):
         us, n, threads, ref = oracle_steps(cfg, w, ctx, kv, budget, 64)
         scale = float(np.abs(ref).max())
         err = float(np.abs(g - ref).max())
-        tol = (2e-2 if cfg.quant == "w8a16" else 1e-2) * scale
+        tol = (2e-2 if cfg.quant in ("w8a16", "w4a16") else 1e-2) * scale
         parity = {"verdict": "PASS" if err <= tol else "FAIL", "max_abs_dlogit": err,
                   "tolerance": tol, "max_abs_logit": scale,
                   "argmax_match": int(np.argmax(g)) == int(np.argmax(ref))}
@@ -454,8 +456,10 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": ("int8 weights x int16 activations, i32 then f32 accumulate"
-                      if cfg.quant == "w8a16" else "bf16 weights x f32 activations, f32 accumulate"),
+            "dtype": {"w8a16": "int8 weights x int16 activations, i32 then f32 accumulate",
+                      "w4a16": "int4 weights (fp16 group scales) x int16 activations, "
+                               "i32 then f32 accumulate"}.get(
+                          cfg.quant, "bf16 weights x f32 activations, f32 accumulate"),
             "data": "synthetic (seeded random-init weights and KV cache)",
             "config": dict(workload_config(name, cfg, ctx),
                            parallelism=f"replicas{world}" if world > 1 else "single"),

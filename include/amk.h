@@ -62,7 +62,7 @@ typedef enum {
 } amk_status;
 
 /* ---- model description ---------------------------------------------------- */
-typedef enum { AMK_QUANT_BF16 = 0, AMK_QUANT_W8A16 = 1 } amk_quant;
+typedef enum { AMK_QUANT_BF16 = 0, AMK_QUANT_W8A16 = 1, AMK_QUANT_W4A16 = 2 } amk_quant;
 
 /* Shapes of a Llama-family decoder (no biases).  head_dim must be even,
  * n_heads a multiple of n_kv_heads.  max_ctx = number of KV-cache rows the
@@ -80,20 +80,26 @@ typedef struct {
  * device pointers.  The embedding, norm gains and a tied head are always
  * bf16.  With AMK_QUANT_W8A16 the linear weights (and an untied LM head) are
  * int8 with one fp16 scale per output row: w_jk = scale_j * q_jk (README,
- * results section: W8A16 per-output-channel int8).  Scale arrays are ignored
- * for bf16. */
+ * results section: W8A16 per-output-channel int8).  With AMK_QUANT_W4A16
+ * (gist.science summary, "Belangrijkste Bijdragen": int4 weight-only) they
+ * are packed int4, [out][in / 2] bytes, input 2i in the low nibble of byte i
+ * (4-bit two's complement), with one fp16 scale per 128 inputs of a row:
+ * scales [out][ceil(in / 128)], w_jk = scale_j,k/128 * q_jk; every in must be
+ * a multiple of 32.  amk_create packs each int4 matrix once into a copy the
+ * handle owns (codes and scales of a row together); the caller's arrays are
+ * not read by decode steps.  Scale arrays are ignored for bf16. */
 typedef struct {
     const void *embed;         /* bf16 [vocab][hidden] */
     const void *final_norm;    /* bf16 [hidden] */
-    const void *lm_head;       /* bf16|int8 [vocab][hidden]; NULL when tied */
-    const void *lm_head_scale; /* fp16 [vocab] (W8A16, untied) */
+    const void *lm_head;       /* bf16|int8|int4 [vocab][hidden]; NULL when tied */
+    const void *lm_head_scale; /* fp16 [vocab] (W8A16) or [vocab][hidden/128] (W4A16), untied */
     const void *const *attn_norm, *const *ffn_norm;  /* bf16 [hidden] */
     const void *const *wq;     /* [n_heads*head_dim][hidden] */
     const void *const *wk, *const *wv; /* [n_kv_heads*head_dim][hidden] */
     const void *const *wo;     /* [hidden][n_heads*head_dim] */
     const void *const *wgate, *const *wup; /* [ffn][hidden] */
     const void *const *wdown;  /* [hidden][ffn] */
-    const void *const *sq, *const *sk, *const *sv, *const *so; /* fp16 [rows] */
+    const void *const *sq, *const *sk, *const *sv, *const *so; /* fp16 [rows] or [rows][groups] */
     const void *const *sgate, *const *sup, *const *sdown;
 } amk_weights;
 

@@ -51,7 +51,8 @@ def make_config(cfg) -> abi.Config:
     c.rms_eps = float(cfg.rms_eps)
     c.rope_theta = float(cfg.rope_theta)
     c.tied_embeddings = 1 if cfg.tied else 0
-    quant = {"bf16": abi.QUANT_BF16, "w8a16": abi.QUANT_W8A16}.get(cfg.quant)
+    quant = {"bf16": abi.QUANT_BF16, "w8a16": abi.QUANT_W8A16,
+             "w4a16": abi.QUANT_W4A16}.get(cfg.quant)
     if quant is None:
         raise AmkError(abi.ERR["AMK_ERR_UNSUPPORTED"],
                        f"no kernel for weight format {cfg.quant!r}")

@@ -20,7 +20,7 @@ STATUS = {
     -9: "AMK_ERR_POISONED", -10: "AMK_ERR_NO_DEVICE",
 }
 ERR = {v: k for k, v in STATUS.items()}
-QUANT_BF16, QUANT_W8A16 = 0, 1
+QUANT_BF16, QUANT_W8A16, QUANT_W4A16 = 0, 1, 2
 ACC_READ, ACC_WRITE, ACC_ACCUM, ACC_READ_PREV, ACC_RESET = range(5)
 BUF_OUTPUT = 1
 RULES = {0: "ok", 1: "V1", 2: "V2", 3: "V3", 4: "V4", 5: "V5", 6: "V6", 7: "V7",

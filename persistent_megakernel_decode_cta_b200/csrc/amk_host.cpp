@@ -28,6 +28,8 @@ extern "C" cudaError_t amk_kernel_configure(int smem_bytes, int quant, int att_e
                                             int fused);
 extern "C" cudaError_t amk_pack_down(const void *wd, void *out, int h, int ffn, int esz,
                                      cudaStream_t stream);
+extern "C" cudaError_t amk_pack_q4(const void *codes, const void *scales, void *out, int rows,
+                                   int K, cudaStream_t stream);
 extern "C" cudaError_t amk_kernel_occupancy(int smem_bytes, int quant, int att_e, int generic,
                                             int fused, int *blocks_per_sm);
 namespace amk {
@@ -170,6 +172,7 @@ struct amk_handle {
     long long *d_xacc = nullptr;    // [L][h] fixed-point residual (fused FFN)
     void *d_act_block = nullptr;    // every activation buffer, one allocation
     void *d_dpack = nullptr;        // [L] packed Wdown (fused FFN), see KParams::dpack
+    void *d_q4 = nullptr;           // W4A16: every int4 matrix as rows of codes + scales
     unsigned long long *d_prof = nullptr;
     uint16_t *d_kv = nullptr;
     size_t kv_bytes = 0, act_bytes = 0;
@@ -231,8 +234,8 @@ int check_weights(const amk_config *c, const amk_weights *w)
     if (!c->tied_embeddings) {
         if (!aligned16(w->lm_head))
             return amk_set_error(AMK_ERR_INVALID_ARG, "lm_head NULL or not 16-byte aligned");
-        if (c->quant == AMK_QUANT_W8A16 && !w->lm_head_scale)
-            return amk_set_error(AMK_ERR_INVALID_ARG, "lm_head_scale NULL for W8A16");
+        if (c->quant != AMK_QUANT_BF16 && !w->lm_head_scale)
+            return amk_set_error(AMK_ERR_INVALID_ARG, "lm_head_scale NULL for int8/int4 weights");
     }
     const void *const *mats[7] = {w->wq, w->wk, w->wv, w->wo, w->wgate, w->wup, w->wdown};
     const void *const *scs[7] = {w->sq, w->sk, w->sv, w->so, w->sgate, w->sup, w->sdown};
@@ -241,7 +244,7 @@ int check_weights(const amk_config *c, const amk_weights *w)
     for (int m = 0; m < 7; ++m) {
         if (!mats[m])
             return amk_set_error(AMK_ERR_INVALID_ARG, "weight pointer array %d NULL", m);
-        if (c->quant == AMK_QUANT_W8A16 && !scs[m])
+        if (c->quant != AMK_QUANT_BF16 && !scs[m])
             return amk_set_error(AMK_ERR_INVALID_ARG, "scale pointer array %d NULL", m);
     }
     for (int l = 0; l < c->n_layers; ++l) {
@@ -251,7 +254,7 @@ int check_weights(const amk_config *c, const amk_weights *w)
             if (!aligned16(mats[m][l]))
                 return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d weight %d NULL or not "
                                      "16-byte aligned", l, m);
-            if (c->quant == AMK_QUANT_W8A16 && !scs[m][l])
+            if (c->quant != AMK_QUANT_BF16 && !scs[m][l])
                 return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d scale %d NULL", l, m);
         }
     }
@@ -341,13 +344,14 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     }
     const amk_plan *P = H->plan;
     const int q8 = P->cfg.quant == AMK_QUANT_W8A16 ? 1 : 0;
-    cudaError_t e = amk_kernel_configure(P->smem_bytes, q8, P->att_e, P->generic, P->ffn_fused);
+    const int qm = P->cfg.quant;  // 0 bf16, 1 int8, 2 int4
+    cudaError_t e = amk_kernel_configure(P->smem_bytes, qm, P->att_e, P->generic, P->ffn_fused);
     if (e != cudaSuccess) {
         free_handle(H);
         return cuda_fail(e, "cudaFuncSetAttribute");
     }
     int per_sm = 0;
-    e = amk_kernel_occupancy(P->smem_bytes, q8, P->att_e, P->generic, P->ffn_fused, &per_sm);
+    e = amk_kernel_occupancy(P->smem_bytes, qm, P->att_e, P->generic, P->ffn_fused, &per_sm);
     if (e != cudaSuccess || per_sm < 1) {
         free_handle(H);
         return amk_set_error(AMK_ERR_LAUNCH, "kernel does not fit one SM (smem %d B)",
@@ -398,9 +402,56 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
         free_handle(H);
         return cuda_fail(e, "host buffers");
     }
+    // W4A16: pack every int4 matrix (codes and group scales of a row together)
+    // into one allocation, and resolve the tasks against the packed copies
+    amk_weights wq4 = *w;
+    std::vector<const void *> q4_ptrs;
+    if (qm == AMK_QUANT_W4A16) {
+        const int hh = c.hidden, qr = c.n_heads * c.head_dim, kr = c.n_kv_heads * c.head_dim;
+        const int F = c.ffn;
+        const int rows7[7] = {qr, kr, kr, hh, F, F, hh};
+        const int ks7[7] = {hh, hh, hh, qr, hh, hh, F};
+        const void *const *mats[7] = {w->wq, w->wk, w->wv, w->wo, w->wgate, w->wup, w->wdown};
+        const void *const *scs[7] = {w->sq, w->sk, w->sv, w->so, w->sgate, w->sup, w->sdown};
+        size_t total = 0;
+        for (int m = 0; m < 7; ++m)
+            total += (size_t)L * rows7[m] * amk::q4_row_bytes(ks7[m]);
+        if (!c.tied_embeddings)
+            total += (size_t)c.vocab * amk::q4_row_bytes(hh);
+        if ((rc = dalloc(H, &H->d_q4, total))) {
+            free_handle(H);
+            return rc;
+        }
+        q4_ptrs.resize((size_t)7 * L);
+        uint8_t *dst = static_cast<uint8_t *>(H->d_q4);
+        for (int m = 0; m < 7; ++m)
+            for (int l = 0; l < L; ++l) {
+                if ((e = amk_pack_q4(mats[m][l], scs[m][l], dst, rows7[m], ks7[m], H->stream)) !=
+                    cudaSuccess) {
+                    free_handle(H);
+                    return cuda_fail(e, "pack int4 weights");
+                }
+                q4_ptrs[(size_t)m * L + l] = dst;
+                dst += (size_t)rows7[m] * amk::q4_row_bytes(ks7[m]);
+            }
+        if (!c.tied_embeddings) {
+            if ((e = amk_pack_q4(w->lm_head, w->lm_head_scale, dst, c.vocab, hh, H->stream)) !=
+                cudaSuccess) {
+                free_handle(H);
+                return cuda_fail(e, "pack int4 LM head");
+            }
+            wq4.lm_head = dst;
+        }
+        const void *const *packed[7];
+        for (int m = 0; m < 7; ++m)
+            packed[m] = q4_ptrs.data() + (size_t)m * L;
+        wq4.wq = packed[0], wq4.wk = packed[1], wq4.wv = packed[2], wq4.wo = packed[3];
+        wq4.wgate = packed[4], wq4.wup = packed[5], wq4.wdown = packed[6];
+    }
+    const amk_weights *wr = qm == AMK_QUANT_W4A16 ? &wq4 : w;
     std::vector<TaskDesc> resolved(P->tasks.size());
     for (size_t t = 0; t < resolved.size(); ++t)
-        amk_resolve_task(P, w, H->d_kv, (int)t, &resolved[t], P->ffn_fused ? 1 : 0);
+        amk_resolve_task(P, wr, H->d_kv, (int)t, &resolved[t], P->ffn_fused ? 1 : 0);
     // fused FFN: the handle's packed copy of every layer's Wdown
     for (int l = 0; P->ffn_fused && l < L; ++l) {
         const size_t lb = (size_t)c.hidden * c.ffn * (q8 ? 1 : 2);
@@ -420,7 +471,7 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     }
     std::vector<TaskDesc> resolved0(P->pos0 ? P->pos0->tasks.size() : 0);
     for (size_t t = 0; t < resolved0.size(); ++t)
-        amk_resolve_task(P->pos0, w, H->d_kv, (int)t, &resolved0[t], P->pos0->ffn_fused ? 1 : 0);
+        amk_resolve_task(P->pos0, wr, H->d_kv, (int)t, &resolved0[t], P->pos0->ffn_fused ? 1 : 0);
     if (P->pos0 &&
         ((e = cudaMemcpyAsync(H->d_tasks0, resolved0.data(), sizeof(TaskDesc) * resolved0.size(),
                               cudaMemcpyHostToDevice, H->stream)) != cudaSuccess ||
@@ -470,7 +521,7 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     k.qkv_rows = P->qkv_rows;
     k.group = P->group;
     k.attn_splits = P->opt.attn_splits;
-    k.quant = q8;
+    k.quant = qm;
     k.tied = c.tied_embeddings ? 1 : 0;
     k.rms_eps = c.rms_eps;
     k.rope_theta = c.rope_theta;

@@ -40,6 +40,15 @@ constexpr int kMaxTaskRows = 256;   // output rows of one GEMV task (red buffer)
 // positions, but at least kMinAttnChunk, so that short contexts use fewer,
 // longer chunks (the kernel and the host's arrival count both use this).
 constexpr int kMinAttnChunk = 32;
+// W4A16 weights: inputs per fp16 scale, and the bytes of one packed row of K
+// inputs as the ring streams it: K / 2 code bytes (input 2i in the low nibble
+// of byte i, 4-bit two's complement), then the row's ceil(K / 128) scales,
+// zero-padded to a multiple of 16 bytes.
+constexpr int kQ4Group = 128;
+inline __host__ __device__ int q4_row_bytes(int K)
+{
+    return (K / 2 + 2 * ((K + kQ4Group - 1) / kQ4Group) + 15) & ~15;
+}
 inline __host__ __device__ int attn_chunk_len(int n, int splits)
 {
     const int c = (n + splits - 1) / splits;

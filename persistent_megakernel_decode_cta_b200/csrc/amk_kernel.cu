@@ -14,6 +14,7 @@ const void *amk_kernel_q0_f0(int e);
 const void *amk_kernel_q0_f1(int e);
 const void *amk_kernel_q1_f0(int e);
 const void *amk_kernel_q1_f1(int e);
+const void *amk_kernel_q2_f0(int e);
 const void *amk_kernel_generic();
 
 // Wdown of one layer, [hidden][ffn] row-major, re-laid once per handle as
@@ -45,6 +46,8 @@ const void *kernel_for(int quant, int att_e, int generic, int fused)
     int e = 0;
     while (e < 4 && (1 << e) < att_e)
         ++e;
+    if (quant == 2)  // int4 models never take the fused FFN level
+        return amk_kernel_q2_f0(e);
     if (quant)
         return fused ? amk_kernel_q1_f1(e) : amk_kernel_q1_f0(e);
     return fused ? amk_kernel_q0_f1(e) : amk_kernel_q0_f0(e);
@@ -72,6 +75,35 @@ extern "C" cudaError_t amk_pack_down(const void *wd, void *out, int h, int ffn, 
     const size_t n = (size_t)h * ncg;
     amk_pack_down_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
         static_cast<const uint4 *>(wd), static_cast<uint4 *>(out), h, ncg);
+    return cudaGetLastError();
+}
+
+// An int4 matrix [rows][K / 2] with fp16 scales [rows][ceil(K / 128)], re-laid
+// once per handle as rows of q4_row_bytes(K): the codes, the scales, zeros.
+// One thread per 16-bit unit of the output (K / 2 is a multiple of 16).
+__global__ void amk_pack_q4_kernel(const uint16_t *codes, const uint16_t *scales, uint16_t *out,
+                                   int rows, int K)
+{
+    const int U = q4_row_bytes(K) / 2, cu = K / 4, ng = (K + kQ4Group - 1) / kQ4Group;
+    const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (size_t)rows * U)
+        return;
+    const int row = (int)(idx / U), u = (int)(idx % U);
+    uint16_t v = 0;
+    if (u < cu)
+        v = codes[(size_t)row * cu + u];
+    else if (u < cu + ng)
+        v = scales[(size_t)row * ng + (u - cu)];
+    out[idx] = v;
+}
+
+extern "C" cudaError_t amk_pack_q4(const void *codes, const void *scales, void *out, int rows,
+                                   int K, cudaStream_t stream)
+{
+    const size_t n = (size_t)rows * (q4_row_bytes(K) / 2);
+    amk_pack_q4_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
+        static_cast<const uint16_t *>(codes), static_cast<const uint16_t *>(scales),
+        static_cast<uint16_t *>(out), rows, K);
     return cudaGetLastError();
 }
 

@@ -447,7 +447,8 @@ __device__ __forceinline__ Geom task_geom(const KParams &p, const TaskDesc &d)
     }
     // GEMV tiles: the chunk stream and warp layout come with the record
     // (the host computed them when it resolved the task)
-    int K = p.hidden, esz = p.quant ? 1 : 2;
+    // bytes per weight: 2 (bf16), 1 (int8), 0 (packed int4 rows with their scales)
+    int K = p.hidden, esz = p.quant == 1 ? 1 : p.quant == 2 ? 0 : 2;
     if (d.kind == TK_OPROJ)
         K = p.n_heads * p.head_dim;
     else if (d.kind == TK_DOWN)
@@ -456,7 +457,7 @@ __device__ __forceinline__ Geom task_geom(const KParams &p, const TaskDesc &d)
         esz = 2;
     g.K = K;
     g.esz = esz;
-    g.RB = K * esz;
+    g.RB = esz ? K * esz : q4_row_bytes(K);
     g.VB = (g.RB & 15) == 0 ? 16 : ((g.RB & 7) == 0 ? 8 : 4);
     g.R = d.r1 - d.r0;
     g.rpc = d.rpc;
@@ -1118,14 +1119,39 @@ __device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c)
 // a step = max|x| / 65534 per element) and packs them in pairs, q[i][k] =
 // elements 2k, 2k + 1 of vector i; the int8 x int16 products then add up
 // exactly in int32 (a lane's sum stays below 64 * 127 * 32767 < 2^31).
+//
+// Packed int4 weights (ESZ = 0): 32 codes per vector.  The activations are
+// quantised the same way and packed in the order the nibble split of
+// gemv_rows needs: for the 8 elements 8k .. 8k + 7 of a vector, q[i][4k ..
+// 4k + 3] = (0, 2), (4, 6), (1, 3), (5, 7); xs[i] = 8 x the sum of the
+// vector's int16 activations (the bias the offset codes carry).
 template <int ESZ, int NI_>
 struct LaneX {
-    static constexpr int E = 16 / ESZ;   // elements per vector
+    static constexpr int E = ESZ ? 16 / ESZ : 32;  // elements per vector
     static constexpr int NI = NI_;       // vectors per lane at most (NI E <= 64 activations)
     float f[ESZ == 2 ? NI : 1][ESZ == 2 ? E : 1];
-    uint32_t q[ESZ == 1 ? NI : 1][8];
-    float scale;                         // int8: value of one int16 step
+    uint32_t q[ESZ == 2 ? 1 : NI][ESZ == 0 ? 16 : 8];
+    int xs[ESZ == 0 ? NI : 1];
+    float scale;                         // int8 / int4: value of one int16 step
 };
+
+// int16 pairs of a times unsigned bytes 0, 1 (lo) or 2, 3 (hi) of b.
+__device__ __forceinline__ int dp2a_lo_u(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ int dp2a_hi_u(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t pack_i16(int a, int b)
+{
+    return ((uint32_t)a & 0xffffu) | ((uint32_t)b << 16);
+}
 
 // Rows j0 + RG r (r < RW) of a ring chunk against the lane's activations;
 // each row's warp total goes to red[rowbase + row] (the warp's red slice).
@@ -1135,15 +1161,54 @@ struct LaneX {
 // that the compiler can issue the loads of all RW rows ahead of the math.
 template <int ESZ, int NI, int RW>
 __device__ __forceinline__ void gemv_rows(const LaneX<ESZ, NI> &x, uint32_t stage_a,
-                                          const uint32_t (&voff)[NI], int RB, int RG, int j0,
-                                          uint32_t red_a, int rowbase, int lane)
+                                          const uint32_t (&voff)[NI], const uint32_t (&soff)[NI],
+                                          int RB, int RG, int j0, uint32_t red_a, int rowbase,
+                                          int lane)
 {
     float sr[RW];
     uint32_t ra[RW];
 #pragma unroll
     for (int r = 0; r < RW; ++r)
         ra[r] = stage_a + (uint32_t)((j0 + r * RG) * RB);
-    if constexpr (ESZ == 2) {
+    if constexpr (ESZ == 0) {
+        // int4: XOR 0x8 per nibble turns 4-bit two's complement into code + 8;
+        // even and odd codes as unsigned bytes, dp2a against the int16 pairs,
+        // minus the bias, exact in int32 (|sum| < 32 * 15 * 32767); then the
+        // vector's group scale (at byte soff[i] of the row) in fp32
+        float acc[RW][2];
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+            acc[r][0] = acc[r][1] = 0.f;
+#pragma unroll
+        for (int i = 0; i < NI; ++i) {
+            uint4 w[RW];
+            float sc[RW];
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                w[r] = lds128(ra[r] + voff[i]);
+                sc[r] = fp16_to_f((uint16_t)lds16(ra[r] + soff[i]));
+            }
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                const uint32_t A[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+                int s0 = 0, s1 = 0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t t = A[q] ^ 0x88888888u;
+                    const uint32_t lo = t & 0x0f0f0f0fu;
+                    const uint32_t hi = (t >> 4) & 0x0f0f0f0fu;
+                    s0 = dp2a_lo_u(x.q[i][4 * q], lo, s0);
+                    s1 = dp2a_hi_u(x.q[i][4 * q + 1], lo, s1);
+                    s0 = dp2a_lo_u(x.q[i][4 * q + 2], hi, s0);
+                    s1 = dp2a_hi_u(x.q[i][4 * q + 3], hi, s1);
+                }
+                acc[r][i & 1] = fmaf((float)(s0 + s1 - x.xs[i]), sc[r], acc[r][i & 1]);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+            sr[r] = (acc[r][0] + acc[r][1]) * x.scale;
+    } else if constexpr (ESZ == 2) {
         float acc[RW][4];
 #pragma unroll
         for (int r = 0; r < RW; ++r)
@@ -1216,7 +1281,7 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
 {
     using LX = LaneX<ESZ, NI>;
     constexpr int E = LX::E;
-    const int NV = g.RB >> 4;
+    const int NV = ESZ ? g.RB >> 4 : g.K >> 5;  // int4 rows: code vectors, then the scales
     const int VPS = (NV + g.KS - 1) >> g.ks_log2;
     const int RG = g.RG, RB = g.RB, rpc = g.rpc, R = g.R, nck = g.nck;
     const int rg = warp & (RG - 1), ks = warp >> g.rg_log2;
@@ -1254,6 +1319,33 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
                 for (int e = 0; e < E; ++e)
                     x.f[i][e] = xf[i][e];
             x.scale = 1.f;
+        } else if constexpr (ESZ == 0) {
+            float amax = 0.f;
+#pragma unroll
+            for (int i = 0; i < NI; ++i)
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    amax = fmaxf(amax, fabsf(xf[i][e]));
+            const float inv = amax > 0.f ? 32767.f / amax : 0.f;
+            x.scale = amax * (1.f / 32767.f);
+#pragma unroll
+            for (int i = 0; i < NI; ++i) {
+                int sum = 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    int v[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        v[e] = max(-32767, min(32767, __float2int_rn(xf[i][8 * k + e] * inv)));
+                        sum += v[e];
+                    }
+                    x.q[i][4 * k] = pack_i16(v[0], v[2]);
+                    x.q[i][4 * k + 1] = pack_i16(v[4], v[6]);
+                    x.q[i][4 * k + 2] = pack_i16(v[1], v[3]);
+                    x.q[i][4 * k + 3] = pack_i16(v[5], v[7]);
+                }
+                x.xs[i] = 8 * sum;
+            }
         } else {
             float amax = 0.f;
 #pragma unroll
@@ -1275,11 +1367,15 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
     }
     // byte offset in a row of the lane's vector i: its own while i < ni,
     // else (zero activations) one that the slice surely holds
-    uint32_t voff[NI];
+    // (int4 rows: the vector's group scale is at soff[i], after the K / 2
+    // code bytes of the row, one fp16 per 128 inputs = 4 vectors)
+    uint32_t voff[NI], soff[NI];
 #pragma unroll
-    for (int i = 0; i < NI; ++i)
-        voff[i] = (uint32_t)(i < ni ? vb + lane + 32 * i : ni > 0 ? vb + lane : min(vb, NV - 1)) *
-                  16;
+    for (int i = 0; i < NI; ++i) {
+        const int v = i < ni ? vb + lane + 32 * i : ni > 0 ? vb + lane : min(vb, NV - 1);
+        voff[i] = (uint32_t)v * 16;
+        soff[i] = ESZ ? 0u : (uint32_t)(g.K / 2 + 2 * (v >> 2));
+    }
     const uint32_t red_a = s.red_a + (uint32_t)warp * kMaxTaskRows * 4;
     const int SB = p.stage_bytes;
     // rows rg + RG m (m < nrw) of a chunk are this warp's: rpc / RG of a full
@@ -1307,13 +1403,16 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
         }
         int m = 0;
         for (; m + 4 <= nrw; m += 4)
-            gemv_rows<ESZ, NI, 4>(x, stage_a, voff, RB, RG, rg + RG * m, red_a, rowbase, lane);
+            gemv_rows<ESZ, NI, 4>(x, stage_a, voff, soff, RB, RG, rg + RG * m, red_a, rowbase,
+                                  lane);
         if (m + 2 <= nrw) {
-            gemv_rows<ESZ, NI, 2>(x, stage_a, voff, RB, RG, rg + RG * m, red_a, rowbase, lane);
+            gemv_rows<ESZ, NI, 2>(x, stage_a, voff, soff, RB, RG, rg + RG * m, red_a, rowbase,
+                                  lane);
             m += 2;
         }
         if (m < nrw)
-            gemv_rows<ESZ, NI, 1>(x, stage_a, voff, RB, RG, rg + RG * m, red_a, rowbase, lane);
+            gemv_rows<ESZ, NI, 1>(x, stage_a, voff, soff, RB, RG, rg + RG * m, red_a, rowbase,
+                                  lane);
         release_stage(p, s, kc, lane);
         kc.advance(p.ring_stages);
         if (wt)
@@ -1328,9 +1427,13 @@ __device__ __forceinline__ bool gemv16(const KParams &p, const SmemLayout &s, co
                                        RingPos &kc, int warp, int lane, const float *xg,
                                        uint64_t *wt)
 {
-    const int vps = ((g.RB >> 4) + g.KS - 1) >> g.ks_log2;
+    const int vps = ((ESZ ? g.RB >> 4 : g.K >> 5) + g.KS - 1) >> g.ks_log2;
     const int nimax = (vps + 31) >> 5;
-    if constexpr (ESZ == 2) {
+    if constexpr (ESZ == 0) {
+        if (nimax <= 1)
+            return gemv16_task<0, 1>(p, s, g, kc, warp, lane, xg, wt);
+        return gemv16_task<0, 2>(p, s, g, kc, warp, lane, xg, wt);
+    } else if constexpr (ESZ == 2) {
         if (nimax <= 2)
             return gemv16_task<2, 2>(p, s, g, kc, warp, lane, xg, wt);
         if (nimax <= 4)
@@ -1358,10 +1461,15 @@ __device__ __forceinline__ bool run_gemv(const KParams &p, const SmemLayout &s, 
                                          uint64_t *wt)
 {
     if constexpr (!GENERIC) {
-        if constexpr (Q8)
+        if constexpr (Q8 == 2) {
+            if (g.esz == 2)  // a tied LM head stays bf16
+                return gemv16<2>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16<0>(p, s, g, kc, warp, lane, xg, wt);
+        } else if constexpr (Q8 == 1) {
             return gemv16<1>(p, s, g, kc, warp, lane, xg, wt);
-        else
+        } else {
             return gemv16<2>(p, s, g, kc, warp, lane, xg, wt);
+        }
     } else {
         if (g.esz == 2) {
             if (g.VB == 16)
@@ -2032,7 +2140,7 @@ __device__ __forceinline__ bool ffn_down(const KParams &p, const SmemLayout &s, 
         a = gt / (1.f + __expf(-gt)) * up;
         s.vec[ct] = a;
     }
-    const bool q8 = GENERIC ? g.esz == 1 : Q8 != 0;
+    const bool q8 = GENERIC ? g.esz == 1 : Q8 == 1;
     if (q8) {
         float m = fabsf(a);
 #pragma unroll
@@ -2058,7 +2166,7 @@ __device__ __forceinline__ bool ffn_down(const KParams &p, const SmemLayout &s, 
     }
     const int ncb = g.ncb;
     if (g.esz == 1) {
-        if constexpr (GENERIC || Q8) {
+        if constexpr (GENERIC || Q8 == 1) {
             if (ncb <= 2)
                 return ffn_down_i8<2>(p, s, g, d, kc, ct, lane);
             if (ncb <= 4)
@@ -2066,7 +2174,7 @@ __device__ __forceinline__ bool ffn_down(const KParams &p, const SmemLayout &s, 
             return ffn_down_i8<8>(p, s, g, d, kc, ct, lane);
         }
     } else {
-        if constexpr (GENERIC || !Q8)
+        if constexpr (GENERIC || Q8 == 0)
             return ffn_down_bf16(p, s, g, d, kc, ct, lane);
     }
     return false;

@@ -98,7 +98,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     if (h <= 0 || L <= 0 || nh <= 0 || nkv <= 0 || hd <= 0 || F <= 0 || V <= 0 ||
         c.max_ctx <= 0 || n_sms <= 0)
         return amk_set_error(AMK_ERR_INVALID_ARG, "lowering: non-positive shape or SM count");
-    if (c.quant != AMK_QUANT_BF16 && c.quant != AMK_QUANT_W8A16)
+    if (c.quant != AMK_QUANT_BF16 && c.quant != AMK_QUANT_W8A16 && c.quant != AMK_QUANT_W4A16)
         return amk_set_error(AMK_ERR_INVALID_ARG, "lowering: unknown quant mode %d", c.quant);
     if (!(c.rms_eps >= 0.f) || !(c.rope_theta > 0.f))
         return amk_set_error(AMK_ERR_INVALID_ARG, "lowering: bad rms_eps or rope_theta");
@@ -113,7 +113,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     // whose GEMV does less work per byte; the depth at a fixed ring size
     // matters far less than the stage size
     if (opt.stage_bytes <= 0)
-        opt.stage_bytes = c.quant == AMK_QUANT_W8A16 ? 48 * 1024 : 64 * 1024;
+        opt.stage_bytes = c.quant != AMK_QUANT_BF16 ? 48 * 1024 : 64 * 1024;
     if (opt.ring_stages <= 0)
         opt.ring_stages = std::max(2, std::min(amk::kMaxStages, 192 * 1024 / opt.stage_bytes));
     if (opt.ring_stages < 2 || opt.ring_stages > amk::kMaxStages || opt.stage_bytes < 1024 ||
@@ -140,15 +140,21 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     if (G > 32 || lph * G > 32 || hd % lph || att_e > 16 || (att_e & (att_e - 1)))
         return amk_set_error(AMK_ERR_UNSUPPORTED, "attention layout: group %d x head_dim %d "
                              "does not fit one warp", G, hd);
-    const int esz = c.quant == AMK_QUANT_W8A16 ? 1 : 2;
-    const int head_esz = (c.tied_embeddings || c.quant != AMK_QUANT_W8A16) ? 2 : 1;
+    // bytes per weight: 2 (bf16), 1 (int8), or 0 for packed int4 rows
+    const bool q4 = c.quant == AMK_QUANT_W4A16;
+    const int esz = c.quant == AMK_QUANT_W8A16 ? 1 : q4 ? 0 : 2;
+    const int head_esz = c.tied_embeddings ? 2 : esz;
+    auto rowb = [](int K, int e) -> int64_t { return e ? (int64_t)K * e : amk::q4_row_bytes(K); };
     struct Mat { int rows, K, esz; const char *name; };
     const Mat mats[] = {{nh * hd, h, esz, "wq"}, {nkv * hd, h, esz, "wk"},
                         {nkv * hd, h, esz, "wv"}, {h, nh * hd, esz, "wo"},
                         {F, h, esz, "wgate"},     {F, h, esz, "wup"},
                         {h, F, esz, "wdown"},     {V, h, head_esz, "lm_head"}};
     for (const Mat &m : mats) {
-        const int64_t rb = (int64_t)m.K * m.esz;
+        const int64_t rb = rowb(m.K, m.esz);
+        if (m.esz == 0 && m.K % 32)
+            return amk_set_error(AMK_ERR_UNSUPPORTED, "%s: W4A16 rows need a multiple of 32 "
+                                 "inputs (whole 16-byte code vectors), not %d", m.name, m.K);
         if (m.K > kMaxK)
             return amk_set_error(AMK_ERR_UNSUPPORTED, "%s: inner dimension %d > %d", m.name,
                                  m.K, kMaxK);
@@ -202,10 +208,16 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     P->att_hpb = 32 / lph;
     P->att_pg = std::max(1, 32 / (lph * G));
     P->att_e = hd / lph;
+    // the generic instance takes odd row widths and a bf16 tied head on int8
+    // layers; the int4 instance runs a tied bf16 head itself and has no odd
+    // rows (K % 32 == 0 above), so int4 never needs it
     P->generic = (c.tied_embeddings && c.quant == AMK_QUANT_W8A16) ? 1 : 0;
     for (const Mat &m : mats)
-        if (((int64_t)m.K * m.esz) % 16)
+        if (rowb(m.K, m.esz) % 16)
             P->generic = 1;
+    if (q4 && P->generic)
+        return amk_set_error(AMK_ERR_UNSUPPORTED, "W4A16: a tied head of %d-byte rows is not "
+                             "a multiple of 16 bytes", h * 2);
 
     // FFN fusion: the columns [a, b) of Wdown come as 2-D TMA boxes of 16
     // bytes x box_rows rows, so the slice starts and the row pitch must be
@@ -216,12 +228,14 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
             box_rows = br;
     // slice width: a multiple of 16 bytes of a Wdown row, about one slice per
     // SM, at most 128 (the gate/up half of the red buffer)
-    const int ffn_gran = 16 / esz;
+    // (int4 weights keep separate FFN levels: no fused int4 down projection)
+    const int fesz = q4 ? 1 : esz;
+    const int ffn_gran = 16 / fesz;
     const int ffn_units = F / ffn_gran, n_target = n_sms * std::max(1, opt.tasks_per_sm);
     const int ffn_w = std::min((ffn_units + n_target - 1) / n_target * ffn_gran,
                                amk::kMaxTaskRows / 2 / ffn_gran * ffn_gran);
     const int64_t ffn_fit = box_rows ? (int64_t)opt.stage_bytes /
-                                           ((int64_t)ffn_w * esz * box_rows) * box_rows
+                                           ((int64_t)ffn_w * fesz * box_rows) * box_rows
                                      : 0;
     // default (ffn_fused = 1): fuse when a residual row is at most 1.5 KB.  The
     // fused level adds every slice's partial down projection into the same
@@ -229,10 +243,10 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     // the width; measured on B200 it gains 3% on the SmolLM2 shape (1152 B) but
     // loses 2% on Llama-1B W8A16 (2 KB), 4% on Llama-7B and 10% on TinyLlama.
     // ffn_fused = 2 fuses whenever the shape allows.
-    const bool shape_ok = F % ffn_gran == 0 && box_rows > 0 && ((int64_t)F * esz) % 16 == 0 &&
-                          (ffn_fit >= h || ffn_fit >= 256);
+    const bool shape_ok = !q4 && F % ffn_gran == 0 && box_rows > 0 &&
+                          ((int64_t)F * fesz) % 16 == 0 && (ffn_fit >= h || ffn_fit >= 256);
     const bool fused = shape_ok && (opt.ffn_fused >= 2 ||
-                                    (opt.ffn_fused == 1 && (int64_t)h * esz <= 1536));
+                                    (opt.ffn_fused == 1 && (int64_t)h * fesz <= 1536));
     P->ffn_fused = fused ? 1 : 0;
     P->ffn_box_rows = fused ? box_rows : 0;
 
@@ -258,7 +272,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     const int tps = std::max(1, opt.tasks_per_sm);
     auto gemv_level = [&](uint8_t kind, int layer, int rows, int K, int e, int target,
                           int max_rows, uint8_t mat, std::vector<Logical> &out) {
-        const int64_t rb = (int64_t)K * e;
+        const int64_t rb = rowb(K, e);
         int n = std::max(target, (rows + max_rows - 1) / max_rows);
         std::vector<std::pair<int, int>> tl;
         for (;; ++n) {  // granule rounding may grow a tile past max_rows
@@ -501,7 +515,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     // ---- bytes streamed per step -------------------------------------------
     int64_t wb = 0;
     for (const Mat &m : mats) {
-        const int64_t bytes = (int64_t)m.rows * m.K * m.esz;
+        const int64_t bytes = (int64_t)m.rows * rowb(m.K, m.esz);  // int4: scales included
         const bool is_head = !strcmp(m.name, "lm_head");
         wb += is_head ? bytes : bytes * L;
         if (m.esz == 1)
@@ -542,7 +556,9 @@ void amk_task_geometry(const amk_plan *P, amk::TaskDesc *dp, int packed_down)
     const amk_config &c = P->cfg;
     const int stage = P->opt.stage_bytes;
     constexpr int W = amk::kConsumerWarps;
-    int K = c.hidden, esz = c.quant == AMK_QUANT_W8A16 ? 1 : 2, parts = 1;
+    // bytes per weight: 2 (bf16), 1 (int8), 0 (packed int4 rows with their scales)
+    int K = c.hidden, parts = 1;
+    int esz = c.quant == AMK_QUANT_W8A16 ? 1 : c.quant == AMK_QUANT_W4A16 ? 0 : 2;
     if (d.kind == amk::TK_OPROJ)
         K = c.n_heads * c.head_dim;
     else if (d.kind == amk::TK_DOWN)
@@ -551,17 +567,19 @@ void amk_task_geometry(const amk_plan *P, amk::TaskDesc *dp, int packed_down)
         parts = 2;
     else if (d.kind == amk::TK_LMHEAD && c.tied_embeddings)
         esz = 2;
-    const int RB = K * esz, R = d.r1 - d.r0;
+    const int RB = esz ? K * esz : amk::q4_row_bytes(K), R = d.r1 - d.r0;
     const int gran = gran_rows(RB);
     int rpc = stage / RB;
     rpc -= rpc % gran;
     // warp layout: each lane keeps at most 64 activations of its K-slice in
     // registers.  K is split across more warps when a row needs it, and also
     // while that gives every warp fewer than four rows of a chunk (the GEMV
-    // takes rows four at a time) and still leaves each lane a whole vector
+    // takes rows four at a time) and still leaves each lane a whole vector.
+    // int4 rows: 32 codes per 16-byte vector (the scales after them are not
+    // vectors of the slice), at most two vectors per lane
     const int VB = (RB % 16 == 0) ? 16 : ((RB % 8 == 0) ? 8 : 4);
-    const int NV = RB / VB;
-    const int max_vec = 64 / (VB / esz);
+    const int NV = esz ? RB / VB : K / 32;
+    const int max_vec = esz ? 64 / (VB / esz) : 2;
     const int rows = std::min(rpc, R);
     int KS = 1, ks_log2 = 0;
     while (KS < W) {
@@ -609,7 +627,11 @@ void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *k
     amk::TaskDesc d = P->tasks[t];
     const int l = d.layer;
     const bool q8 = c.quant == AMK_QUANT_W8A16;
-    const int esz = q8 ? 1 : 2;
+    const bool q4 = c.quant == AMK_QUANT_W4A16;
+    // row bytes of a K-input weight row (int4: the packed row, scales included)
+    auto rb = [&](int K) -> int64_t {
+        return q4 ? amk::q4_row_bytes(K) : (int64_t)K * (q8 ? 1 : 2);
+    };
     auto row = [](const void *base, int64_t r, int64_t row_bytes) {
         return static_cast<const void *>(static_cast<const uint8_t *>(base) + r * row_bytes);
     };
@@ -623,7 +645,7 @@ void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *k
     case amk::TK_QKV: {
         const void *const *mats[3] = {w->wq, w->wk, w->wv};
         const void *const *scs[3] = {w->sq, w->sk, w->sv};
-        d.w0 = row(mats[d.mat][l], d.r0, (int64_t)h * esz);
+        d.w0 = row(mats[d.mat][l], d.r0, rb(h));
         d.s0 = srow(scs[d.mat], d.r0);
         d.gain = static_cast<const uint16_t *>(w->attn_norm[l]);
         break;
@@ -635,23 +657,23 @@ void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *k
         break;
     }
     case amk::TK_OPROJ:
-        d.w0 = row(w->wo[l], d.r0, (int64_t)c.n_heads * c.head_dim * esz);
+        d.w0 = row(w->wo[l], d.r0, rb(c.n_heads * c.head_dim));
         d.s0 = srow(w->so, d.r0);
         break;
     case amk::TK_GATEUP:
-        d.w0 = row(w->wgate[l], d.r0, (int64_t)h * esz);
-        d.w1 = row(w->wup[l], d.r0, (int64_t)h * esz);
+        d.w0 = row(w->wgate[l], d.r0, rb(h));
+        d.w1 = row(w->wup[l], d.r0, rb(h));
         d.s0 = srow(w->sgate, d.r0);
         d.s1 = srow(w->sup, d.r0);
         d.gain = static_cast<const uint16_t *>(w->ffn_norm[l]);
         break;
     case amk::TK_DOWN:
-        d.w0 = row(w->wdown[l], d.r0, (int64_t)c.ffn * esz);
+        d.w0 = row(w->wdown[l], d.r0, rb(c.ffn));
         d.s0 = srow(w->sdown, d.r0);
         break;
     case amk::TK_FFN:  // Wdown comes through the layer's tensor map
-        d.w0 = row(w->wgate[l], d.r0, (int64_t)h * esz);
-        d.w1 = row(w->wup[l], d.r0, (int64_t)h * esz);
+        d.w0 = row(w->wgate[l], d.r0, rb(h));
+        d.w1 = row(w->wup[l], d.r0, rb(h));
         d.s0 = srow(w->sgate, d.r0);
         d.s1 = srow(w->sup, d.r0);
         d.s2 = srow(w->sdown, 0);
@@ -659,7 +681,8 @@ void amk_resolve_task(const amk_plan *P, const amk_weights *w, const uint16_t *k
         break;
     default: {  // TK_LMHEAD
         const bool head_q8 = q8 && !c.tied_embeddings;
-        d.w0 = row(c.tied_embeddings ? w->embed : w->lm_head, d.r0, (int64_t)h * (head_q8 ? 1 : 2));
+        d.w0 = row(c.tied_embeddings ? w->embed : w->lm_head, d.r0,
+                   c.tied_embeddings ? (int64_t)h * 2 : rb(h));
         d.s0 = head_q8 ? static_cast<const uint16_t *>(w->lm_head_scale) + d.r0 : nullptr;
         d.gain = static_cast<const uint16_t *>(w->final_norm);
         break;

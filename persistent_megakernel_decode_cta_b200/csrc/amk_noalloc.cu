@@ -109,6 +109,9 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
         return amk_set_error(AMK_ERR_POS_RANGE, "amk_decode_step_noalloc: token %d / pos %d "
                              "out of range", token_id, pos);
     const bool q8 = c.quant == AMK_QUANT_W8A16;
+    if (c.quant == AMK_QUANT_W4A16)
+        return amk_set_error(AMK_ERR_UNSUPPORTED, "amk_decode_step_noalloc: int4 weights are "
+                             "packed by amk_create, which allocates; use amk_create");
     if (!ok16(w->embed) || !ok16(w->final_norm) || !w->attn_norm || !w->ffn_norm ||
         (!c.tied_embeddings && (!ok16(w->lm_head) || (q8 && !w->lm_head_scale))))
         return amk_set_error(AMK_ERR_INVALID_ARG, "amk_decode_step_noalloc: weights");

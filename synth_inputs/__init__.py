@@ -94,6 +94,11 @@ CONFIGS: Dict[str, ModelConfig] = {
                            max_ctx=2112),
     "llama7b_w8": ModelConfig("llama7b_w8", 4096, 32, 32, 32, 128, 11008,
                               32000, max_ctx=2112, quant="w8a16"),
+    # int4 weight-only variants (the pages' int4 figure is on SmolLM2-135M)
+    "smol135_w4": ModelConfig("smol135_w4", 576, 30, 9, 3, 64, 1536, 49152,
+                              max_ctx=256, tied=True, quant="w4a16"),
+    "llama7b_w4": ModelConfig("llama7b_w4", 4096, 32, 32, 32, 128, 11008,
+                              32000, max_ctx=2112, quant="w4a16"),
 }
 
 

@@ -53,6 +53,46 @@ def test_tiny_greedy(variant, n_sms):
         assert np.allclose(gk, rk, rtol=2 ** -7, atol=atol)
 
 
+def test_tiny_w4a16_greedy():
+    """int4 weights with 128-input group scales (the down projection's 192
+    inputs end in a group of 64), 8 greedy steps against the oracle."""
+    cfg = si.get_config("tiny").with_(quant="w4a16", ffn=192, name="tiny_w4")
+    pair = Pair(cfg)
+    st = pair.dec.stats()
+    assert (st.ring_stages, st.stage_bytes) == (4, 49152)
+    worst, checked = greedy_teacher_forced(pair, si.make_prompt(cfg, 4), 8)
+    assert checked >= 6
+
+
+@pytest.mark.parametrize("name,ctxs", [
+    ("smol135_w4", [0, 128]),   # tied bf16 head on int4 layers, 576-input rows
+    ("llama7b_w4", [0, 2048]),
+])
+def test_w4a16_full_size(name, ctxs):
+    cfg = si.get_config(name)
+    pair = Pair(cfg)
+    for ctx in ctxs:
+        pair.dec.reset()
+        pair.orc.reset()
+        if ctx:
+            pair.fill_kv(ctx)
+        tok = si.make_prompt(cfg, 1, seed=10 + ctx)[0]
+        g, am, ref, ref_am = pair.step(tok, ctx)
+        compare(cfg, g, am, ref, ref_am, what=f"{name} ctx {ctx}")
+    del pair
+    torch.cuda.empty_cache()
+
+
+def test_w4a16_greedy_32_steps():
+    """The int4 path over many steps: SmolLM2 W4A16, 32 greedy steps."""
+    cfg = si.get_config("smol135_w4")
+    pair = Pair(cfg)
+    worst, checked = greedy_teacher_forced(pair, si.make_prompt(cfg, 1), 31)
+    assert checked >= 16
+    del pair
+    torch.cuda.empty_cache()
+
+
 def test_tiny_device_token_chaining():
     """token_id = -1 feeds the previous step's device argmax (no host copy):
     the chained run must give exactly the tokens of a run whose tokens are

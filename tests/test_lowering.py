@@ -145,7 +145,7 @@ def test_balanced_tiles_on_148_sms():
     (dict(ffn=12290), "AMK_ERR_UNSUPPORTED"),            # down K above the register slice
     (dict(hidden=0), "AMK_ERR_INVALID_ARG"),
     (dict(ffn=171), "AMK_ERR_UNSUPPORTED"),              # odd bf16 K: row not 4-byte aligned
-    (dict(quant="w4a16"), "AMK_ERR_UNSUPPORTED"),        # int4: oracle only, no kernel
+    (dict(quant="w4a16"), "AMK_ERR_UNSUPPORTED"),        # int4 rows of 172 inputs: not 32-multiples
 ])
 def test_unsupported_shapes_rejected(edit, status):
     cfg = si.get_config("tiny").with_(**edit)
@@ -175,3 +175,47 @@ def test_ring_shape_resolved_per_weight_format(name):
     assert (st.ring_stages, st.stage_bytes) == (6, 32768)
     st = amk.Plan(cfg, 148, amk.default_options(ring_stages=2, stage_bytes=65536)).stats()
     assert (st.ring_stages, st.stage_bytes) == (2, 65536)
+
+
+@pytest.mark.parametrize("name", ["smol135_w4", "llama7b_w4", "tinyllama", "llama1b_w8"])
+def test_w4a16_lowering(name):
+    """int4 plans: 48 KiB stages, split FFN levels, and streamed bytes equal
+    to the codes and group scales plus the padding of each row to 16 bytes."""
+    cfg = si.get_config(name).with_(quant="w4a16")
+    st = amk.Plan(cfg, 148).stats()
+    assert (st.ring_stages, st.stage_bytes) == (4, 48 * 1024)
+    sb = si.streamed_weight_bytes(cfg)
+    assert sb <= st.weight_bytes <= sb * 1.025
+    kinds, _ = amk.Plan(cfg, 148, amk.default_options(ffn_fused=2)).task_info()
+    assert 7 not in kinds  # no fused FFN level for int4 weights
+
+
+def test_w4a16_rows_need_whole_code_vectors():
+    cfg = si.get_config("tiny").with_(quant="w4a16", ffn=192)
+    amk.Plan(cfg, 4)
+    with pytest.raises(amk.AmkError) as e:
+        amk.Plan(cfg.with_(ffn=176), 4)
+    assert e.value.name == "AMK_ERR_UNSUPPORTED"
+
+
+def test_noalloc_refuses_int4_models_on_the_host():
+    """int4 weights are packed by amk_create, which allocates: the
+    no-allocation step refuses them before any device work (the pointers
+    below are aligned stand-ins that are never dereferenced)."""
+    import ctypes
+    from persistent_megakernel_decode_cta_b200 import abi
+    cfg = si.get_config("smol135_w4")
+    plan = amk.Plan(cfg, 148)
+    fake = 1 << 20
+    ptrs = (ctypes.c_void_p * cfg.n_layers)(*([fake] * cfg.n_layers))
+    ws = abi.Weights()
+    for f in ("embed", "final_norm"):
+        setattr(ws, f, fake)
+    for name in ("attn_norm", "ffn_norm", "wq", "wk", "wv", "wo", "wgate", "wup", "wdown",
+                 "sq", "sk", "sv", "so", "sgate", "sup", "sdown"):
+        setattr(ws, name, ctypes.cast(ptrs, abi.c_vpp))
+    lib = abi.lib()
+    rc = lib.amk_decode_step_noalloc(plan._p, ctypes.byref(ws), fake, 0, 0, fake, None, None)
+    assert rc == abi.ERR["AMK_ERR_UNSUPPORTED"]
+    assert b"int4" in lib.amk_last_error()
+    plan.close()
