@@ -446,6 +446,27 @@ def run_ours(args):
         phases = phase_shares(pdec.profile())
         pdec.close()
 
+    # ---- HBM read ceiling on this machine (outside the timed region) --------------
+    # A plain streaming read (torch's sum of a 4 GiB bf16 tensor, fp32
+    # accumulate): the decode step only reads weights and KV, so its fraction
+    # of this read rate is reported beside the fraction of the copy peak
+    # (which counts read and write bytes).
+    read_gbs = None
+    if rank == 0:
+        buf = torch.empty(2 << 30, dtype=torch.bfloat16, device="cuda").fill_(1.0)
+        torch.cuda.synchronize()
+        for _ in range(2):
+            buf.sum(dtype=torch.float32)
+        ra, rb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ra.record()
+        for _ in range(10):
+            buf.sum(dtype=torch.float32)
+        rb.record()
+        torch.cuda.synchronize()
+        read_gbs = buf.numel() * 2 * 10 / (ra.elapsed_time(rb) * 1e-3) / 1e9
+        del buf
+        torch.cuda.empty_cache()
+
     nbytes = algorithmic_bytes(cfg, ctx)
     peak, peak_kind = measured_peak()
     achieved = nbytes / (kernel_ms * 1e-3) / 1e9
@@ -468,7 +489,11 @@ def run_ours(args):
                          "frac": achieved / peak, "traffic": load_traffic(name),
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
                          "algorithmic_bytes_per_launch": nbytes,
-                         "kernel_us_per_launch": kernel_ms * 1e3},
+                         "kernel_us_per_launch": kernel_ms * 1e3,
+                         "read_ceiling_gbs": read_gbs,
+                         "frac_of_read_ceiling": achieved / read_gbs if read_gbs else None,
+                         "read_ceiling_how": "torch sum of a 4 GiB bf16 tensor on this GPU, "
+                                             "10 launches, CUDA events (read bytes only)"},
             "achieved_gbs": achieved,
             "cpu_baseline": cpu_base,
             "e2e": {"value": job_us_per_token(e2e_s * 1e3, K_e2e, world), "unit": UNIT,
@@ -493,6 +518,77 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_noalloc(args):
+    """Times amk_decode_step_noalloc on the workload (one GPU): device time
+    per call (CUDA events on the stream) and host time per call (the task
+    table is resolved on the host and uploaded into the static array on
+    every call), next to amk_decode_step on the same weights.  Prints one
+    JSON line; not part of the driver's contract."""
+    import persistent_megakernel_decode_cta_b200 as amk
+    from persistent_megakernel_decode_cta_b200 import build as amk_build
+    amk_build.build()
+    torch.cuda.set_device(0)
+    name = args.workload
+    mname, ctx = WORKLOADS[name]
+    cfg = si.get_config(mname)
+    w = si.make_model(cfg, seed=0, device="cuda")
+    kv_fill = si.make_kv_fill(cfg, ctx, device="cuda") if ctx else None
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    plan = amk.Plan(cfg, sms)
+    ws, keep = amk.weights_struct(cfg, w)
+    kv = torch.zeros((cfg.n_layers, 2, cfg.n_kv_heads, cfg.max_ctx, cfg.head_dim),
+                     dtype=torch.bfloat16, device="cuda")
+    if kv_fill is not None:
+        kv[:, :, :, :ctx].copy_(kv_fill)
+    logits = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+    tok = si.make_prompt(cfg, 1, seed=10 + ctx)[0]
+    st = plan.stats()
+    for _ in range(max(args.warmup, 3)):
+        amk.decode_step_noalloc(plan, ws, kv, tok, ctx, logits)
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    host = []
+    ev[0].record()
+    for i in range(K):
+        t0 = time.perf_counter()
+        amk.decode_step_noalloc(plan, ws, kv, tok, ctx, logits)
+        host.append(time.perf_counter() - t0)
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    dev = [ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(K)]
+    dec = amk.Decoder(cfg, w)
+    if kv_fill is not None:
+        for l in range(cfg.n_layers):
+            k, v = dec.kv(l)
+            k[:, :ctx].copy_(kv_fill[l, 0])
+            v[:, :ctx].copy_(kv_fill[l, 1])
+    dec.step(tok, ctx, want_argmax=False)
+    for _ in range(3):
+        dec.step(tok, ctx, want_argmax=False)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(K):
+        dec.step(tok, ctx, want_argmax=False)
+    b.record()
+    torch.cuda.synchronize()
+    alloc_us = a.elapsed_time(b) * 1e3 / K
+    dec.close()
+    table = st.n_tasks * 96 + (sms + 1) * 4
+    print(json.dumps({
+        "metric": "amk_decode_step_noalloc us/token", "workload": name, "steps": K,
+        "device_us_per_call": {"p10": float(np.percentile(dev, 10)),
+                               "p50": float(np.percentile(dev, 50)),
+                               "p90": float(np.percentile(dev, 90))},
+        "host_us_per_call": {"p50": float(np.percentile(host, 50) * 1e6),
+                             "p90": float(np.percentile(host, 90) * 1e6)},
+        "amk_decode_step_us_per_call": alloc_us,
+        "schedule_upload_bytes_per_call": table, "tasks": st.n_tasks,
+    }), flush=True)
+    plan.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -502,10 +598,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-phases", action="store_true",
                     help="skip the profiled step that reports the phase-timer shares")
+    ap.add_argument("--noalloc", action="store_true",
+                    help="time amk_decode_step_noalloc (schedule upload per call included) "
+                         "instead of the bench line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.noalloc:
+        run_noalloc(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

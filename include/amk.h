@@ -139,7 +139,11 @@ typedef struct {
                                  on its own mbarrier (KiB; 0 = default 64: one piece per
                                  stage; smaller pieces let the cap bind more finely but cost
                                  the producer more issue work) */
-    int32_t reserved[2];
+    int32_t sm_rotate;        /* SM assignment: each level's tiles go to the least-loaded
+                                 SMs scanning from SM (level index * sm_rotate) mod n_sms,
+                                 so the knob moves tiles between SMs without changing the
+                                 balance; 0 (default) = always from SM 0 */
+    int32_t reserved;
 } amk_options;
 
 typedef struct amk_handle amk_handle;
@@ -364,11 +368,13 @@ AMK_API int amk_get_error_info(amk_handle *h, amk_error_info *out);
  * the set-up: it looks up the static array's device address
  * (cudaGetSymbolAddress, which may load the library's device code), so make
  * that first call before any stream capture; later calls look the address
- * up again, so it stays right after a cudaDeviceReset.  Every call
- * re-uploads the schedule and clears the counters in the shared array, which
- * keeps the last call's contents: calls that can overlap on the GPU (other
- * streams, other host threads) race on it and must be serialised by the
- * caller. */
+ * up again, so it stays right after a cudaDeviceReset.  A call uploads the
+ * schedule (the task table resolved against w and kv_cache) into the shared
+ * array unless the previous call on the device left the same plan's table
+ * there, resolved against the same pointers in the same CUDA context; every
+ * call clears the counters.  The array keeps the last call's contents: calls
+ * that can overlap on the GPU (other streams, other host threads) race on it
+ * and must be serialised by the caller. */
 #define AMK_NOALLOC_SCRATCH_BYTES (16u << 20)
 AMK_API int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *w, void *kv_cache,
                                     int32_t token_id, int32_t pos, float *logits_dev,

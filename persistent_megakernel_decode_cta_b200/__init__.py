@@ -13,7 +13,7 @@ from typing import Dict, List, Optional, Tuple
 from . import abi
 
 __all__ = ["AmkError", "Decoder", "Plan", "validate_graph", "default_options", "version",
-           "make_config"]
+           "make_config", "weights_struct", "decode_step_noalloc"]
 
 
 class AmkError(RuntimeError):
@@ -195,37 +195,64 @@ class _DevArray:
                                          "strides": None}
 
 
+_PER_LAYER = ("attn_norm", "ffn_norm", "wq", "wk", "wv", "wo", "wgate", "wup", "wdown",
+              "sq", "sk", "sv", "so", "sgate", "sup", "sdown")
+
+
+def weights_struct(cfg, weights: Dict[str, object]):
+    """An amk_weights for torch CUDA tensors (the dict of
+    ``synth_inputs.make_model``).  Returns (struct, keep-alive list): the
+    pointer arrays the struct points into live as long as the list."""
+    w = abi.Weights()
+    keep = []
+
+    def ptr(t):
+        return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+    w.embed = ptr(weights["embed"])
+    w.final_norm = ptr(weights["final_norm"])
+    w.lm_head = ptr(weights.get("lm_head"))
+    w.lm_head_scale = ptr(weights.get("lm_head_scale"))
+    L = cfg.n_layers
+    for name in _PER_LAYER:
+        lst = weights.get(name)
+        if lst is None:
+            setattr(w, name, None)
+            continue
+        arr = (ctypes.c_void_p * L)(*[t.data_ptr() for t in lst])
+        keep.append(arr)
+        setattr(w, name, ctypes.cast(arr, abi.c_vpp))
+    return w, keep
+
+
+def decode_step_noalloc(plan: "Plan", w, kv, token: int, pos: int, logits,
+                        want_argmax: bool = False, stream=None) -> Optional[int]:
+    """amk_decode_step_noalloc: one decode step that allocates nothing.  ``w``
+    from weights_struct; ``kv`` (bf16 [L, 2, n_kv_heads, max_ctx, head_dim])
+    and ``logits`` (float32 [vocab]) are caller-owned torch CUDA tensors."""
+    import torch
+    am = abi.c_i32(-1)
+    st = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    rc = abi.lib().amk_decode_step_noalloc(plan._p, ctypes.byref(w), kv.data_ptr(), int(token),
+                                           int(pos), logits.data_ptr(),
+                                           ctypes.byref(am) if want_argmax else None,
+                                           ctypes.c_void_p(st))
+    _check(rc, "amk_decode_step_noalloc")
+    return int(am.value) if want_argmax else None
+
+
 class Decoder:
     """One amk_handle: weights borrowed from torch CUDA tensors, KV cache and
     workspace owned by the library."""
 
-    _PER_LAYER = ("attn_norm", "ffn_norm", "wq", "wk", "wv", "wo", "wgate", "wup", "wdown",
-                  "sq", "sk", "sv", "so", "sgate", "sup", "sdown")
+    _PER_LAYER = _PER_LAYER
 
     def __init__(self, cfg, weights: Dict[str, object], options: Optional[abi.Options] = None,
                  stream=None):
         import torch
         self.cfg = cfg
         self._weights = weights  # keep the borrowed tensors alive
-        self._keep = []
-        w = abi.Weights()
-
-        def ptr(t):
-            return None if t is None else ctypes.c_void_p(t.data_ptr())
-
-        w.embed = ptr(weights["embed"])
-        w.final_norm = ptr(weights["final_norm"])
-        w.lm_head = ptr(weights.get("lm_head"))
-        w.lm_head_scale = ptr(weights.get("lm_head_scale"))
-        L = cfg.n_layers
-        for name in self._PER_LAYER:
-            lst = weights.get(name)
-            if lst is None:
-                setattr(w, name, None)
-                continue
-            arr = (ctypes.c_void_p * L)(*[t.data_ptr() for t in lst])
-            self._keep.append(arr)
-            setattr(w, name, ctypes.cast(arr, abi.c_vpp))
+        w, self._keep = weights_struct(cfg, weights)
         if stream is None:
             stream = torch.cuda.current_stream().cuda_stream
         self.stream = stream

@@ -46,7 +46,8 @@ class Options(ctypes.Structure):
                 ("tasks_per_sm", c_i32), ("n_sms", c_i32), ("wait_timeout_us", c_u32),
                 ("debug_skip_signal_task", c_i32), ("profile", c_i32),
                 ("l2_prefetch_kb", c_i32), ("ffn_fused", c_i32),
-                ("pos0_plan", c_i32), ("inflight_kb", c_i32), ("copy_piece_kb", c_i32), ("reserved", c_i32 * 2)]
+                ("pos0_plan", c_i32), ("inflight_kb", c_i32), ("copy_piece_kb", c_i32),
+                ("sm_rotate", c_i32), ("reserved", c_i32)]
 
 
 class GraphWait(ctypes.Structure):

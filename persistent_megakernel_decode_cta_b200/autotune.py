@@ -1,9 +1,9 @@
 """Schedule-knob search for the decode megakernel on the current device.
 
 The schedule of a step is fixed by a few knobs (README "Two autoresearch
-loops": tiling, SM assignment, pipelining depth): the weight ring's depth and
-stage size, the split-K attention chunks, the fused FFN level, the L2
-lookahead.  ``tune`` tries a grid of them the way the pages' schedule loop
+loops": tiling, SM assignment, pipelining depth): GEMV row tiles per SM per
+level, the rotation of the tile-to-SM map, the weight ring's stage size and
+in-flight cap, the split-K attention chunks, the fused FFN level.  ``tune`` tries a grid of them the way the pages' schedule loop
 does -- lower, validate, check, measure, keep or drop -- with a correctness
 gate that needs no reference implementation: every candidate is lowered and
 validated by ``amk_create`` (a rejected schedule is dropped), and its first
@@ -24,12 +24,17 @@ from typing import Dict, Iterable, List, Optional, Tuple
 
 from . import Decoder, AmkError, default_options
 
+# The pages' schedule knobs: tiling (tasks_per_sm: GEMV row tiles per SM per
+# level), SM assignment (sm_rotate), pipelining depth (the ring's stages and
+# stage size, the in-flight cap), fusion grouping (ffn_fused) and the
+# split-K attention chunks.
 DEFAULT_SPACE: Dict[str, List[int]] = {
-    "ring_stages": [0, 2],  # 0: as many stages as make 192 KiB (6 x 32, 4 x 48, 3 x 64 KiB)
-    "stage_bytes": [32768, 49152, 65536],
-    "attn_splits": [0, 2, 4],
+    "stage_bytes": [32768, 49152, 65536],  # ring_stages 0: as many as make 192 KiB
+    "attn_splits": [0, 2, 8],
     "ffn_fused": [1, 2, -1],
-    "l2_prefetch_kb": [0, 128],
+    "tasks_per_sm": [1, 2],
+    "sm_rotate": [0, 37],
+    "inflight_kb": [0, 96],
 }
 
 
@@ -54,7 +59,7 @@ def _time_steps(dec: Decoder, ctx: int, steps: int, warmup: int) -> float:
 
 def tune(cfg, weights, ctx: int = 0, kv=None, space: Optional[Dict[str, Iterable[int]]] = None,
          steps: int = 20, warmup: int = 3, token: int = 0,
-         rtol: float = 1e-3) -> Tuple[object, List[Dict]]:
+         rtol: Optional[float] = None) -> Tuple[object, List[Dict]]:
     """Returns (the fastest passing amk_options, one report row per candidate:
     knobs, status "ok" / "rejected: ..." / "mismatch", us per step, max |dlogit|).
 
@@ -62,6 +67,13 @@ def tune(cfg, weights, ctx: int = 0, kv=None, space: Optional[Dict[str, Iterable
     positions 0..ctx-1 as a [n_layers, 2, n_kv_heads, ctx, head_dim] bf16
     tensor on the device."""
     import torch
+
+    if rtol is None:
+        # bf16 schedules differ only in rounding order; int8 / int4 GEMVs
+        # quantise each lane's activations to int16 with the lane's own
+        # scale, and a different K split moves those grids (both stay within
+        # the 2e-2 parity bound of the exact step)
+        rtol = 1e-3 if getattr(cfg, "quant", "bf16") == "bf16" else 1e-2
 
     def make(opts):
         dec = Decoder(cfg, weights, opts)

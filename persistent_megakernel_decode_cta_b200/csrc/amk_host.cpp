@@ -12,6 +12,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -96,9 +97,11 @@ extern "C" int amk_plan_create(const amk_config *cfg, const amk_options *opt, in
     if (!cfg || !out)
         return amk_set_error(AMK_ERR_INVALID_ARG, "amk_plan_create: NULL argument");
     *out = nullptr;
+    static std::atomic<uint64_t> next_uid{1};
     amk_plan *P = new (std::nothrow) amk_plan();
     if (!P)
         return amk_set_error(AMK_ERR_OOM, "amk_plan_create: out of host memory");
+    P->uid = next_uid.fetch_add(1);
     auto lower_checked = [&](amk_plan *Q, int pos0) {
         int r = amk_lower(cfg, opt, n_sms, Q, pos0);
         if (r == AMK_OK) {
@@ -115,6 +118,8 @@ extern "C" int amk_plan_create(const amk_config *cfg, const amk_options *opt, in
     int rc = lower_checked(P, 0);
     if (rc == AMK_OK && P->opt.pos0_plan > 0) {
         P->pos0 = new (std::nothrow) amk_plan();
+        if (P->pos0)
+            P->pos0->uid = next_uid.fetch_add(1);
         rc = P->pos0 ? lower_checked(P->pos0, 1)
                      : amk_set_error(AMK_ERR_OOM, "amk_plan_create: out of host memory");
     }

@@ -90,6 +90,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         if (opt_in->pos0_plan != 0) opt.pos0_plan = opt_in->pos0_plan;
         if (opt_in->inflight_kb != 0) opt.inflight_kb = opt_in->inflight_kb;
         if (opt_in->copy_piece_kb > 0) opt.copy_piece_kb = opt_in->copy_piece_kb;
+        if (opt_in->sm_rotate > 0) opt.sm_rotate = opt_in->sm_rotate;
         opt.n_sms = opt_in->n_sms;
     }
     const amk_config &c = *cfg;
@@ -120,6 +121,17 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         opt.stage_bytes % 1024)
         return amk_set_error(AMK_ERR_INVALID_ARG, "ring_stages in [2,%d], stage_bytes a "
                              "multiple of 1024", amk::kMaxStages);
+    // in-flight cap left at 0: 64 KiB, or 96 KiB for bf16 models whose layer
+    // streams at least 1 MiB per SM (bandwidth-bound levels: measured on
+    // B200, Llama-7B bf16 at KV context 2048 runs 1.2 % faster with 96 KiB,
+    // while TinyLlama, SmolLM2 and the int8 shapes gain nothing or lose up
+    // to 1 %, their levels being bound by latency, not by the stream)
+    if (opt.inflight_kb == 0 && c.quant == AMK_QUANT_BF16) {
+        const int64_t layer_bytes =
+            2 * ((int64_t)h * (nh * hd + 2 * nkv * hd) + (int64_t)nh * hd * h + 3 * (int64_t)h * F);
+        if (layer_bytes / n_sms >= (int64_t)1 << 20)
+            opt.inflight_kb = 96;
+    }
     const int G = nh / nkv;
     // attention lane layout: lph lanes per head, E = hd / lph elements per
     // lane, the G heads of a group side by side, and as many position groups
@@ -357,8 +369,12 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     }
 
     // ---- SM assignment: per level, heaviest task to the least-loaded SM --------
+    // (ties go to the SM with the least streamed so far, then to the first in
+    // the level's scan order, which starts at SM (level * sm_rotate) mod n_sms:
+    // the SM-assignment knob moves tiles between SMs without unbalancing them)
     std::vector<std::vector<TaskDesc>> queues(n_sms);
     std::vector<int64_t> cum(n_sms, 0);
+    int lvi = 0;
     for (auto &lv : levels) {
         std::vector<int> idx(lv.size());
         std::iota(idx.begin(), idx.end(), 0);
@@ -366,11 +382,14 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
                          [&](int a, int b) { return lv[a].cost > lv[b].cost; });
         std::vector<int64_t> load(n_sms, 0);
         std::vector<std::vector<int>> mine(n_sms);
+        const int start = (int)(((int64_t)lvi++ * std::max(0, opt.sm_rotate)) % n_sms);
         for (int i : idx) {
-            int best = 0;
-            for (int s = 1; s < n_sms; ++s)
+            int best = start;
+            for (int j = 1; j < n_sms; ++j) {
+                const int s = (start + j) % n_sms;
                 if (load[s] < load[best] || (load[s] == load[best] && cum[s] < cum[best]))
                     best = s;
+            }
             load[best] += std::max<int64_t>(lv[i].cost, 1);
             cum[best] += lv[i].cost;
             mine[best].push_back(i);

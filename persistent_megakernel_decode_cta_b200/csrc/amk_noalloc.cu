@@ -10,10 +10,12 @@
 // scratch (task table, counters, error word, argmax key, activations) lives
 // in the fixed array g_scratch below, which exists once per GPU from the
 // moment the library's device code is loaded until the process exits.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "amk.h"
 #include "amk_internal.h"
@@ -83,6 +85,73 @@ int scratch_address(unsigned char **out)
                              cudaGetErrorString(e));
     *out = static_cast<unsigned char *>(p);
     return AMK_OK;
+}
+
+// What the static array holds from the last call on a device: the plan and
+// the pointers its task table was resolved against, and the CUDA context it
+// was written in (a context id is never reused in a process, so a reset of
+// the device shows as a new id).  A call with the same key finds the task
+// table, queue offsets and tensor maps in place and uploads nothing but the
+// cleared counters; any other call rewrites them.
+struct UploadKey {
+    uint64_t plan_uid = 0, ctx_id = 0, wsig = 0;
+    const void *kv = nullptr;
+    unsigned char *base = nullptr;
+};
+constexpr int kMaxDevices = 64;
+std::mutex g_upload_mu;
+UploadKey g_uploaded[kMaxDevices];
+
+// FNV-1a over the weight pointers the task table holds.
+uint64_t weights_signature(const amk_config &c, const amk_weights *w)
+{
+    uint64_t h = 1469598103934665603ull;
+    auto mix = [&](const void *p) {
+        uint64_t v = (uint64_t)(uintptr_t)p;
+        for (int i = 0; i < 8; ++i, v >>= 8) {
+            h ^= (v & 0xff);
+            h *= 1099511628211ull;
+        }
+    };
+    mix(w->embed), mix(w->final_norm), mix(w->lm_head), mix(w->lm_head_scale);
+    const void *const *arr[16] = {w->attn_norm, w->ffn_norm, w->wq,    w->wk,
+                                  w->wv,        w->wo,       w->wgate, w->wup,
+                                  w->wdown,     w->sq,       w->sk,    w->sv,
+                                  w->so,        w->sgate,    w->sup,   w->sdown};
+    for (int a = 0; a < 16; ++a)
+        for (int l = 0; l < c.n_layers; ++l)
+            mix(arr[a] ? arr[a][l] : nullptr);
+    return h;
+}
+
+// The id of the calling thread's current CUDA context (0 if unknown: then
+// every call uploads).
+uint64_t current_context_id()
+{
+    typedef CUresult (*GetCurrent)(CUcontext *);
+    typedef CUresult (*GetId)(CUcontext, unsigned long long *);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static bool looked = false;
+    if (!looked) {
+        void *f1 = nullptr, *f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) ==
+                cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) == cudaSuccess &&
+            q2 == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<GetCurrent>(f1);
+            get_id = reinterpret_cast<GetId>(f2);
+        }
+        looked = true;
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
 }
 
 bool ok16(const void *p) { return p && ((uintptr_t)p % 16) == 0; }
@@ -165,38 +234,54 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
             if (!ok16(mats[m][l]) || (q8 && !scs[m][l]))
                 return amk_set_error(AMK_ERR_INVALID_ARG, "layer %d weight %d", l, m);
     }
-    // schedule tables with resolved pointers, in batches through a stack
-    // buffer (pageable sources: cudaMemcpyAsync stages them before returning,
-    // so the buffer can be reused at once)
-    e = cudaMemcpyAsync(base + lay.qoff, P.queue_off.data(), sizeof(int32_t) * P.queue_off.size(),
-                        cudaMemcpyHostToDevice, st);
-    if (e != cudaSuccess)
-        return fail_cuda(e, "schedule upload");
-    amk::TaskDesc batch[64];
-    const uint16_t *kv = static_cast<const uint16_t *>(kv_cache);
-    const int T = (int)P.tasks.size();
-    for (int t0 = 0; t0 < T; t0 += 64) {
-        const int n = T - t0 < 64 ? T - t0 : 64;
-        for (int i = 0; i < n; ++i)
-            amk_resolve_task(&P, w, kv, t0 + i, &batch[i], 0);
-        e = cudaMemcpyAsync(base + lay.tasks + sizeof(amk::TaskDesc) * (size_t)t0, batch,
-                            sizeof(amk::TaskDesc) * (size_t)n, cudaMemcpyHostToDevice, st);
+    // schedule tables with resolved pointers (skipped when the array already
+    // holds this plan's, resolved against these pointers in this context)
+    const UploadKey ukey{P.uid, current_context_id(), weights_signature(c, w), kv_cache, base};
+    bool cached = false;
+    if (dev >= 0 && dev < kMaxDevices && ukey.ctx_id != 0) {
+        std::lock_guard<std::mutex> lock(g_upload_mu);
+        const UploadKey &u = g_uploaded[dev];
+        cached = u.plan_uid == ukey.plan_uid && u.ctx_id == ukey.ctx_id && u.wsig == ukey.wsig &&
+                 u.kv == ukey.kv && u.base == ukey.base;
+        g_uploaded[dev] = UploadKey{};  // rewritten below; valid again once it is
+    }
+    if (!cached) {
+        // in batches through a stack buffer (pageable sources: cudaMemcpyAsync
+        // stages them before returning, so the buffer can be reused at once)
+        e = cudaMemcpyAsync(base + lay.qoff, P.queue_off.data(), sizeof(int32_t) * P.queue_off.size(),
+                            cudaMemcpyHostToDevice, st);
         if (e != cudaSuccess)
             return fail_cuda(e, "schedule upload");
-    }
-    // tensor maps of Wdown (fused FFN), through a stack buffer
-    if (P.ffn_fused) {
-        alignas(64) unsigned char mbuf[128 * 16];
-        for (int l0 = 0; l0 < c.n_layers; l0 += 16) {
-            const int n = c.n_layers - l0 < 16 ? c.n_layers - l0 : 16;
-            const int mrc = amk_encode_down_maps(&P, w, l0, n, mbuf);
-            if (mrc != AMK_OK)
-                return mrc;
-            e = cudaMemcpyAsync(base + lay.dmaps + 128 * (size_t)l0, mbuf, 128 * (size_t)n,
-                                cudaMemcpyHostToDevice, st);
+        amk::TaskDesc batch[64];
+        const uint16_t *kv = static_cast<const uint16_t *>(kv_cache);
+        const int T = (int)P.tasks.size();
+        for (int t0 = 0; t0 < T; t0 += 64) {
+            const int n = T - t0 < 64 ? T - t0 : 64;
+            for (int i = 0; i < n; ++i)
+                amk_resolve_task(&P, w, kv, t0 + i, &batch[i], 0);
+            e = cudaMemcpyAsync(base + lay.tasks + sizeof(amk::TaskDesc) * (size_t)t0, batch,
+                                sizeof(amk::TaskDesc) * (size_t)n, cudaMemcpyHostToDevice, st);
             if (e != cudaSuccess)
-                return fail_cuda(e, "tensor map upload");
+                return fail_cuda(e, "schedule upload");
         }
+        // tensor maps of Wdown (fused FFN), through a stack buffer
+        if (P.ffn_fused) {
+            alignas(64) unsigned char mbuf[128 * 16];
+            for (int l0 = 0; l0 < c.n_layers; l0 += 16) {
+                const int n = c.n_layers - l0 < 16 ? c.n_layers - l0 : 16;
+                const int mrc = amk_encode_down_maps(&P, w, l0, n, mbuf);
+                if (mrc != AMK_OK)
+                    return mrc;
+                e = cudaMemcpyAsync(base + lay.dmaps + 128 * (size_t)l0, mbuf, 128 * (size_t)n,
+                                    cudaMemcpyHostToDevice, st);
+                if (e != cudaSuccess)
+                    return fail_cuda(e, "tensor map upload");
+            }
+        }
+    }
+    if (dev >= 0 && dev < kMaxDevices && ukey.ctx_id != 0) {
+        std::lock_guard<std::mutex> lock(g_upload_mu);
+        g_uploaded[dev] = ukey;
     }
     // what must start at zero: counters, error word, argmax keys
     e = cudaMemsetAsync(base + lay.ctr, 0, lay.qkv - lay.ctr, st);

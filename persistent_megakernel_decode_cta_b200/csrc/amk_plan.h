@@ -24,6 +24,7 @@ struct amk_plan {
     int ffn_box_rows = 0;  // rows of a Wdown TMA box (divides hidden)
     int is_pos0 = 0;     // 1: the schedule of steps at position 0 (no attention level)
     amk_plan *pos0 = nullptr;  // owned: that schedule, for a plan of all other steps
+    uint64_t uid = 0;          // unique in the process (amk_plan_create numbers plans)
     amk_plan() = default;
     amk_plan(const amk_plan &) = delete;
     amk_plan &operator=(const amk_plan &) = delete;

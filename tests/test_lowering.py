@@ -219,3 +219,25 @@ def test_noalloc_refuses_int4_models_on_the_host():
     assert rc == abi.ERR["AMK_ERR_UNSUPPORTED"]
     assert b"int4" in lib.amk_last_error()
     plan.close()
+
+
+def test_sm_rotation_moves_tiles_not_balance():
+    """The SM-assignment knob: a rotated plan validates, keeps every level's
+    bytes per SM as balanced as the default plan, and puts tiles on other SMs."""
+    cfg = si.get_config("tinyllama")
+    a = amk.Plan(cfg, 148)
+    b = amk.Plan(cfg, 148, amk.default_options(sm_rotate=37))
+    ga, gb = a.graph(), b.graph()
+    assert len(ga["tasks"]) == len(gb["tasks"])
+    sa = [t["sm"] for t in ga["tasks"]]
+    sb = [t["sm"] for t in gb["tasks"]]
+    # levels with fewer tiles than SMs leave other SMs idle under rotation, so
+    # queue lengths move a little; the tiles and their bytes do not change
+    la = [len(q) for q in ga["queues"]]
+    lb = [len(q) for q in gb["queues"]]
+    assert max(lb) - min(lb) <= max(la) - min(la) + 3
+    ka, _ = a.task_info()
+    kb, _ = b.task_info()
+    assert sorted(ka) == sorted(kb)
+    assert sa != sb
+    assert a.stats().weight_bytes == b.stats().weight_bytes
