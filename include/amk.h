@@ -336,6 +336,21 @@ AMK_API int amk_get_profile(amk_handle *h, uint64_t *out, int64_t n_u64);
 typedef struct { int32_t code, task, counter, sm; uint32_t seen, target; } amk_error_info;
 AMK_API int amk_get_error_info(amk_handle *h, amk_error_info *out);
 
+/* ---- measurement ------------------------------------------------------- */
+/* The read ceiling of the decode step's weight stream (README, "Why a
+ * megakernel": the floor of a decode step is the bytes it reads over the
+ * memory bandwidth): the kernel's own bulk copies -- cp.async.bulk into a
+ * shared-memory ring of `stages` stages of stage_bytes on mbarriers, one CTA
+ * per SM on n_sms CTAs, evict-first L2 policy -- with nothing consuming them,
+ * over `bytes` of the device buffer buf (caller-owned, at least 1 GiB so that
+ * L2 cannot hold it, 16-byte aligned; only read).  One warm-up launch, then
+ * `reps` timed ones (CUDA events on cuda_stream); *gbs = the best read rate
+ * in GB/s.  Synchronises the stream; allocates n_sms words of device memory
+ * for the copies' status.  AMK_ERR_INVALID_ARG on a bad argument,
+ * AMK_ERR_TIMEOUT if a copy did not land within 1 s, AMK_ERR_CUDA otherwise. */
+AMK_API int amk_read_ceiling(const void *buf, int64_t bytes, int32_t n_sms, int32_t stage_bytes,
+                             int32_t stages, int32_t reps, void *cuda_stream, double *gbs);
+
 /* ---- decoding without allocating -------------------------------------- */
 /* (No counterpart in the AutoMegaKernel pages: an addition for callers that
  * may not allocate device memory.)  Some callers cannot call cudaMalloc: a

@@ -13,7 +13,7 @@ from typing import Dict, List, Optional, Tuple
 from . import abi
 
 __all__ = ["AmkError", "Decoder", "Plan", "validate_graph", "default_options", "version",
-           "make_config", "weights_struct", "decode_step_noalloc"]
+           "make_config", "weights_struct", "decode_step_noalloc", "read_ceiling"]
 
 
 class AmkError(RuntimeError):
@@ -239,6 +239,21 @@ def decode_step_noalloc(plan: "Plan", w, kv, token: int, pos: int, logits,
                                            ctypes.c_void_p(st))
     _check(rc, "amk_decode_step_noalloc")
     return int(am.value) if want_argmax else None
+
+
+def read_ceiling(buf, n_sms: int, stage_bytes: int = 32768, stages: int = 3, reps: int = 5,
+                 stream=None) -> float:
+    """amk_read_ceiling: GB/s of the decode kernel's bulk-copy weight stream
+    with nothing consuming it, over the torch CUDA tensor ``buf`` (>= 1 GiB)."""
+    import torch
+    g = ctypes.c_double(0.0)
+    st = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    rc = abi.lib().amk_read_ceiling(ctypes.c_void_p(buf.data_ptr()),
+                                    buf.numel() * buf.element_size(), int(n_sms),
+                                    int(stage_bytes), int(stages), int(reps), ctypes.c_void_p(st),
+                                    ctypes.byref(g))
+    _check(rc, "amk_read_ceiling")
+    return g.value
 
 
 class Decoder:

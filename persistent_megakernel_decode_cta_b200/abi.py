@@ -128,6 +128,8 @@ SIGNATURES = {
     "amk_get_error_info": (ctypes.c_int, [c_vp, ctypes.POINTER(ErrorInfo)]),
     "amk_get_workspace": (ctypes.c_int, [c_vp, ctypes.POINTER(Workspace)]),
     "amk_get_profile": (ctypes.c_int, [c_vp, ctypes.POINTER(ctypes.c_uint64), c_i64]),
+    "amk_read_ceiling": (ctypes.c_int, [c_vp, c_i64, c_i32, c_i32, c_i32, c_i32, c_vp,
+                                        ctypes.POINTER(ctypes.c_double)]),
     "amk_decode_step_noalloc": (ctypes.c_int, [c_vp, ctypes.POINTER(Weights), c_vp, c_i32,
                                                c_i32, c_vp, ctypes.POINTER(c_i32), c_vp]),
 }

@@ -64,3 +64,14 @@ def test_create_without_device_fails_cleanly():
                               ctypes.byref(h))
     assert rc == abi.ERR["AMK_ERR_NO_DEVICE"]
     assert not h.value
+
+
+def test_read_ceiling_rejects_small_buffers_on_the_host():
+    """Arguments are checked before any device work: a buffer smaller than
+    1 GiB (L2 could hold it) is refused."""
+    import ctypes
+    from persistent_megakernel_decode_cta_b200 import abi
+    g = ctypes.c_double(0.0)
+    rc = abi.lib().amk_read_ceiling(ctypes.c_void_p(1 << 20), 1 << 20, 148, 32768, 3, 1, None,
+                                    ctypes.byref(g))
+    assert rc == abi.ERR["AMK_ERR_INVALID_ARG"]
