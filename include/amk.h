@@ -143,7 +143,12 @@ typedef struct {
                                  SMs scanning from SM (level index * sm_rotate) mod n_sms,
                                  so the knob moves tiles between SMs without changing the
                                  balance; 0 (default) = always from SM 0 */
-    int32_t reserved;
+    int32_t debug_checks;     /* 1: debug checks (race-detection substitutes): amk_create
+                                 bounds-checks every resolved task record (rows within their
+                                 matrix, KV blocks within the handle's cache, chunk geometry
+                                 covering the rows) and puts a 256-byte guard of 0xA5 after
+                                 every device buffer the handle owns, which amk_check_guards
+                                 verifies after steps; 0 (default): off */
 } amk_options;
 
 typedef struct amk_handle amk_handle;
@@ -330,6 +335,14 @@ AMK_API int amk_get_workspace(amk_handle *h, amk_workspace *out);
 #define AMK_PROF_KINDS 8
 #define AMK_PROF_FIELDS 8
 AMK_API int amk_get_profile(amk_handle *h, uint64_t *out, int64_t n_u64);
+
+/* Debug checks (amk_options.debug_checks = 1): synchronises the handle's
+ * stream and reads back the guard after every device buffer the handle owns;
+ * *n_bad = the number of guards a kernel or copy wrote into (0 when every
+ * buffer stayed within its bounds): canary words in place of a race
+ * detector, so that a task writing past its buffer shows up.
+ * AMK_ERR_INVALID_ARG if the handle was created without debug checks. */
+AMK_API int amk_check_guards(amk_handle *h, int32_t *n_bad);
 
 /* After AMK_ERR_TIMEOUT: the task that gave up, the counter it waited on,
  * the value it saw and the value it needed. */

@@ -352,6 +352,13 @@ class Decoder:
         _check(abi.lib().amk_get_stats(self._h, ctypes.byref(s)), "amk_get_stats")
         return s
 
+    def check_guards(self) -> int:
+        """Guards a kernel or copy wrote into (amk_check_guards; needs
+        options.debug_checks = 1); 0 when every buffer stayed in bounds."""
+        n = abi.c_i32(-1)
+        _check(abi.lib().amk_check_guards(self._h, ctypes.byref(n)), "amk_check_guards")
+        return int(n.value)
+
     def error_info(self) -> abi.ErrorInfo:
         e = abi.ErrorInfo()
         _check(abi.lib().amk_get_error_info(self._h, ctypes.byref(e)), "amk_get_error_info")

@@ -47,7 +47,7 @@ class Options(ctypes.Structure):
                 ("debug_skip_signal_task", c_i32), ("profile", c_i32),
                 ("l2_prefetch_kb", c_i32), ("ffn_fused", c_i32),
                 ("pos0_plan", c_i32), ("inflight_kb", c_i32), ("copy_piece_kb", c_i32),
-                ("sm_rotate", c_i32), ("reserved", c_i32)]
+                ("sm_rotate", c_i32), ("debug_checks", c_i32)]
 
 
 class GraphWait(ctypes.Structure):
@@ -128,6 +128,7 @@ SIGNATURES = {
     "amk_get_error_info": (ctypes.c_int, [c_vp, ctypes.POINTER(ErrorInfo)]),
     "amk_get_workspace": (ctypes.c_int, [c_vp, ctypes.POINTER(Workspace)]),
     "amk_get_profile": (ctypes.c_int, [c_vp, ctypes.POINTER(ctypes.c_uint64), c_i64]),
+    "amk_check_guards": (ctypes.c_int, [c_vp, ctypes.POINTER(c_i32)]),
     "amk_read_ceiling": (ctypes.c_int, [c_vp, c_i64, c_i32, c_i32, c_i32, c_i32, c_vp,
                                         ctypes.POINTER(ctypes.c_double)]),
     "amk_decode_step_noalloc": (ctypes.c_int, [c_vp, ctypes.POINTER(Weights), c_vp, c_i32,

@@ -161,6 +161,10 @@ struct amk_handle {
     int device = 0;
     cudaStream_t stream = nullptr;
     std::vector<void *> dev_allocs;
+    // debug_checks: a guard of kGuardBytes after every device buffer the handle
+    // owns, filled with kGuardByte at create
+    bool guards_on = false;
+    std::vector<const void *> guards;
     TaskDesc *d_tasks = nullptr;
     int32_t *d_qoff = nullptr;
     uint32_t *d_ctr = nullptr;
@@ -202,15 +206,78 @@ int cuda_fail(cudaError_t e, const char *what)
 
 bool aligned16(const void *p) { return p && ((uintptr_t)p % 16) == 0; }
 
+constexpr size_t kGuardBytes = 256;
+constexpr int kGuardByte = 0xA5;
+
 template <typename T>
 int dalloc(amk_handle *H, T **out, size_t bytes)
 {
     void *p = nullptr;
-    cudaError_t e = cudaMalloc(&p, bytes ? bytes : 16);
+    bytes = bytes ? bytes : 16;
+    const size_t body = (bytes + 15) & ~(size_t)15;
+    cudaError_t e = cudaMalloc(&p, H->guards_on ? body + kGuardBytes : bytes);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaMalloc");
     H->dev_allocs.push_back(p);
+    if (H->guards_on) {
+        uint8_t *g = static_cast<uint8_t *>(p) + body;
+        if ((e = cudaMemset(g, kGuardByte, kGuardBytes)) != cudaSuccess)
+            return cuda_fail(e, "guard fill");
+        H->guards.push_back(g);
+    }
     *out = static_cast<T *>(p);
+    return AMK_OK;
+}
+
+// Debug bounds check of resolved task records (amk_options.debug_checks):
+// every GEMV tile's rows lie within its matrix, its chunk geometry covers
+// them, and every attention tile's KV blocks lie within the handle's cache.
+int check_task_records(const amk_plan *P, const std::vector<TaskDesc> &ts, const uint16_t *kv,
+                       size_t kv_bytes)
+{
+    const amk_config &c = P->cfg;
+    const int hq = c.n_heads * c.head_dim, hk = c.n_kv_heads * c.head_dim;
+    for (size_t i = 0; i < ts.size(); ++i) {
+        const TaskDesc &d = ts[i];
+        auto bad = [&](const char *what) {
+            return amk_set_error(AMK_ERR_VALIDATION, "debug check: task %zu (kind %d, layer %d): %s",
+                                 i, d.kind, d.layer, what);
+        };
+        if (d.layer < 0 || d.layer >= c.n_layers)
+            return bad("layer out of range");
+        if (d.kind == amk::TK_ATTN) {
+            const uint8_t *lo = reinterpret_cast<const uint8_t *>(kv);
+            const size_t blk = (size_t)c.max_ctx * c.head_dim * 2;
+            for (const void *w : {d.w0, d.w1}) {
+                const uint8_t *q = static_cast<const uint8_t *>(w);
+                if (q < lo || q + blk > lo + kv_bytes)
+                    return bad("KV block outside the cache");
+            }
+            if (d.r0 < 0 || d.r0 >= c.n_kv_heads || d.r1 < 0 || d.r1 >= P->opt.attn_splits)
+                return bad("attention head or chunk out of range");
+            continue;
+        }
+        int rows = c.hidden;
+        switch (d.kind) {
+        case amk::TK_QKV: rows = d.mat == 0 ? hq : hk; break;
+        case amk::TK_GATEUP: case amk::TK_FFN: rows = c.ffn; break;
+        case amk::TK_LMHEAD: rows = c.vocab; break;
+        default: break;  // OPROJ, DOWN: hidden rows
+        }
+        const int R = d.r1 - d.r0;
+        if (d.r0 < 0 || R <= 0 || d.r1 > rows || R > amk::kMaxTaskRows)
+            return bad("row range outside the matrix or above the task limit");
+        if (!d.w0 || d.rpc == 0 || d.nck == 0 || (int)d.nck * d.rpc < R ||
+            ((int)d.nck - 1) * d.rpc >= R)
+            return bad("chunk geometry does not cover the rows exactly");
+        const int parts = (d.kind == amk::TK_GATEUP || d.kind == amk::TK_FFN) ? 2 : 1;
+        if (d.ngu != d.nck * parts ||
+            d.nchunks != d.ngu + (d.kind == amk::TK_FFN ? d.nck2 : 0) ||
+            (1 << d.ks_log2) * (1 << d.rg_log2) != amk::kConsumerWarps || d.rpc % (1 << d.rg_log2))
+            return bad("chunk or warp geometry inconsistent");
+        if (d.kind == amk::TK_FFN && ((int)d.nck2 * d.rpc2 < c.hidden || d.ncb == 0))
+            return bad("fused FFN Wdown chunks do not cover hidden");
+    }
     return AMK_OK;
 }
 
@@ -334,6 +401,7 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
         return amk_set_error(AMK_ERR_OOM, "amk_create: out of host memory");
     cudaGetDevice(&H->device);
     H->stream = static_cast<cudaStream_t>(cuda_stream);
+    H->guards_on = opt && opt->debug_checks > 0;
     int sms = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, H->device);
     int n_sms = (opt && opt->n_sms > 0) ? opt->n_sms : sms;
@@ -466,6 +534,10 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
             return cuda_fail(e, "pack Wdown");
         }
     }
+    if (H->guards_on && (rc = check_task_records(P, resolved, H->d_kv, H->kv_bytes)) != AMK_OK) {
+        free_handle(H);
+        return rc;
+    }
     if ((e = cudaMemcpyAsync(H->d_tasks, resolved.data(), sizeof(TaskDesc) * resolved.size(),
                              cudaMemcpyHostToDevice, H->stream)) != cudaSuccess ||
         (e = cudaMemcpyAsync(H->d_qoff, P->queue_off.data(),
@@ -477,6 +549,11 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     std::vector<TaskDesc> resolved0(P->pos0 ? P->pos0->tasks.size() : 0);
     for (size_t t = 0; t < resolved0.size(); ++t)
         amk_resolve_task(P->pos0, wr, H->d_kv, (int)t, &resolved0[t], P->pos0->ffn_fused ? 1 : 0);
+    if (H->guards_on && P->pos0 &&
+        (rc = check_task_records(P->pos0, resolved0, H->d_kv, H->kv_bytes)) != AMK_OK) {
+        free_handle(H);
+        return rc;
+    }
     if (P->pos0 &&
         ((e = cudaMemcpyAsync(H->d_tasks0, resolved0.data(), sizeof(TaskDesc) * resolved0.size(),
                               cudaMemcpyHostToDevice, H->stream)) != cudaSuccess ||
@@ -770,6 +847,33 @@ extern "C" int amk_get_profile(amk_handle *h, uint64_t *out, int64_t n_u64)
         e = cudaStreamSynchronize(h->stream);
     if (e != cudaSuccess)
         return cuda_fail(e, "amk_get_profile");
+    return AMK_OK;
+}
+
+extern "C" int amk_check_guards(amk_handle *h, int32_t *n_bad)
+{
+    if (!h || !n_bad)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_check_guards: NULL argument");
+    if (!h->guards_on)
+        return amk_set_error(AMK_ERR_INVALID_ARG, "amk_check_guards: the handle was created "
+                             "without debug_checks");
+    cudaError_t e = cudaStreamSynchronize(h->stream);
+    int32_t bad = 0;
+    std::vector<uint8_t> buf(kGuardBytes);
+    for (const void *g : h->guards) {
+        if (e == cudaSuccess)
+            e = cudaMemcpy(buf.data(), g, kGuardBytes, cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess)
+            break;
+        for (uint8_t v : buf)
+            if (v != (uint8_t)kGuardByte) {
+                ++bad;
+                break;
+            }
+    }
+    if (e != cudaSuccess)
+        return cuda_fail(e, "amk_check_guards");
+    *n_bad = bad;
     return AMK_OK;
 }
 

@@ -91,6 +91,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         if (opt_in->inflight_kb != 0) opt.inflight_kb = opt_in->inflight_kb;
         if (opt_in->copy_piece_kb > 0) opt.copy_piece_kb = opt_in->copy_piece_kb;
         if (opt_in->sm_rotate > 0) opt.sm_rotate = opt_in->sm_rotate;
+        opt.debug_checks = opt_in->debug_checks;
         opt.n_sms = opt_in->n_sms;
     }
     const amk_config &c = *cfg;

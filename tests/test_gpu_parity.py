@@ -330,3 +330,25 @@ def test_wait_timeout_is_reported_and_recoverable():
     good = Pair(cfg, weights=pair.w, options=amk.default_options(n_sms=4))
     g, am, ref, ref_am = good.step(3, 0)
     compare(cfg, g, am, ref, ref_am, "after timeout")
+
+
+@pytest.mark.parametrize("name,ctx,steps", [
+    ("tiny", 0, 12),          # split FFN levels, attention at every position up to 11
+    ("smol135", 120, 6),      # fused FFN level, several split-K attention chunks
+    ("llama1b_w8", 500, 3),   # int8, long cache
+])
+def test_debug_checks_keep_every_buffer_in_bounds(name, ctx, steps):
+    """With debug checks on, amk_create bounds-checks every task record, and
+    after several steps (parity-checked) no kernel or copy has written into
+    the guard after any of the handle's device buffers."""
+    cfg = si.get_config(name)
+    pair = Pair(cfg, options=amk.default_options(debug_checks=1))
+    if ctx:
+        pair.fill_kv(ctx)
+    prompt = si.make_prompt(cfg, steps)
+    for i, t in enumerate(prompt):
+        g, am, ref, ref_am = pair.step(t, ctx + i)
+        compare(cfg, g, am, ref, ref_am, what=f"{name} debug pos {ctx + i}")
+    assert pair.dec.check_guards() == 0
+    del pair
+    torch.cuda.empty_cache()
