@@ -259,7 +259,9 @@ def phase_shares(P):
     P = P.astype(np.float64)
     total = float((P[:, 0, 1] - P[:, 0, 0]).sum())
     prod = float((P[:, 0, 3] - P[:, 0, 0]).sum())
-    wait = float(P[:, 1:, 1].sum())
+    # waits for a task's inputs: counter polls (field 1) or, with flagged
+    # waits, thread 0's polls of the flagged words (field 3)
+    wait = float(P[:, 1:, 1].sum()) + float(P[:, 1:, 3].sum())
     prologue = float(P[:, 1:, 2].sum())
     ring = float(P[:, 1:, 6].sum()) / 8.0
     compute = float(P[:, 1:, 7].sum()) / 8.0
@@ -271,14 +273,14 @@ def phase_shares(P):
         if n == 0:
             continue
         f = P[:, k, :].sum(axis=0) / n / 1e3
-        per_kind[name] = {"tasks": int(n), "counter_wait_us": f[1], "prologue_us": f[2],
+        per_kind[name] = {"tasks": int(n), "counter_wait_us": f[1] + f[3], "prologue_us": f[2],
                           "ring_wait_us": f[6] / 8.0, "gemv_or_attention_us": f[7] / 8.0,
                           "epilogue_release_us": f[5], "run_us": f[4]}
     return {
         "counter_wait": wait / total, "prologue": prologue / total,
         "ring_wait": ring / total, "gemv_or_attention": compute / total,
         "epilogue_release": epi / total,
-        "other": max(0.0, 1.0 - (wait + run) / total),
+        "other": max(0.0, 1.0 - (float(P[:, 1:, 1].sum()) + run) / total),
         "producer_stalled": float(P[:, 0, 2].sum()) / prod if prod > 0 else None,
         "per_task_kind_us": per_kind,
         "how": "phase timers (globaltimer) of one profiled step after the timed region; "
@@ -504,7 +506,9 @@ def run_ours(args):
             "clocks": clocks.summary(),
             "schedule": {"tasks": st.n_tasks, "ctas": st.n_sms, "ring_stages": st.ring_stages,
                          "stage_bytes": st.stage_bytes, "attn_splits": st.attn_splits,
-                         "smem_bytes": st.smem_bytes, "threads_per_cta": st.threads_per_cta},
+                         "smem_bytes": st.smem_bytes, "threads_per_cta": st.threads_per_cta,
+                         "waits": "flagged words" if st.flagged_waits else "level counters",
+                         "ffn_fused": bool(st.ffn_fused)},
         }
         if parity["verdict"] != "PASS":
             line["value"] = None

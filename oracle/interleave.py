@@ -9,18 +9,24 @@ algorithm: it executes the schedule's semantics.
 Semantics (tasks are atomic):
   * SM s runs its queue in order; the head task may run once, for every
     (counter, t) it waits on, the number of finished signals to that counter
-    is >= t.  Running it adds 1 per signal.
+    is >= t, and, for every READ_FLAGGED range it has, every task with a
+    WRITE or ACCUM overlapping that range has finished (a flagged word takes
+    the epoch's tag from its one writer, or when its accumulation is done; a
+    task that writes what it flag-reads never runs).  Running it adds 1 per
+    signal.
   * A state is the set of finished tasks.  All reachable states are
     enumerated from the empty set.
   * Deadlock: a reachable state with unfinished tasks and no runnable head.
   * "a always before b": no reachable state contains b but not a.
 Verdicts, on overlapping accesses of different tasks:
-  READ needs every WRITE/ACCUM always before it; WRITE/WRITE, WRITE/ACCUM and
+  READ (and READ_FLAGGED) needs every WRITE/ACCUM always before it; WRITE/WRITE, WRITE/ACCUM and
   RESET/RESET need one fixed order; READ_PREV needs to be always before every
   WRITE/ACCUM/RESET; RESET needs every other access always before it.
 The purely syntactic conditions (ids and ranges, thresholds 1 <= t <= number
-of producers, full-count waits on shared counters, outputs written, reset
-coverage of double-buffered accumulators) are definitions, checked as written.
+of producers, full-count waits on shared counters, every element of a
+READ_FLAGGED range written exactly once or only accumulated, outputs written,
+reset coverage of double-buffered accumulators) are definitions, checked as
+written.
 
 Graph format (plain Python): {
   "n_counters": int,
@@ -28,13 +34,13 @@ Graph format (plain Python): {
   "tasks": [{"sm": int, "waits": [(ctr, t)], "signals": [ctr],
              "accesses": [(buf, kind, begin, end)]}],
   "queues": [[task ids in order] per SM]}
-kinds: 0 READ, 1 WRITE, 2 ACCUM, 3 READ_PREV, 4 RESET.
+kinds: 0 READ, 1 WRITE, 2 ACCUM, 3 READ_PREV, 4 RESET, 5 READ_FLAGGED.
 """
 from __future__ import annotations
 
 from typing import Dict, List, Tuple
 
-READ, WRITE, ACCUM, READ_PREV, RESET = range(5)
+READ, WRITE, ACCUM, READ_PREV, RESET, READ_FLAGGED = range(6)
 
 
 def _syntax(g) -> str:
@@ -61,7 +67,8 @@ def _syntax(g) -> str:
             if not (0 <= c < C):
                 return "V7"
         for (b, k, lo, hi) in task["accesses"]:
-            if not (0 <= b < B) or k not in (READ, WRITE, ACCUM, READ_PREV, RESET):
+            if not (0 <= b < B) or k not in (READ, WRITE, ACCUM, READ_PREV, RESET,
+                                             READ_FLAGGED):
                 return "V7"
             if lo < 0 or hi <= lo or hi > bufs[b]["size"]:
                 return "V7"
@@ -77,7 +84,38 @@ def _syntax(g) -> str:
         for c, t in task["waits"]:
             if nprod[c] > 1 and t != nprod[c]:
                 return "V3"
+    # V10: each flagged-read element has exactly one value to wait for
+    for task in g["tasks"]:
+        for (b, k, lo, hi) in task["accesses"]:
+            if k != READ_FLAGGED:
+                continue
+            for x in range(lo, hi):
+                nw = na = 0
+                for other in g["tasks"]:
+                    for (b2, k2, lo2, hi2) in other["accesses"]:
+                        if b2 == b and lo2 <= x < hi2:
+                            nw += k2 == WRITE
+                            na += k2 == ACCUM
+                if not ((nw == 1 and na == 0) or (nw == 0 and na >= 1)):
+                    return "V10"
     return ""
+
+
+def _flag_deps(g):
+    """Per task, the tasks whose WRITE/ACCUM its READ_FLAGGED ranges wait for."""
+    tasks = g["tasks"]
+    deps = []
+    for task in tasks:
+        d = set()
+        for (b, k, lo, hi) in task["accesses"]:
+            if k != READ_FLAGGED:
+                continue
+            for w, other in enumerate(tasks):
+                for (b2, k2, lo2, hi2) in other["accesses"]:
+                    if b2 == b and k2 in (WRITE, ACCUM) and lo2 < hi and lo < hi2:
+                        d.add(w)
+        deps.append(d)
+    return deps
 
 
 def _post_syntax(g) -> str:
@@ -108,6 +146,7 @@ def _reachable(g) -> Tuple[List[int], bool]:
     tasks, queues = g["tasks"], g["queues"]
     T = len(tasks)
     full = (1 << T) - 1
+    fdeps = _flag_deps(g)
     start = 0
     seen = {start}
     stack = [start]
@@ -124,7 +163,8 @@ def _reachable(g) -> Tuple[List[int], bool]:
             head = next((t for t in q if not st >> t & 1), None)
             if head is None:
                 continue
-            if all(counts.get(c, 0) >= th for c, th in tasks[head]["waits"]):
+            if (all(counts.get(c, 0) >= th for c, th in tasks[head]["waits"])
+                    and all(st >> w & 1 for w in fdeps[head])):
                 moved = True
                 nxt = st | (1 << head)
                 if nxt not in seen:
@@ -137,7 +177,7 @@ def _reachable(g) -> Tuple[List[int], bool]:
 
 def check(g) -> Tuple[bool, str]:
     """(accepted, reason) with reason in {"ok", "V2", "V3", "V7", "V8", "V9",
-    "deadlock", "race"}."""
+    "V10", "deadlock", "race"}."""
     r = _syntax(g)
     if r:
         return False, r
@@ -168,7 +208,7 @@ def check(g) -> Tuple[bool, str]:
             tb, bb, kb, lb, hb = accs[j]
             if ta == tb or ba != bb or not (la < hb and lb < ha):
                 continue
-            if ka == READ and kb in (WRITE, ACCUM) and not always_before(tb, ta):
+            if ka in (READ, READ_FLAGGED) and kb in (WRITE, ACCUM) and not always_before(tb, ta):
                 return False, "race"
             if (((ka == WRITE and kb in (WRITE, ACCUM)) or (ka == RESET and kb == RESET))
                     and not (always_before(ta, tb) or always_before(tb, ta))):

@@ -325,14 +325,16 @@ class Decoder:
 
     def workspace(self) -> Dict[str, object]:
         """fp32 views of the last step's activations: qkv [L, qkv_rows],
-        xmid / xout [L, hidden], act [L, ffn]."""
+        xmid / xout [L, hidden], act [L, ffn] (the value halves of the
+        flagged words)."""
         import torch
         ws = abi.Workspace()
         _check(abi.lib().amk_get_workspace(self._h, ctypes.byref(ws)), "amk_get_workspace")
         L = self.cfg.n_layers
 
         def view(p, n):
-            return torch.as_tensor(_DevArray(p, (L, n), "<f4"), device="cuda")
+            w = torch.as_tensor(_DevArray(p, (L, n, 2), "<f4"), device="cuda")
+            return w[:, :, 0]
 
         return {"qkv": view(ws.qkv, ws.qkv_rows), "xmid": view(ws.xmid, self.cfg.hidden),
                 "xout": view(ws.xout, self.cfg.hidden), "act": view(ws.act, self.cfg.ffn)}

@@ -21,10 +21,10 @@ STATUS = {
 }
 ERR = {v: k for k, v in STATUS.items()}
 QUANT_BF16, QUANT_W8A16, QUANT_W4A16 = 0, 1, 2
-ACC_READ, ACC_WRITE, ACC_ACCUM, ACC_READ_PREV, ACC_RESET = range(5)
+ACC_READ, ACC_WRITE, ACC_ACCUM, ACC_READ_PREV, ACC_RESET, ACC_READ_FLAGGED = range(6)
 BUF_OUTPUT = 1
 RULES = {0: "ok", 1: "V1", 2: "V2", 3: "V3", 4: "V4", 5: "V5", 6: "V6", 7: "V7",
-         8: "V8", 9: "V9"}
+         8: "V8", 9: "V9", 10: "V10"}
 
 
 class Config(ctypes.Structure):
@@ -47,7 +47,7 @@ class Options(ctypes.Structure):
                 ("debug_skip_signal_task", c_i32), ("profile", c_i32),
                 ("l2_prefetch_kb", c_i32), ("ffn_fused", c_i32),
                 ("pos0_plan", c_i32), ("inflight_kb", c_i32), ("copy_piece_kb", c_i32),
-                ("sm_rotate", c_i32), ("debug_checks", c_i32)]
+                ("sm_rotate", c_i32), ("debug_checks", c_i32), ("flagged_waits", c_i32)]
 
 
 class GraphWait(ctypes.Structure):
@@ -88,7 +88,8 @@ class PlanStats(ctypes.Structure):
     _fields_ = [("n_tasks", c_i32), ("n_counters", c_i32), ("n_sms", c_i32),
                 ("ring_stages", c_i32), ("stage_bytes", c_i32), ("attn_splits", c_i32),
                 ("smem_bytes", c_i32), ("threads_per_cta", c_i32),
-                ("weight_bytes", c_i64), ("kv_row_bytes", c_i64), ("epoch", c_i64)]
+                ("weight_bytes", c_i64), ("kv_row_bytes", c_i64), ("epoch", c_i64),
+                ("flagged_waits", c_i32), ("ffn_fused", c_i32)]
 
 
 class ErrorInfo(ctypes.Structure):

@@ -87,6 +87,7 @@ extern "C" int amk_default_options(amk_options *o)
     o->debug_skip_signal_task = -1;
     o->ffn_fused = 1;
     o->pos0_plan = 1;
+    o->flagged_waits = 1;
     return AMK_OK;
 }
 
@@ -174,9 +175,10 @@ struct amk_handle {
     uint32_t *d_ctr0 = nullptr;
     uint32_t epoch0 = 0;  // steps run with it since the last reset
     ErrorWord *d_err = nullptr;
-    float *d_qkv = nullptr, *d_part = nullptr, *d_attn = nullptr, *d_xmid = nullptr,
-          *d_xout = nullptr;
-    float *d_act = nullptr, *d_logits = nullptr;
+    uint64_t *d_qkv = nullptr, *d_attn = nullptr, *d_xmid = nullptr, *d_xout = nullptr,
+             *d_act = nullptr;  // flagged words
+    float *d_part = nullptr, *d_logits = nullptr;
+    uint32_t tag = 0;  // tag of the last step's flagged words (0: none yet)
     unsigned long long *d_argkey = nullptr;
     long long *d_xacc = nullptr;    // [L][h] fixed-point residual (fused FFN)
     void *d_act_block = nullptr;    // every activation buffer, one allocation
@@ -184,7 +186,7 @@ struct amk_handle {
     void *d_q4 = nullptr;           // W4A16: every int4 matrix as rows of codes + scales
     unsigned long long *d_prof = nullptr;
     uint16_t *d_kv = nullptr;
-    size_t kv_bytes = 0, act_bytes = 0;
+    size_t kv_bytes = 0, act_bytes = 0, fw_bytes = 0;  // fw: the flagged words from d_qkv
     ErrorWord *h_err = nullptr;            // pinned
     unsigned long long *h_key = nullptr;   // pinned
     cudaEvent_t err_ev = nullptr;
@@ -354,6 +356,7 @@ int zero_state(amk_handle *H)
         return cuda_fail(e, "amk_reset_kv");
     H->epoch = 0;
     H->epoch0 = 0;
+    H->tag = 0;  // the flagged words were cleared with the block above
     H->arrive_base = 0;
     H->poisoned = false;
     H->err_pending = false;
@@ -437,9 +440,12 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     const size_t attn_f = (size_t)L * c.n_heads * hd;
     const size_t h_f = (size_t)L * c.hidden, act_f = (size_t)L * c.ffn;
     H->kv_bytes = (size_t)L * 2 * nkv * c.max_ctx * hd * sizeof(uint16_t);
-    // activations in one block: xacc (int64) | qkv | part | attn | xmid | xout | act
+    // activations in one block: xacc (int64) | qkv | attn | xmid | xout | act
+    // (flagged words, 8 bytes each) | part (fp32)
     const size_t xacc_b = P->ffn_fused ? (size_t)L * c.hidden * sizeof(long long) : 0;
-    H->act_bytes = xacc_b + (qkv_f + part_f + attn_f + 2 * h_f + act_f) * sizeof(float);
+    const size_t words = qkv_f + attn_f + 2 * h_f + act_f;
+    H->fw_bytes = words * sizeof(uint64_t);
+    H->act_bytes = xacc_b + H->fw_bytes + part_f * sizeof(float);
     float *act_block = nullptr;
     if ((rc = dalloc(H, &H->d_tasks, sizeof(TaskDesc) * P->tasks.size())) ||
         (rc = dalloc(H, &H->d_qoff, sizeof(int32_t) * P->queue_off.size())) ||
@@ -463,12 +469,12 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     }
     H->d_act_block = act_block;
     H->d_xacc = P->ffn_fused ? reinterpret_cast<long long *>(act_block) : nullptr;
-    H->d_qkv = reinterpret_cast<float *>(reinterpret_cast<char *>(act_block) + xacc_b);
-    H->d_part = H->d_qkv + qkv_f;
-    H->d_attn = H->d_part + part_f;
+    H->d_qkv = reinterpret_cast<uint64_t *>(reinterpret_cast<char *>(act_block) + xacc_b);
+    H->d_attn = H->d_qkv + qkv_f;
     H->d_xmid = H->d_attn + attn_f;
     H->d_xout = H->d_xmid + h_f;
     H->d_act = H->d_xout + h_f;
+    H->d_part = reinterpret_cast<float *>(H->d_act + act_f);
     if ((e = cudaMallocHost(&H->h_err, sizeof(ErrorWord))) != cudaSuccess ||
         (e = cudaMallocHost(&H->h_key, 2 * sizeof(unsigned long long))) != cudaSuccess ||
         (e = cudaEventCreateWithFlags(&H->err_ev, cudaEventDisableTiming)) != cudaSuccess) {
@@ -617,6 +623,7 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     k.generic = P->generic;
     k.timeout_ns = (uint64_t)P->opt.wait_timeout_us * 1000ull;
     k.skip_signal_task = P->opt.debug_skip_signal_task;
+    k.flagged = P->flagged;
     k.lookahead = (uint32_t)std::max(0, P->opt.l2_prefetch_kb) * 1024u;
     k.inflight = amk_inflight_bytes(&P->opt);
     k.piece = amk_piece_bytes(&P->opt);
@@ -684,6 +691,15 @@ int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev,
     }
     k.arrive_base = H->arrive_base;
     k.parity = (int32_t)(H->epoch & 1u);
+    // a fresh tag per step; when the 32-bit tag runs out, every flagged word
+    // is cleared (stream-ordered before this launch) and the tags start over
+    if (H->tag == 0xFFFFFFFFu) {
+        cudaError_t ce = cudaMemsetAsync(H->d_qkv, 0, H->fw_bytes, H->stream);
+        if (ce != cudaSuccess)
+            return cuda_fail(ce, "flagged words clear");
+        H->tag = 0;
+    }
+    k.tag = H->tag + 1;
     if (logits_dev)
         k.logits = logits_dev;
     if (H->d_prof) {
@@ -702,6 +718,7 @@ int launch_step(amk_handle *H, int32_t token_id, int32_t pos, float *logits_dev,
                              "cooperative launch: %s", cudaGetErrorString(e));
     }
     H->epoch += 1;
+    H->tag += 1;
     if (at0)
         H->epoch0 += 1;
     {  // non-empty attention chunks of this step: each arrives once unless alone
@@ -808,6 +825,8 @@ extern "C" int amk_plan_get_stats(const amk_plan *P, amk_plan_stats *o)
     o->threads_per_cta = amk::kThreads;
     o->weight_bytes = P->weight_bytes;
     o->kv_row_bytes = P->kv_row_bytes;
+    o->flagged_waits = P->flagged;
+    o->ffn_fused = P->ffn_fused;
     return AMK_OK;
 }
 

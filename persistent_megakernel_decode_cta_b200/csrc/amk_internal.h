@@ -134,13 +134,15 @@ struct KParams {
     ErrorWord *err;
     // weights (the per-task pointers live in the task records)
     const uint16_t *embed;
-    // state and activations (fp32 unless noted)
-    float *qkv;       // [L][qkv_rows]: q | k | v, before RoPE
+    // state and activations.  The vectors one level hands to the next are
+    // flagged words: 64 bits each, the fp32 value in the low half and the tag
+    // of the step that wrote it in the high half (see fw_st in the kernel)
+    uint64_t *qkv;    // [L][qkv_rows]: q | k | v, before RoPE (flagged)
     float *part;      // [L][nkv][C][G][hd + 2]: split-K partials (m, l, o[hd])
-    float *attn;      // [L][nh * hd]: attention output (the chunks merged)
-    float *xmid;      // [L][h]: residual after attention
-    float *xout;      // [L][h]: residual after the FFN
-    float *act;       // [L][ffn]: SwiGLU activations
+    uint64_t *attn;   // [L][nh * hd]: attention output, the chunks merged (flagged)
+    uint64_t *xmid;   // [L][h]: residual after attention (flagged)
+    uint64_t *xout;   // [L][h]: residual after the FFN (flagged)
+    uint64_t *act;    // [L][ffn]: SwiGLU activations (flagged)
     long long *xacc;  // [L][h]: residual after the FFN in fixed point (value * 2^32), when
                       // the FFN level is fused: OPROJ writes the residual, FFN slices add
     const void *dmaps;  // [L] 128-byte tensor maps of Wdown (fused FFN), 64-byte aligned
@@ -172,7 +174,11 @@ struct KParams {
     uint32_t piece;             // bytes of a copy piece (multiple of 16)
     int32_t att_chunk;          // positions per split-K attention chunk at this step
     int32_t att_P;              // KV positions per ring stage (stage_bytes / (4 head_dim))
-    int32_t skip_signal_task;   // test hook, -1 = off
+    int32_t skip_signal_task;   // test hook, -1 = off (with flagged waits: that task's
+                                // flagged words carry a wrong tag)
+    uint32_t tag;               // this step's tag in the flagged words (never 0)
+    int32_t flagged;            // 1: tasks wait on the flagged words they read instead of
+                                // level counters, and signal no counter (FFN levels split)
     unsigned long long *prof;   // [n_sms][kProfKinds][kProfFields] phase timers, or null
 };
 constexpr int kProfKinds = AMK_PROF_KINDS;

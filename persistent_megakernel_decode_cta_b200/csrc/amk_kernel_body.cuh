@@ -152,6 +152,34 @@ __device__ __forceinline__ void red_release_add(uint32_t *p, uint32_t v)
 {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+constexpr int kFwRoundWords = 48;  // flagged words a GEMV lane loads in one round
+// Flagged words carry a value from one level to the next: the fp32 value in
+// the low half and the tag of the step that wrote it in the high half of one
+// aligned 64-bit word, stored and loaded as single relaxed accesses at GPU
+// scope (each is single-copy atomic).  A reader that finds its step's tag
+// holds that step's value, so the writer issues no fence before its readers
+// may go on, and a reader's poll of the data is its whole wait.
+__device__ __forceinline__ void fw_st(uint64_t *a, float v, uint32_t tag)
+{
+    const uint64_t w = ((uint64_t)tag << 32) | (uint64_t)__float_as_uint(v);
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(a), "l"(w) : "memory");
+}
+__device__ __forceinline__ uint64_t fw_ld(const uint64_t *a)
+{
+    uint64_t w;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(a) : "memory");
+    return w;
+}
+// two consecutive words (16-byte aligned), each loaded as its own access
+__device__ __forceinline__ void fw_ld2(const uint64_t *a, uint64_t &x, uint64_t &y)
+{
+    asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];"
+                 : "=l"(x), "=l"(y)
+                 : "l"(a)
+                 : "memory");
+}
+__device__ __forceinline__ float fw_val(uint64_t w) { return __uint_as_float((uint32_t)w); }
+__device__ __forceinline__ bool fw_ok(uint64_t w, uint32_t tag) { return (uint32_t)(w >> 32) == tag; }
 // The residual after a fused FFN level is held in fixed point (value * 2^32
 // in an int64): integer addition is associative, so the FFN slices' partial
 // down projections add up to the same bits in any order.  |value| < 2^31.
@@ -866,6 +894,233 @@ __device__ void record_error(const KParams &p, uint32_t code, int task, int ctr,
     }
 }
 
+// A flagged read gives up on an abort of this CTA, on an error another SM
+// recorded, or after the wait limit, which it records (code 1, no counter;
+// seen = the tag it last found, target = this step's).  s.flags[2] holds the
+// index of the CTA's current task.
+__device__ __forceinline__ void fw_record_timeout(const KParams &p, const SmemLayout &s,
+                                               uint64_t last)
+{
+    record_error(p, 1u, *reinterpret_cast<volatile int *>(s.flags + 2), -1,
+                 (uint32_t)(last >> 32), p.tag);
+}
+__device__ __forceinline__ bool fw_give_up(const KParams &p, const SmemLayout &s, uint64_t t0,
+                                           uint64_t last, uint32_t it)
+{
+    if (*reinterpret_cast<volatile int *>(s.flags) != 0 || ld_relaxed(&p.err->code) != 0u)
+        return true;
+    if (gtimer() - t0 > p.timeout_ns || it > (1u << 26)) {
+        fw_record_timeout(p, s, last);
+        return true;
+    }
+    return false;
+}
+
+// Phase timers: consumer thread 0 adds the time it spent polling flagged
+// words past the first load (the task's wait for its inputs) to a 64-bit
+// slot at s.flags + 4, which the consumer loop clears at each task.
+__device__ __forceinline__ void fw_note(const KParams &p, const SmemLayout &s, uint64_t t0)
+{
+    if (p.prof && threadIdx.x == kProducerThreads) {
+        volatile unsigned long long *a =
+            reinterpret_cast<volatile unsigned long long *>(s.flags + 4);
+        *a = *a + (gtimer() - t0);
+    }
+}
+
+// Thread ct's elements i = ct + 256 j (j < NJ, i < n) of a flagged vector:
+// all loads go out at once, then the words still without this step's tag are
+// loaded again, all at once, until every one has it.  False when the read
+// gave up (the caller raises the CTA's abort flag before its next barrier).
+template <int NJ>
+__device__ __forceinline__ bool fw_read_strided(const KParams &p, const SmemLayout &s,
+                                                const uint64_t *src, int n, int ct,
+                                                float (&xv)[NJ])
+{
+    static_assert(NJ <= 32, "pending bits");
+    const uint32_t tag = p.tag;
+    uint64_t w[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+        const int i = ct + j * kConsumerThreads;
+        w[j] = i < n ? fw_ld(src + i) : (uint64_t)tag << 32;
+    }
+    uint32_t pend = 0u;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+        xv[j] = fw_val(w[j]);
+        if (!fw_ok(w[j], tag))
+            pend |= 1u << j;
+    }
+    uint64_t t0 = 0;
+    // (the words are usually there by the first load once the task's inputs
+    // are complete; the compiler is told so, to keep this loop out of the
+    // straight-line code)
+    for (uint32_t it = 0; __builtin_expect(pend != 0u, 0); ++it) {
+        if (it == 0)
+            t0 = gtimer();
+#pragma unroll
+        for (int j = 0; j < NJ; ++j)
+            if (pend & (1u << j))
+                w[j] = fw_ld(src + ct + j * kConsumerThreads);
+        uint64_t last = 0;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            if (pend & (1u << j)) {
+                if (fw_ok(w[j], tag)) {
+                    xv[j] = fw_val(w[j]);
+                    pend &= ~(1u << j);
+                } else {
+                    last = w[j];
+                }
+            }
+        }
+        if (pend && (it & 15) == 15 && fw_give_up(p, s, t0, last, it))
+            return false;
+    }
+    if (t0)
+        fw_note(p, s, t0);
+    return true;
+}
+
+// The words at a[j] (null: none, value 0) of flagged vectors, as above.
+template <int N>
+__device__ __forceinline__ bool fw_gather(const KParams &p, const SmemLayout &s,
+                                          const uint64_t *const (&a)[N], float (&v)[N])
+{
+    const uint32_t tag = p.tag;
+    uint64_t w[N];
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+        w[j] = a[j] ? fw_ld(a[j]) : (uint64_t)tag << 32;
+    uint32_t pend = 0u;
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+        v[j] = fw_val(w[j]);
+        if (!fw_ok(w[j], tag))
+            pend |= 1u << j;
+    }
+    uint64_t t0 = 0;
+    // (the words are usually there by the first load once the task's inputs
+    // are complete; the compiler is told so, to keep this loop out of the
+    // straight-line code)
+    for (uint32_t it = 0; __builtin_expect(pend != 0u, 0); ++it) {
+        if (it == 0)
+            t0 = gtimer();
+#pragma unroll
+        for (int j = 0; j < N; ++j)
+            if (pend & (1u << j))
+                w[j] = fw_ld(a[j]);
+        uint64_t last = 0;
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            if (pend & (1u << j)) {
+                if (fw_ok(w[j], tag)) {
+                    v[j] = fw_val(w[j]);
+                    pend &= ~(1u << j);
+                } else {
+                    last = w[j];
+                }
+            }
+        }
+        if (pend && (it & 15) == 15 && fw_give_up(p, s, t0, last, it))
+            return false;
+    }
+    if (t0)
+        fw_note(p, s, t0);
+    return true;
+}
+
+// A GEMV lane's activations from a flagged vector: vector v = vb + lane +
+// 32 i (i < ni; zeros for the others) holds the E elements at xg + v E, read
+// two words at a time.  The vectors go in rounds of RI (a round's raw words
+// take two registers each, so a lane with 64 activations reads them in two
+// rounds); every load of a round goes out before any word of it is looked at.
+template <int NI, int E, int RI>
+__device__ __forceinline__ bool fw_lane_round(const KParams &p, const SmemLayout &s,
+                                              const uint64_t *xg, int vb, int ni, int lane,
+                                              int i0, float (&xf)[NI][E])
+{
+    constexpr int H = E / 2;
+    static_assert(RI * H <= 32, "pending bits");
+    const uint32_t tag = p.tag;
+    uint64_t wa[RI][H], wb[RI][H];
+    const uint64_t none = (uint64_t)tag << 32;  // a zero with this step's tag
+#pragma unroll
+    for (int r = 0; r < RI; ++r) {
+        const int i = i0 + r;
+        const uint64_t *vp = xg + (size_t)(vb + lane + 32 * i) * E;
+#pragma unroll
+        for (int e = 0; e < H; ++e) {
+            wa[r][e] = wb[r][e] = none;
+            if (i < ni)
+                fw_ld2(vp + 2 * e, wa[r][e], wb[r][e]);
+        }
+    }
+    uint32_t pend = 0u;
+#pragma unroll
+    for (int r = 0; r < RI; ++r)
+#pragma unroll
+        for (int e = 0; e < H; ++e) {
+            xf[i0 + r][2 * e] = fw_val(wa[r][e]);
+            xf[i0 + r][2 * e + 1] = fw_val(wb[r][e]);
+            if (!fw_ok(wa[r][e], tag) || !fw_ok(wb[r][e], tag))
+                pend |= 1u << (r * H + e);
+        }
+    uint64_t t0 = 0;
+    // (the words are usually there by the first load once the task's inputs
+    // are complete; the compiler is told so, to keep this loop out of the
+    // straight-line code)
+    for (uint32_t it = 0; __builtin_expect(pend != 0u, 0); ++it) {
+        if (it == 0)
+            t0 = gtimer();
+#pragma unroll
+        for (int r = 0; r < RI; ++r) {
+            const uint64_t *vp = xg + (size_t)(vb + lane + 32 * (i0 + r)) * E;
+#pragma unroll
+            for (int e = 0; e < H; ++e)
+                if (pend & (1u << (r * H + e)))
+                    fw_ld2(vp + 2 * e, wa[r][e], wb[r][e]);
+        }
+        uint64_t last = 0;
+#pragma unroll
+        for (int r = 0; r < RI; ++r)
+#pragma unroll
+            for (int e = 0; e < H; ++e) {
+                const uint32_t bit = 1u << (r * H + e);
+                if (pend & bit) {
+                    if (fw_ok(wa[r][e], tag) && fw_ok(wb[r][e], tag)) {
+                        xf[i0 + r][2 * e] = fw_val(wa[r][e]);
+                        xf[i0 + r][2 * e + 1] = fw_val(wb[r][e]);
+                        pend &= ~bit;
+                    } else {
+                        last = fw_ok(wa[r][e], tag) ? wb[r][e] : wa[r][e];
+                    }
+                }
+            }
+        if (pend && (it & 15) == 15 && fw_give_up(p, s, t0, last, it))
+            return false;
+    }
+    if (t0)
+        fw_note(p, s, t0);
+    return true;
+}
+
+template <int NI, int E, int W = kFwRoundWords>
+__device__ __forceinline__ bool fw_lane_vectors(const KParams &p, const SmemLayout &s,
+                                                const uint64_t *xg, int vb, int ni, int lane,
+                                                float (&xf)[NI][E])
+{
+    // one round up to W words, else rounds of at most min(W, 32)
+    constexpr int WR = W < 32 ? W : 32;
+    constexpr int RI = NI * E <= W ? NI : (WR / E > 0 ? WR / E : 1);
+#pragma unroll
+    for (int i0 = 0; i0 < NI; i0 += RI)
+        if (!fw_lane_round<NI, E, (RI < NI ? RI : NI)>(p, s, xg, vb, ni, lane, i0, xf))
+            return false;
+    return true;
+}
+
 // Counter wait by consumer thread 0; returns false on timeout / abort.
 __device__ bool wait_counter(const KParams &p, const TaskDesc &d, int ti)
 {
@@ -908,25 +1163,31 @@ __device__ float block_sum(float v, const SmemLayout &s, int ct)
     return t;
 }
 
-// vec[i] = g_i * x_i / sqrt(mean x^2 + eps), x from L2 (fp32) or the
-// embedding row (bf16).  The gains gv (thread t: elements t + 256 j) were
-// loaded before the task's counter wait, so that their first touch in HBM
-// is off the critical path; every load of x is issued before any store (one
-// L2 round trip); hidden <= kMaxPerThread * 256.
+// vec[i] = g_i * x_i / sqrt(mean x^2 + eps), x from flagged words, the
+// fixed-point residual or the embedding row (bf16).  The gains gv (thread t:
+// elements t + 256 j, raw bf16 bits, first used here) were loaded before the
+// task's wait, so that their first touch in HBM is off the critical path;
+// every load of x is issued before
+// any store (one L2 round trip once the words are there); hidden <=
+// kMaxPerThread * 256.
 constexpr int kMaxPerThread = 16;
-__device__ void rmsnorm_prologue(const KParams &p, const SmemLayout &s, const float *x_f32,
+__device__ void rmsnorm_prologue(const KParams &p, const SmemLayout &s, const uint64_t *x_fw,
                                  const uint16_t *x_bf16, const long long *x_fix,
-                                 const float (&gv)[kMaxPerThread], int ct)
+                                 const uint32_t (&gv)[kMaxPerThread], int ct)
 {
     const int n = p.hidden;
     float xv[kMaxPerThread];
+    if (x_fw) {
+        if (!fw_read_strided<kMaxPerThread>(p, s, x_fw, n, ct, xv))
+            s.flags[0] = 1;  // before block_sum's barrier: every thread sees it after
+    } else {
 #pragma unroll
-    for (int j = 0; j < kMaxPerThread; ++j) {
-        const int i = ct + j * kConsumerThreads;
-        xv[j] = 0.f;
-        if (i < n)
-            xv[j] = x_f32 ? __ldcg(x_f32 + i)
-                          : x_fix ? from_fix(__ldcg(x_fix + i)) : bf16_to_f(__ldg(x_bf16 + i));
+        for (int j = 0; j < kMaxPerThread; ++j) {
+            const int i = ct + j * kConsumerThreads;
+            xv[j] = 0.f;
+            if (i < n)
+                xv[j] = x_fix ? from_fix(__ldcg(x_fix + i)) : bf16_to_f(__ldg(x_bf16 + i));
+        }
     }
     float ss = 0.f;
 #pragma unroll
@@ -938,7 +1199,7 @@ __device__ void rmsnorm_prologue(const KParams &p, const SmemLayout &s, const fl
     for (int j = 0; j < kMaxPerThread; ++j) {
         const int i = ct + j * kConsumerThreads;
         if (i < n)
-            s.vec[vidx(i)] = gv[j] * (xv[j] * inv);
+            s.vec[vidx(i)] = bf16_to_f((uint16_t)gv[j]) * (xv[j] * inv);
     }
     consumer_bar();
 }
@@ -951,7 +1212,7 @@ __device__ void rmsnorm_prologue(const KParams &p, const SmemLayout &s, const fl
 // shared vector (prologue output) or, when xg is set, straight from L2.
 template <int ESZ, int VB>
 __device__ __forceinline__ bool gemv_task(const KParams &p, const SmemLayout &s, const Geom g,
-                                          RingPos &kc, int warp, int lane, const float *xg,
+                                          RingPos &kc, int warp, int lane, const uint64_t *xg,
                                           uint64_t *wt)
 {
     constexpr int E = VB / ESZ;   // elements per vector (even)
@@ -965,41 +1226,43 @@ __device__ __forceinline__ bool gemv_task(const KParams &p, const SmemLayout &s,
     const int ve = min(vb + VPS, NV);
     const int ni = (ve - vb - lane + 31) / 32;  // vectors this lane holds (may be <= 0)
     // the lane's activations: 16-byte pieces of its vectors (8 bytes when a
-    // vector holds 2 elements), from the padded shared vector or from L2
+    // vector holds 2 elements), from the padded shared vector or from the
+    // flagged words xg
     f2_t xp[NI][EP];
+    if (xg) {
+        float xf[NI][E];
+        if (!fw_lane_vectors<NI, E, 16>(p, s, xg, vb, ni, lane, xf))
+            return false;
 #pragma unroll
-    for (int i = 0; i < NI; ++i) {
-        const int v = vb + lane + 32 * i;
-        if constexpr (E >= 4) {
+        for (int i = 0; i < NI; ++i)
 #pragma unroll
-            for (int e = 0; e < E; e += 4) {
-                float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (i < ni) {
-                    if (xg) {
-                        t = __ldcg(reinterpret_cast<const float4 *>(xg + v * E + e));
-                    } else {
+            for (int e = 0; e < EP; ++e)
+                xp[i][e] = pk2(xf[i][2 * e], xf[i][2 * e + 1]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < NI; ++i) {
+            const int v = vb + lane + 32 * i;
+            if constexpr (E >= 4) {
+#pragma unroll
+                for (int e = 0; e < E; e += 4) {
+                    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (i < ni) {
                         const uint4 u = lds128(s.vec_a + (uint32_t)vidx(v * E + e) * 4);
                         t = make_float4(__uint_as_float(u.x), __uint_as_float(u.y),
                                         __uint_as_float(u.z), __uint_as_float(u.w));
                     }
+                    xp[i][e / 2] = pk2(t.x, t.y);
+                    xp[i][e / 2 + 1] = pk2(t.z, t.w);
                 }
-                xp[i][e / 2] = pk2(t.x, t.y);
-                xp[i][e / 2 + 1] = pk2(t.z, t.w);
-            }
-        } else {
-            float a = 0.f, b = 0.f;
-            if (i < ni) {
-                if (xg) {
-                    const float2 t = __ldcg(reinterpret_cast<const float2 *>(xg + v * E));
-                    a = t.x;
-                    b = t.y;
-                } else {
+            } else {
+                float a = 0.f, b = 0.f;
+                if (i < ni) {
                     const uint2 t = lds64(s.vec_a + (uint32_t)vidx(v * E) * 4);
                     a = __uint_as_float(t.x);
                     b = __uint_as_float(t.y);
                 }
+                xp[i][0] = pk2(a, b);
             }
-            xp[i][0] = pk2(a, b);
         }
     }
     const uint32_t red_a = s.red_a + (uint32_t)warp * kMaxTaskRows * 4;
@@ -1274,9 +1537,9 @@ __device__ __forceinline__ void gemv_rows(const LaneX<ESZ, NI> &x, uint32_t stag
 // transposed shuffle reduction serves the four rows.  NI (vectors a lane
 // holds) is a template parameter so that the activation registers are sized
 // to the shape, not to the largest one.
-template <int ESZ, int NI>
+template <int ESZ, int NI, int W = kFwRoundWords>
 __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &s, const Geom g,
-                                            RingPos &kc, int warp, int lane, const float *xg,
+                                            RingPos &kc, int warp, int lane, const uint64_t *xg,
                                             uint64_t *wt)
 {
     using LX = LaneX<ESZ, NI>;
@@ -1291,25 +1554,23 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
     LX x;
     {
         float xf[NI][E];
+        if (xg) {
+            if (!fw_lane_vectors<NI, E, W>(p, s, xg, vb, ni, lane, xf))
+                return false;
+        } else {
 #pragma unroll
-        for (int i = 0; i < NI; ++i) {
-            const int v = vb + lane + 32 * i;
+            for (int i = 0; i < NI; ++i) {
+                const int v = vb + lane + 32 * i;
 #pragma unroll
-            for (int e = 0; e < E; e += 4) {
-                float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (i < ni) {
-                    if (xg) {
-                        t = __ldcg(reinterpret_cast<const float4 *>(xg + v * E + e));
-                    } else {
-                        const uint4 u = lds128(s.vec_a + (uint32_t)vidx(v * E + e) * 4);
-                        t = make_float4(__uint_as_float(u.x), __uint_as_float(u.y),
-                                        __uint_as_float(u.z), __uint_as_float(u.w));
-                    }
+                for (int e = 0; e < E; e += 4) {
+                    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                    if (i < ni)
+                        u = lds128(s.vec_a + (uint32_t)vidx(v * E + e) * 4);
+                    xf[i][e] = __uint_as_float(u.x);
+                    xf[i][e + 1] = __uint_as_float(u.y);
+                    xf[i][e + 2] = __uint_as_float(u.z);
+                    xf[i][e + 3] = __uint_as_float(u.w);
                 }
-                xf[i][e] = t.x;
-                xf[i][e + 1] = t.y;
-                xf[i][e + 2] = t.z;
-                xf[i][e + 3] = t.w;
             }
         }
         if constexpr (ESZ == 2) {
@@ -1422,33 +1683,33 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
 }
 
 // Dispatch on the vectors a lane holds for this task's K-slice.
-template <int ESZ>
+template <int ESZ, int W = kFwRoundWords>
 __device__ __forceinline__ bool gemv16(const KParams &p, const SmemLayout &s, const Geom &g,
-                                       RingPos &kc, int warp, int lane, const float *xg,
+                                       RingPos &kc, int warp, int lane, const uint64_t *xg,
                                        uint64_t *wt)
 {
     const int vps = ((ESZ ? g.RB >> 4 : g.K >> 5) + g.KS - 1) >> g.ks_log2;
     const int nimax = (vps + 31) >> 5;
     if constexpr (ESZ == 0) {
         if (nimax <= 1)
-            return gemv16_task<0, 1>(p, s, g, kc, warp, lane, xg, wt);
-        return gemv16_task<0, 2>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<0, 1, W>(p, s, g, kc, warp, lane, xg, wt);
+        return gemv16_task<0, 2, W>(p, s, g, kc, warp, lane, xg, wt);
     } else if constexpr (ESZ == 2) {
         if (nimax <= 2)
-            return gemv16_task<2, 2>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<2, 2, W>(p, s, g, kc, warp, lane, xg, wt);
         if (nimax <= 4)
-            return gemv16_task<2, 4>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<2, 4, W>(p, s, g, kc, warp, lane, xg, wt);
         if (nimax <= 6)
-            return gemv16_task<2, 6>(p, s, g, kc, warp, lane, xg, wt);
-        return gemv16_task<2, 8>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<2, 6, W>(p, s, g, kc, warp, lane, xg, wt);
+        return gemv16_task<2, 8, W>(p, s, g, kc, warp, lane, xg, wt);
     } else {
         if (nimax <= 1)
-            return gemv16_task<1, 1>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<1, 1, W>(p, s, g, kc, warp, lane, xg, wt);
         if (nimax <= 2)
-            return gemv16_task<1, 2>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<1, 2, W>(p, s, g, kc, warp, lane, xg, wt);
         if (nimax <= 3)
-            return gemv16_task<1, 3>(p, s, g, kc, warp, lane, xg, wt);
-        return gemv16_task<1, 4>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<1, 3, W>(p, s, g, kc, warp, lane, xg, wt);
+        return gemv16_task<1, 4, W>(p, s, g, kc, warp, lane, xg, wt);
     }
 }
 
@@ -1457,7 +1718,7 @@ __device__ __forceinline__ bool gemv16(const KParams &p, const SmemLayout &s, co
 // time (models with odd row widths, or a bf16 tied head on int8 layers).
 template <int Q8, int GENERIC>
 __device__ __forceinline__ bool run_gemv(const KParams &p, const SmemLayout &s, const Geom &g,
-                                         RingPos &kc, int warp, int lane, const float *xg,
+                                         RingPos &kc, int warp, int lane, const uint64_t *xg,
                                          uint64_t *wt)
 {
     if constexpr (!GENERIC) {
@@ -1471,15 +1732,17 @@ __device__ __forceinline__ bool run_gemv(const KParams &p, const SmemLayout &s, 
             return gemv16<2>(p, s, g, kc, warp, lane, xg, wt);
         }
     } else {
+        // (smaller rounds of flagged activation loads: this instance holds
+        // every path, and the registers are shared by all of them)
         if (g.esz == 2) {
             if (g.VB == 16)
-                return gemv16<2>(p, s, g, kc, warp, lane, xg, wt);
+                return gemv16<2, 16>(p, s, g, kc, warp, lane, xg, wt);
             if (g.VB == 8)
                 return gemv_task<2, 8>(p, s, g, kc, warp, lane, xg, wt);
             return gemv_task<2, 4>(p, s, g, kc, warp, lane, xg, wt);
         }
         if (g.VB == 16)
-            return gemv16<1>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16<1, 16>(p, s, g, kc, warp, lane, xg, wt);
         if (g.VB == 8)
             return gemv_task<1, 8>(p, s, g, kc, warp, lane, xg, wt);
         return gemv_task<1, 4>(p, s, g, kc, warp, lane, xg, wt);
@@ -1496,11 +1759,6 @@ __device__ __forceinline__ float row_total(const SmemLayout &s, const Geom &g, i
     for (int ks = 0; ks < g.KS; ++ks)
         y += s.red[(rg + g.RG * ks) * kMaxTaskRows + t];
     return y;
-}
-
-__device__ __forceinline__ float row_scale(const uint16_t *scale, int t)
-{
-    return scale ? fp16_to_f(__ldg(scale + t)) : 1.f;
 }
 
 // RoPE angle of pair i at position pos (HF rotate_half): a = pos * w_i with
@@ -1551,7 +1809,7 @@ __device__ __forceinline__ void lds_bf16(uint32_t a, float (&out)[E])
 template <int E>
 __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s,
                                           const TaskDesc &d, const Geom &g, RingPos &kc,
-                                          int ct, int warp, int lane, uint64_t *wt)
+                                          int ct, int warp, int lane, uint64_t *wt, uint32_t otag)
 {
     const int l = d.layer, gi = d.r0, c = d.r1;
     const int hd = p.head_dim, G = p.group, nh = p.n_heads, nkv = p.n_kv_heads;
@@ -1560,7 +1818,7 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
     float *kn = qs + G * hd;                 // [hd] new K row (bf16 value)
     float *vn = kn + hd;                     // [hd] new V row (bf16 value)
     float *ws = vn + hd;                     // [8][G][hd + 2] per-warp partials
-    const float *qkv = p.qkv + (size_t)l * p.qkv_rows;
+    const uint64_t *qkv = p.qkv + (size_t)l * p.qkv_rows;
     if (g.j1 <= g.j0)
         return true;  // empty chunk: no partial (the merge skips it)
     // prologue: q of the group's G heads and k get RoPE (pairs i, i + hd/2),
@@ -1572,34 +1830,64 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
                    (size_t)p.pos * hd;
     uint16_t *vd = const_cast<uint16_t *>(static_cast<const uint16_t *>(d.w1)) +
                    (size_t)p.pos * hd;
-    for (int i = ct; i < (G + 1) * half; i += kConsumerThreads) {
-        const int hh = i / half, e = i % half;
-        const float *src = hh < G ? qkv + (size_t)(gi * G + hh) * hd
-                                  : qkv + (size_t)nh * hd + (size_t)gi * hd;
-        const float x0 = __ldcg(src + e), x1 = __ldcg(src + e + half);
-        float sn, cs;
-        rope_angle(p.pos, e, hd, p.rope_theta, &sn, &cs);
-        const float y0 = x0 * cs - x1 * sn, y1 = x1 * cs + x0 * sn;
-        if (hh < G) {
-            qs[hh * hd + e] = y0 * qscale;
-            qs[hh * hd + e + half] = y1 * qscale;
-        } else {
-            const uint16_t b0 = f_to_bf16(y0), b1 = f_to_bf16(y1);
-            kn[e] = bf16_to_f(b0);
-            kn[e + half] = bf16_to_f(b1);
-            if (c == 0) {
-                kd[e] = b0;
-                kd[e + half] = b1;
+    // the flagged words of q, k (as RoPE pairs) and v, two pairs and two v
+    // elements per thread and round, all of a round's words polled at once
+    // (one round for every head size and group up to (G + 1) hd / 2 <= 512)
+    const int npair = (G + 1) * half;
+    const uint64_t *vsrc = qkv + (size_t)(nh + nkv) * hd + (size_t)gi * hd;
+    for (int r0 = 0; r0 < npair || r0 < hd; r0 += 2 * kConsumerThreads) {
+        const uint64_t *a[6];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int i = r0 + ct + k * kConsumerThreads;
+            a[2 * k] = a[2 * k + 1] = nullptr;
+            if (i < npair) {
+                const int hh = i / half, e = i % half;
+                const uint64_t *src = hh < G ? qkv + (size_t)(gi * G + hh) * hd
+                                             : qkv + (size_t)nh * hd + (size_t)gi * hd;
+                a[2 * k] = src + e;
+                a[2 * k + 1] = src + e + half;
+            }
+            a[4 + k] = i < hd ? vsrc + i : nullptr;
+        }
+        float xv[6];
+        if (!fw_gather<6>(p, s, a, xv)) {
+            s.flags[0] = 1;
+            break;
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int i = r0 + ct + k * kConsumerThreads;
+            if (i < npair) {
+                const int hh = i / half, e = i % half;
+                const float x0 = xv[2 * k], x1 = xv[2 * k + 1];
+                float sn, cs;
+                rope_angle(p.pos, e, hd, p.rope_theta, &sn, &cs);
+                const float y0 = x0 * cs - x1 * sn, y1 = x1 * cs + x0 * sn;
+                if (hh < G) {
+                    qs[hh * hd + e] = y0 * qscale;
+                    qs[hh * hd + e + half] = y1 * qscale;
+                } else {
+                    const uint16_t b0 = f_to_bf16(y0), b1 = f_to_bf16(y1);
+                    kn[e] = bf16_to_f(b0);
+                    kn[e + half] = bf16_to_f(b1);
+                    if (c == 0) {
+                        kd[e] = b0;
+                        kd[e + half] = b1;
+                    }
+                }
+            }
+            if (i < hd) {
+                const uint16_t vb = f_to_bf16(xv[4 + k]);
+                vn[i] = bf16_to_f(vb);
+                if (c == 0)
+                    vd[i] = vb;
             }
         }
     }
-    for (int i = ct; i < hd; i += kConsumerThreads) {
-        const uint16_t vb = f_to_bf16(__ldcg(qkv + (size_t)(nh + nkv) * hd + (size_t)gi * hd + i));
-        vn[i] = bf16_to_f(vb);
-        if (c == 0)
-            vd[i] = vb;
-    }
     consumer_bar();
+    if (*reinterpret_cast<volatile int *>(s.flags))
+        return false;
     // lane layout: lph lanes per head hold E = hd / lph of its elements; the
     // G heads of the group take lph * G lanes, and the warp's 32 lanes hold
     // PG such groups, each scoring a different position at the same time.
@@ -1773,7 +2061,7 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
     // its heads directly; otherwise the partial (m, l, o) for the merge
     const bool direct = g.j0 == 0 && g.j1 == p.pos + 1;
     float *out = p.part + ((((size_t)l * nkv + gi) * p.attn_splits + c) * G) * (hd + 2);
-    float *fin = p.attn + (size_t)l * nh * hd + (size_t)gi * G * hd;
+    uint64_t *fin = p.attn + (size_t)l * nh * hd + (size_t)gi * G * hd;
     for (int i = ct; i < G * hd; i += kConsumerThreads) {
         const int hh = i / hd, e = i % hd;
         float M = -INFINITY;
@@ -1789,7 +2077,7 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
             O = fmaf(pw[2 + e], f, O);
         }
         if (direct) {
-            fin[i] = O / L;
+            fw_st(fin + i, O / L, otag);
             continue;
         }
         out[(size_t)hh * (hd + 2) + 2 + e] = O;
@@ -1811,7 +2099,8 @@ __device__ __forceinline__ bool attn_chunk(const KParams &p, const SmemLayout &s
 // K = 1 serves a single non-empty chunk (short contexts: out = o / l).
 template <int K, int B>
 __device__ __forceinline__ void merge_batches(const KParams &p, const float *part, int nne,
-                                              int first, int count, float *out, int ct)
+                                              int first, int count, uint64_t *out, int ct,
+                                              uint32_t otag)
 {
     const int hd = p.head_dim, G = p.group, C = p.attn_splits;
     const size_t cstride = (size_t)G * (hd + 2);  // chunk c + 1 of a head is this far on
@@ -1875,7 +2164,7 @@ __device__ __forceinline__ void merge_batches(const KParams &p, const float *par
         for (int j = 0; j < B; ++j) {
             const int i = ct + (j0 + j) * kConsumerThreads;
             if (i < count)
-                out[i] = O[j] / L[j];
+                fw_st(out + i, O[j] / L[j], otag);
         }
     }
 }
@@ -1902,9 +2191,9 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v)
 template <int E>
 __device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
                                           const TaskDesc &d, const Geom &g, RingPos &kc,
-                                          int ct, int warp, int lane, uint64_t *wt)
+                                          int ct, int warp, int lane, uint64_t *wt, uint32_t otag)
 {
-    if (!attn_chunk<E>(p, s, d, g, kc, ct, warp, lane, wt))
+    if (!attn_chunk<E>(p, s, d, g, kc, ct, warp, lane, wt, otag))
         return false;
     const int l = d.layer, gi = d.r0, C = p.attn_splits;
     const int n = p.pos + 1;
@@ -1922,8 +2211,8 @@ __device__ __forceinline__ bool attn_task(const KParams &p, const SmemLayout &s,
     if (*reinterpret_cast<volatile int *>(last)) {
         const int hd = p.head_dim, G = p.group, N = p.n_heads * hd;
         const float *part = p.part + (size_t)l * p.n_kv_heads * C * G * (hd + 2);
-        float *out = p.attn + (size_t)l * N + (size_t)gi * G * hd;
-        merge_batches<4, 4>(p, part, nne, gi * G * hd, G * hd, out, ct);
+        uint64_t *out = p.attn + (size_t)l * N + (size_t)gi * G * hd;
+        merge_batches<4, 4>(p, part, nne, gi * G * hd, G * hd, out, ct, otag);
     }
     return true;
 }
@@ -1939,26 +2228,46 @@ __device__ void pos0_prologue(const KParams &p, const SmemLayout &s, const TaskD
 {
     const int l = d.layer, hd = p.head_dim, nh = p.n_heads, nkv = p.n_kv_heads, G = p.group;
     const int KV = nkv * hd;  // elements of one of K, V
-    const float *qkv = p.qkv + (size_t)l * p.qkv_rows;
-    const float *ksrc = qkv + (size_t)nh * hd, *vsrc = ksrc + KV;
+    const uint64_t *qkv = p.qkv + (size_t)l * p.qkv_rows;
+    const uint64_t *ksrc = qkv + (size_t)nh * hd, *vsrc = ksrc + KV;
     // element r of V (KV head r / hd) is the output of the G heads of that
-    // group: thread t takes r = t + 256 j, one load and G stores each
-    float v[kMaxPerThread];
+    // group: thread t takes r = t + 256 j, one flagged word and G stores each
+    // and the tile's share of cache row 0: elements i = a + t + 256 k of
+    // (K | V), the first two of them loaded together with the V words
+    const int E = 2 * KV;
+    const int a = (int)((int64_t)d.r0 * E / p.hidden), b = (int)((int64_t)d.r1 * E / p.hidden);
+    const size_t blk = (size_t)p.max_ctx * hd;  // one (layer, K|V, head) block
+    const uint64_t *sh[2];
+    uint64_t shw[2];
 #pragma unroll
-    for (int j = 0; j < kMaxPerThread; ++j) {
-        const int r = ct + j * kConsumerThreads;
-        v[j] = r < KV ? __ldcg(vsrc + r) : 0.f;
+    for (int k = 0; k < 2; ++k) {
+        const int i = a + ct + k * kConsumerThreads;
+        sh[k] = i < b ? ksrc + i : nullptr;
+        shw[k] = sh[k] ? fw_ld(sh[k]) : 0ull;
     }
-    {
-        const int E = 2 * KV;
-        const int a = (int)((int64_t)d.r0 * E / p.hidden), b = (int)((int64_t)d.r1 * E / p.hidden);
-        const size_t blk = (size_t)p.max_ctx * hd;  // one (layer, K|V, head) block
-        for (int i = a + ct; i < b; i += kConsumerThreads) {
+    float v[kMaxPerThread];
+    bool ok = fw_read_strided<kMaxPerThread>(p, s, vsrc, KV, ct, v);
+    for (int i0 = a + ct; i0 < b && ok; i0 += 2 * kConsumerThreads) {
+        float kvv[2];
+        if (i0 == a + ct && (!sh[0] || fw_ok(shw[0], p.tag)) && (!sh[1] || fw_ok(shw[1], p.tag))) {
+            kvv[0] = fw_val(shw[0]);
+            kvv[1] = fw_val(shw[1]);
+        } else {
+            const int i1 = i0 + kConsumerThreads;
+            const uint64_t *w[2] = {ksrc + i0, i1 < b ? ksrc + i1 : nullptr};
+            ok = fw_gather<2>(p, s, w, kvv);
+        }
+        for (int k = 0; k < 2 && ok; ++k) {
+            const int i = i0 + k * kConsumerThreads;
+            if (i >= b)
+                break;
             const int which = i >= KV, r = i - which * KV;  // 0: K, 1: V
             const int g = r / hd, e = r - g * hd;
-            p.kv[(((size_t)l * 2 + which) * nkv + g) * blk + e] = f_to_bf16(__ldcg(ksrc + i));
+            p.kv[(((size_t)l * 2 + which) * nkv + g) * blk + e] = f_to_bf16(kvv[k]);
         }
     }
+    if (!ok)
+        s.flags[0] = 1;  // before the barrier below: every thread sees it after
 #pragma unroll
     for (int j = 0; j < kMaxPerThread; ++j) {
         const int r = ct + j * kConsumerThreads;
@@ -1977,13 +2286,10 @@ __device__ void pos0_prologue(const KParams &p, const SmemLayout &s, const TaskD
 __device__ void attn_prologue(const KParams &p, const SmemLayout &s, int l, int ct)
 {
     const int N = p.n_heads * p.head_dim;
-    const float *src = p.attn + (size_t)l * N;
+    const uint64_t *src = p.attn + (size_t)l * N;
     float v[kMaxPerThread];
-#pragma unroll
-    for (int j = 0; j < kMaxPerThread; ++j) {
-        const int i = ct + j * kConsumerThreads;
-        v[j] = i < N ? __ldcg(src + i) : 0.f;
-    }
+    if (!fw_read_strided<kMaxPerThread>(p, s, src, N, ct, v))
+        s.flags[0] = 1;  // before the barrier below: every thread sees it after
 #pragma unroll
     for (int j = 0; j < kMaxPerThread; ++j) {
         const int i = ct + j * kConsumerThreads;
@@ -2199,14 +2505,17 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
         stage_task(s.ctask_a, p.tasks + qb);
     for (int ti = qb; ti < qe; ++ti) {
         const uint32_t slot = s.ctask_a + ((ti - qb) & 1) * sizeof(TaskDesc);
-        if (ct == 0)
+        if (ct == 0) {
             stage_task_wait();  // record of task ti (issued one task ago)
+            s.flags[2] = ti;    // for the error record of a flagged read that gives up
+        }
         consumer_bar();
         const TaskDesc d = read_staged(slot);
         uint64_t t_w0 = 0, t_w1 = 0, t_pro = 0, t_epi = 0;
         if (prof) {
             t_w0 = gtimer();
             s.wacc[0] = s.wacc[1] = 0ull;
+            *reinterpret_cast<volatile unsigned long long *>(s.flags + 4) = 0ull;
         }
         if (wprof)
             wt_store[0] = wt_store[1] = 0;
@@ -2214,82 +2523,97 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
         // the counter wait: the RMSNorm gains and the int8 row scales of the
         // epilogue (thread t finalises row r0 + t; R <= 256)
         const Geom g = task_geom(p, d);
-        float gv[kMaxPerThread];
+        // (kept as raw bits until first use: a conversion here would wait for
+        // the loads before the task's own wait starts)
+        uint32_t gv[kMaxPerThread];
         const bool norm = d.kind == TK_QKV || d.kind == TK_GATEUP || d.kind == TK_FFN ||
                           d.kind == TK_LMHEAD;
 #pragma unroll
         for (int j = 0; j < kMaxPerThread; ++j) {
             const int i = ct + j * kConsumerThreads;
-            gv[j] = (norm && i < p.hidden) ? bf16_to_f(__ldg(d.gain + i)) : 0.f;
+            gv[j] = (norm && i < p.hidden) ? (uint32_t)__ldg(d.gain + i) : 0u;
         }
-        float sc0 = 1.f, sc1 = 1.f;
+        uint32_t sc0r = 0x3c00u, sc1r = 0x3c00u;  // fp16 1.0
         if (d.kind != TK_ATTN && ct < g.R) {
-            sc0 = row_scale(d.s0, ct);
-            sc1 = row_scale(d.s1, ct);
+            if (d.s0)
+                sc0r = __ldg(d.s0 + ct);
+            if (d.s1)
+                sc1r = __ldg(d.s1 + ct);
         }
         if (ct == 0) {
             if (ti + 1 < qe)  // the slot read at ti - 1 is free again (barrier above)
                 stage_task(s.ctask_a + ((ti + 1 - qb) & 1) * sizeof(TaskDesc), p.tasks + ti + 1);
-            if (!wait_counter(p, d, ti))
+            // with flagged waits the task's reads of its flagged inputs are
+            // its wait (every input of every task is flagged then)
+            if (!p.flagged && !wait_counter(p, d, ti))
                 s.flags[0] = 1;
         }
         consumer_bar();
         if (*reinterpret_cast<volatile int *>(s.flags))
             break;
+        // the tag of this task's flagged outputs (the test hook that withholds
+        // a task's signal gives them a wrong one)
+        const uint32_t otag =
+            (p.flagged && ti == p.skip_signal_task) ? p.tag ^ 0x80000000u : p.tag;
         if (prof)
             t_w1 = gtimer();
         const int l = d.layer;
         bool ok = true;
         if (d.kind == TK_ATTN) {
             if constexpr (!GENERIC) {
-                ok = attn_task<ATT_E>(p, s, d, g, kc, ct, warp, lane, wt);
+                ok = attn_task<ATT_E>(p, s, d, g, kc, ct, warp, lane, wt, otag);
             } else {
                 switch (p.att_e) {
-                case 1: ok = attn_task<1>(p, s, d, g, kc, ct, warp, lane, wt); break;
-                case 2: ok = attn_task<2>(p, s, d, g, kc, ct, warp, lane, wt); break;
-                case 4: ok = attn_task<4>(p, s, d, g, kc, ct, warp, lane, wt); break;
-                case 8: ok = attn_task<8>(p, s, d, g, kc, ct, warp, lane, wt); break;
-                default: ok = attn_task<16>(p, s, d, g, kc, ct, warp, lane, wt); break;
+                case 1: ok = attn_task<1>(p, s, d, g, kc, ct, warp, lane, wt, otag); break;
+                case 2: ok = attn_task<2>(p, s, d, g, kc, ct, warp, lane, wt, otag); break;
+                case 4: ok = attn_task<4>(p, s, d, g, kc, ct, warp, lane, wt, otag); break;
+                case 8: ok = attn_task<8>(p, s, d, g, kc, ct, warp, lane, wt, otag); break;
+                default: ok = attn_task<16>(p, s, d, g, kc, ct, warp, lane, wt, otag); break;
                 }
             }
             if (prof)
                 t_pro = t_epi = gtimer();
         } else {
-            // prologue -> s.vec
-            if (d.kind == TK_QKV) {
-                if (l == 0) {
+            // prologue -> s.vec (one call site per prologue kind: the kernel
+            // is one persistent program, and its instruction footprint counts)
+            if (norm) {
+                // the RMSNorm input: the embedding row (layer 0), the previous
+                // layer's residual (fixed point after a fused FFN level), or
+                // the residual after attention (gate/up, fused FFN)
+                const uint64_t *xw = nullptr;
+                const uint16_t *xb = nullptr;
+                const long long *xq = nullptr;
+                const int lp = d.kind == TK_LMHEAD ? p.n_layers - 1 : l - 1;
+                if (d.kind == TK_GATEUP || d.kind == TK_FFN) {
+                    xw = p.xmid + (size_t)l * p.hidden;
+                } else if (d.kind == TK_QKV && l == 0) {
                     if (token < 0)
                         token = resolve_token(p);
-                    rmsnorm_prologue(p, s, nullptr, p.embed + (size_t)token * p.hidden, nullptr,
-                                     gv, ct);
+                    xb = p.embed + (size_t)token * p.hidden;
                 } else if (p.ffn_fused) {
-                    rmsnorm_prologue(p, s, nullptr, nullptr, p.xacc + (size_t)(l - 1) * p.hidden,
-                                     gv, ct);
+                    xq = p.xacc + (size_t)lp * p.hidden;
                 } else {
-                    rmsnorm_prologue(p, s, p.xout + (size_t)(l - 1) * p.hidden, nullptr, nullptr,
-                                     gv, ct);
+                    xw = p.xout + (size_t)lp * p.hidden;
                 }
+                rmsnorm_prologue(p, s, xw, xb, xq, gv, ct);
             } else if (d.kind == TK_OPROJ) {
                 if (d.flags & TF_POS0)
                     pos0_prologue(p, s, d, ct);
                 else
                     attn_prologue(p, s, l, ct);
-            } else if (d.kind == TK_GATEUP || d.kind == TK_FFN) {
-                rmsnorm_prologue(p, s, p.xmid + (size_t)l * p.hidden, nullptr, nullptr, gv, ct);
-            } else if (d.kind == TK_DOWN) {
-                // no prologue: each warp loads its slice of the SwiGLU
-                // activations from L2 straight into registers
-            } else {  // TK_LMHEAD
-                if (p.ffn_fused)
-                    rmsnorm_prologue(p, s, nullptr, nullptr,
-                                     p.xacc + (size_t)(p.n_layers - 1) * p.hidden, gv, ct);
-                else
-                    rmsnorm_prologue(p, s, p.xout + (size_t)(p.n_layers - 1) * p.hidden, nullptr,
-                                     nullptr, gv, ct);
             }
-            // residual inputs of the epilogue are ready now: fetch them while
-            // the GEMV runs (thread t owns output row r0 + t; R <= 256)
+            // (DOWN has no prologue: each warp loads its slice of the SwiGLU
+            // activations from the flagged words straight into registers)
+            // a prologue that gave up raised the abort flag before its last
+            // barrier (DOWN has none, and nothing since its wait raised it)
+            if (*reinterpret_cast<volatile int *>(s.flags))
+                break;
+            // residual inputs of the epilogue: their loads go out now and are
+            // used after the GEMV (thread t owns output row r0 + t; R <= 256);
+            // a flagged one is checked (and polled again if need be) there
             float base = 0.f;
+            const uint64_t *bsrc = nullptr;
+            uint64_t bw = 0;
             if (ct < g.R) {
                 const int r = d.r0 + ct;
                 if (d.kind == TK_OPROJ) {
@@ -2300,11 +2624,13 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
                     } else if (p.ffn_fused) {
                         base = from_fix(__ldcg(p.xacc + (size_t)(l - 1) * p.hidden + r));
                     } else {
-                        base = __ldcg(p.xout + (size_t)(l - 1) * p.hidden + r);
+                        bsrc = p.xout + (size_t)(l - 1) * p.hidden + r;
                     }
                 } else if (d.kind == TK_DOWN) {
-                    base = __ldcg(p.xmid + (size_t)l * p.hidden + r);
+                    bsrc = p.xmid + (size_t)l * p.hidden + r;
                 }
+                if (bsrc)
+                    bw = fw_ld(bsrc);
             }
             if (prof)
                 t_pro = gtimer();
@@ -2318,19 +2644,30 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
             if (prof)
                 t_epi = gtimer();
             ok = *reinterpret_cast<volatile int *>(s.flags) == 0;
+            const float sc0 = fp16_to_f((uint16_t)sc0r), sc1 = fp16_to_f((uint16_t)sc1r);
+            if (ok && bsrc) {
+                if (fw_ok(bw, p.tag)) {
+                    base = fw_val(bw);
+                } else {
+                    const uint64_t *const a1[1] = {bsrc};
+                    float v1[1];
+                    ok = fw_gather<1>(p, s, a1, v1);
+                    base = v1[0];
+                }
+            }
             if (ok) {
                 // epilogue: thread t finalises output row r0 + t
                 if (d.kind == TK_QKV) {
                     const int off = d.mat == 0 ? 0
                                     : d.mat == 1 ? p.n_heads * p.head_dim
                                                  : (p.n_heads + p.n_kv_heads) * p.head_dim;
-                    float *out = p.qkv + (size_t)l * p.qkv_rows + off + d.r0;
+                    uint64_t *out = p.qkv + (size_t)l * p.qkv_rows + off + d.r0;
                     for (int t = ct; t < g.R; t += kConsumerThreads)
-                        out[t] = row_total(s, g, t) * sc0;
+                        fw_st(out + t, row_total(s, g, t) * sc0, otag);
                 } else if (d.kind == TK_OPROJ) {
                     if (ct < g.R) {
                         const float v = base + row_total(s, g, ct) * sc0;
-                        p.xmid[(size_t)l * p.hidden + d.r0 + ct] = v;
+                        fw_st(p.xmid + (size_t)l * p.hidden + d.r0 + ct, v, otag);
                         if (p.ffn_fused)  // the FFN slices add into this
                             p.xacc[(size_t)l * p.hidden + d.r0 + ct] = to_fix(v);
                     }
@@ -2342,12 +2679,12 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
                         const float gt = row_total(s, g, t) * sc0;
                         const float up = row_total(s, g, g.R + t) * sc1;
                         const float silu = gt / (1.f + __expf(-gt));
-                        p.act[(size_t)l * p.ffn + d.r0 + t] = silu * up;
+                        fw_st(p.act + (size_t)l * p.ffn + d.r0 + t, silu * up, otag);
                     }
                 } else if (d.kind == TK_DOWN) {
                     if (ct < g.R)
-                        p.xout[(size_t)l * p.hidden + d.r0 + ct] =
-                            base + row_total(s, g, ct) * sc0;
+                        fw_st(p.xout + (size_t)l * p.hidden + d.r0 + ct,
+                              base + row_total(s, g, ct) * sc0, otag);
                 } else {  // TK_LMHEAD
                     unsigned long long best = 0ull;
                     for (int t = ct; t < g.R; t += kConsumerThreads) {
@@ -2386,16 +2723,20 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
         if (*reinterpret_cast<volatile int *>(s.flags))
             break;
         // release: the CTA barrier above orders every thread's stores before
-        // this release-add (cumulativity), so the waiters' acquire sees them
-        if (ct == 0 && d.signal_ctr >= 0 && ti != p.skip_signal_task)
+        // this release-add (cumulativity), so the waiters' acquire sees them.
+        // With flagged waits nobody waits on the level counters.
+        if (ct == 0 && !p.flagged && d.signal_ctr >= 0 && ti != p.skip_signal_task)
             red_release_add(p.counters + d.signal_ctr, 1u);
         if (prof) {
             const uint64_t t_end = gtimer();
             unsigned long long *pk = prof + (size_t)d.kind * kProfFields;
+            // the flagged polls of a task happen in its prologue (attention:
+            // its tile), except DOWN's, which its GEMV warps make
+            const uint64_t fw = *reinterpret_cast<volatile unsigned long long *>(s.flags + 4);
             pk[0] += 1;
             pk[1] += t_w1 - t_w0;
-            pk[2] += t_pro - t_w1;
-            pk[3] += 0;
+            pk[2] += t_pro - t_w1 - (d.kind == TK_DOWN ? 0ull : min(fw, t_pro - t_w1));
+            pk[3] += fw;
             pk[4] += t_end - t_w1;
             pk[5] += t_end - t_epi;
             pk[6] += s.wacc[0];

@@ -92,6 +92,7 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
         if (opt_in->copy_piece_kb > 0) opt.copy_piece_kb = opt_in->copy_piece_kb;
         if (opt_in->sm_rotate > 0) opt.sm_rotate = opt_in->sm_rotate;
         opt.debug_checks = opt_in->debug_checks;
+        if (opt_in->flagged_waits != 0) opt.flagged_waits = opt_in->flagged_waits;
         opt.n_sms = opt_in->n_sms;
     }
     const amk_config &c = *cfg;
@@ -250,17 +251,26 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
     const int64_t ffn_fit = box_rows ? (int64_t)opt.stage_bytes /
                                            ((int64_t)ffn_w * fesz * box_rows) * box_rows
                                      : 0;
-    // default (ffn_fused = 1): fuse when a residual row is at most 1.5 KB.  The
-    // fused level adds every slice's partial down projection into the same
-    // hidden-sized accumulator with 64-bit atomics, whose contention grows with
-    // the width; measured on B200 it gains 3% on the SmolLM2 shape (1152 B) but
-    // loses 2% on Llama-1B W8A16 (2 KB), 4% on Llama-7B and 10% on TinyLlama.
-    // ffn_fused = 2 fuses whenever the shape allows.
+    // default (ffn_fused = 1): separate FFN levels with flagged waits.  With
+    // level counters (flagged_waits = -1) the default fuses when a residual row
+    // is at most 1.5 KB: the fused level adds every slice's partial down
+    // projection into the same hidden-sized accumulator with 64-bit atomics,
+    // whose contention grows with the width; measured on B200 it gained 3% on
+    // the SmolLM2 shape (1152 B) but lost 2% on Llama-1B W8A16 (2 KB), 4% on
+    // Llama-7B and 10% on TinyLlama.  A fused level needs the counters (its
+    // residual is a fixed-point sum, not flagged words), and separate levels
+    // with flagged waits measured faster on the SmolLM2 shape too (517 against
+    // 527 us at context 0, 721 against 787 at 128).  ffn_fused = 2 fuses
+    // whenever the shape allows.
     const bool shape_ok = !q4 && F % ffn_gran == 0 && box_rows > 0 &&
                           ((int64_t)F * fesz) % 16 == 0 && (ffn_fit >= h || ffn_fit >= 256);
     const bool fused = shape_ok && (opt.ffn_fused >= 2 ||
-                                    (opt.ffn_fused == 1 && (int64_t)h * fesz <= 1536));
+                                    (opt.ffn_fused == 1 && opt.flagged_waits < 0 &&
+                                     (int64_t)h * fesz <= 1536));
     P->ffn_fused = fused ? 1 : 0;
+    // flagged waits need every input of every task to be a flagged word: with
+    // a fused FFN level the residual is a fixed-point sum, so counters stay
+    P->flagged = !fused && opt.flagged_waits >= 0 ? 1 : 0;
     P->ffn_box_rows = fused ? box_rows : 0;
 
     // ---- logical tasks per level ---------------------------------------------
@@ -451,22 +461,26 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
             const TaskDesc &d = P->tasks[t];
             amk_graph_task &gt = P->gtasks[t];
             gt.sm = s;
+            // with flagged waits the kernel touches no level counter: a task's
+            // waits are its flagged reads (READ_FLAGGED accesses below)
             gt.wait_begin = (int32_t)P->gwaits.size();
-            if (d.wait_ctr >= 0)
+            if (d.wait_ctr >= 0 && !P->flagged)
                 P->gwaits.push_back({d.wait_ctr, (int32_t)d.wait_count});
             gt.wait_count = (int32_t)P->gwaits.size() - gt.wait_begin;
             gt.signal_begin = (int32_t)P->gsignals.size();
-            if (d.signal_ctr >= 0)
+            if (d.signal_ctr >= 0 && !P->flagged)
                 P->gsignals.push_back(d.signal_ctr);
             gt.signal_count = (int32_t)P->gsignals.size() - gt.signal_begin;
             gt.access_begin = (int32_t)P->gacc.size();
             const int l = d.layer;
+            // reads of the activations one level hands to the next
+            const int RD = P->flagged ? AMK_ACC_READ_FLAGGED : AMK_ACC_READ;
             // what the kernel's task of this kind reads and writes
             switch (d.kind) {
             case amk::TK_QKV: {
                 const int off = d.mat == 0 ? 0 : d.mat == 1 ? nh * hd : (nh + nkv) * hd;
                 if (l > 0)
-                    acc(B_XOUT(l - 1), AMK_ACC_READ, 0, h);
+                    acc(B_XOUT(l - 1), RD, 0, h);
                 else
                     acc(B_KEYNEXT, AMK_ACC_READ_PREV, 0, 1);
                 acc(B_QKV(l), AMK_ACC_WRITE, off + d.r0, off + d.r1);
@@ -474,10 +488,9 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
             }
             case amk::TK_ATTN: {
                 const int g = d.r0, ci = d.r1;
-                acc(B_QKV(l), AMK_ACC_READ, (int64_t)g * G * hd, (int64_t)(g + 1) * G * hd);
-                acc(B_QKV(l), AMK_ACC_READ, (int64_t)nh * hd + g * hd,
-                    (int64_t)nh * hd + (g + 1) * hd);
-                acc(B_QKV(l), AMK_ACC_READ, (int64_t)(nh + nkv) * hd + g * hd,
+                acc(B_QKV(l), RD, (int64_t)g * G * hd, (int64_t)(g + 1) * G * hd);
+                acc(B_QKV(l), RD, (int64_t)nh * hd + g * hd, (int64_t)nh * hd + (g + 1) * hd);
+                acc(B_QKV(l), RD, (int64_t)(nh + nkv) * hd + g * hd,
                     (int64_t)(nh + nkv) * hd + (g + 1) * hd);
                 acc(B_ATTN(l), AMK_ACC_ACCUM, (int64_t)g * G * hd, (int64_t)(g + 1) * G * hd);
                 if (ci == 0)
@@ -489,14 +502,14 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
                     // head outputs from the V rows; KV row 0 in shares: the tile
                     // of rows [r0, r1) writes (K | V) elements [r0 E / h, r1 E / h)
                     const int64_t E = (int64_t)2 * nkv * hd;
-                    acc(B_QKV(l), AMK_ACC_READ, (int64_t)nh * hd, (int64_t)(nh + 2 * nkv) * hd);
+                    acc(B_QKV(l), RD, (int64_t)nh * hd, (int64_t)(nh + 2 * nkv) * hd);
                     if (d.r0 * E / h < d.r1 * E / h)
                         acc(B_KVNEW(l), AMK_ACC_WRITE, d.r0 * E / h, d.r1 * E / h);
                 } else {
-                    acc(B_ATTN(l), AMK_ACC_READ, 0, (int64_t)nh * hd);
+                    acc(B_ATTN(l), RD, 0, (int64_t)nh * hd);
                 }
                 if (l > 0)
-                    acc(B_XOUT(l - 1), AMK_ACC_READ, d.r0, d.r1);
+                    acc(B_XOUT(l - 1), RD, d.r0, d.r1);
                 else
                     acc(B_KEYNEXT, AMK_ACC_READ_PREV, 0, 1);
                 acc(B_XMID(l), AMK_ACC_WRITE, d.r0, d.r1);
@@ -504,20 +517,20 @@ int amk_lower(const amk_config *cfg, const amk_options *opt_in, int n_sms, amk_p
                     acc(B_XOUT(l), AMK_ACC_WRITE, d.r0, d.r1);
                 break;
             case amk::TK_FFN:
-                acc(B_XMID(l), AMK_ACC_READ, 0, h);
+                acc(B_XMID(l), RD, 0, h);
                 acc(B_XOUT(l), AMK_ACC_ACCUM, 0, h);
                 break;
             case amk::TK_GATEUP:
-                acc(B_XMID(l), AMK_ACC_READ, 0, h);
+                acc(B_XMID(l), RD, 0, h);
                 acc(B_ACT(l), AMK_ACC_WRITE, d.r0, d.r1);
                 break;
             case amk::TK_DOWN:
-                acc(B_ACT(l), AMK_ACC_READ, 0, F);
-                acc(B_XMID(l), AMK_ACC_READ, d.r0, d.r1);
+                acc(B_ACT(l), RD, 0, F);
+                acc(B_XMID(l), RD, d.r0, d.r1);
                 acc(B_XOUT(l), AMK_ACC_WRITE, d.r0, d.r1);
                 break;
             case amk::TK_LMHEAD:
-                acc(B_XOUT(L - 1), AMK_ACC_READ, 0, h);
+                acc(B_XOUT(L - 1), RD, 0, h);
                 acc(B_LOGITS, AMK_ACC_WRITE, d.r0, d.r1);
                 acc(B_KEY, AMK_ACC_ACCUM, 0, 1);
                 if (d.flags & amk::TF_RESET_ARGKEY)

@@ -57,12 +57,13 @@ Layout layout_of(const amk_plan &P)
     o.ctr = take(sizeof(uint32_t) * (size_t)(P.n_counters + P.n_arrive));
     o.err = take(sizeof(amk::ErrorWord));
     o.argkey = take(2 * sizeof(unsigned long long));
-    o.qkv = take(sizeof(float) * L * P.qkv_rows);
+    // flagged words (8 bytes each) from qkv to the end of act
+    o.qkv = take(sizeof(uint64_t) * L * P.qkv_rows);
+    o.attn = take(sizeof(uint64_t) * L * c.n_heads * c.head_dim);
+    o.xmid = take(sizeof(uint64_t) * L * c.hidden);
+    o.xout = take(sizeof(uint64_t) * L * c.hidden);
+    o.act = take(sizeof(uint64_t) * L * c.ffn);
     o.part = take(sizeof(float) * L * part);
-    o.attn = take(sizeof(float) * L * c.n_heads * c.head_dim);
-    o.xmid = take(sizeof(float) * L * c.hidden);
-    o.xout = take(sizeof(float) * L * c.hidden);
-    o.act = take(sizeof(float) * L * c.ffn);
     o.xacc = take(P.ffn_fused ? sizeof(long long) * L * c.hidden : 0);
     o.dmaps = take(P.ffn_fused ? 128 * L : 0);
     o.total = off;
@@ -101,6 +102,13 @@ struct UploadKey {
 constexpr int kMaxDevices = 64;
 std::mutex g_upload_mu;
 UploadKey g_uploaded[kMaxDevices];
+// The tag of the last step each device's array ran (every call takes the
+// next one), and the plan that ran it.  Plans lay the array out differently:
+// where this plan keeps flagged words another may have kept anything (a
+// fixed-point residual's high half is a small integer, like a tag), so the
+// flagged words are cleared whenever the plan changes.
+uint32_t g_fw_tag[kMaxDevices];
+uint64_t g_fw_plan[kMaxDevices];
 
 // FNV-1a over the weight pointers the task table holds.
 uint64_t weights_signature(const amk_config &c, const amk_weights *w)
@@ -287,6 +295,24 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     e = cudaMemsetAsync(base + lay.ctr, 0, lay.qkv - lay.ctr, st);
     if (e != cudaSuccess)
         return fail_cuda(e, "scratch clear");
+    // this step's tag; when the device's tags run out, the plan changed, or
+    // the device ordinal is beyond the table, the flagged words are cleared
+    // first
+    uint32_t tag = 1;
+    bool clear = true;
+    if (dev >= 0 && dev < kMaxDevices) {
+        std::lock_guard<std::mutex> lock(g_upload_mu);
+        tag = ++g_fw_tag[dev];
+        clear = tag == 0 || g_fw_plan[dev] != P.uid;
+        g_fw_plan[dev] = P.uid;
+        if (tag == 0)
+            tag = g_fw_tag[dev] = 1;
+    }
+    if (clear) {
+        e = cudaMemsetAsync(base + lay.qkv, 0, lay.part - lay.qkv, st);
+        if (e != cudaSuccess)
+            return fail_cuda(e, "scratch clear");
+    }
 
     amk::KParams k{};
     k.tasks = reinterpret_cast<const amk::TaskDesc *>(base + lay.tasks);
@@ -294,13 +320,13 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     k.counters = reinterpret_cast<uint32_t *>(base + lay.ctr);
     k.err = reinterpret_cast<amk::ErrorWord *>(base + lay.err);
     k.embed = static_cast<const uint16_t *>(w->embed);
-    k.qkv = reinterpret_cast<float *>(base + lay.qkv);
+    k.qkv = reinterpret_cast<uint64_t *>(base + lay.qkv);
     k.part = reinterpret_cast<float *>(base + lay.part);
-    k.attn = reinterpret_cast<float *>(base + lay.attn);
+    k.attn = reinterpret_cast<uint64_t *>(base + lay.attn);
     k.arrive = reinterpret_cast<uint32_t *>(base + lay.ctr) + P.n_counters;
-    k.xmid = reinterpret_cast<float *>(base + lay.xmid);
-    k.xout = reinterpret_cast<float *>(base + lay.xout);
-    k.act = reinterpret_cast<float *>(base + lay.act);
+    k.xmid = reinterpret_cast<uint64_t *>(base + lay.xmid);
+    k.xout = reinterpret_cast<uint64_t *>(base + lay.xout);
+    k.act = reinterpret_cast<uint64_t *>(base + lay.act);
     k.xacc = reinterpret_cast<long long *>(base + lay.xacc);
     k.dmaps = base + lay.dmaps;
     k.dpack = nullptr;  // no room for a packed copy: the tensor maps read the caller's Wdown
@@ -341,6 +367,8 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     k.parity = 0;
     k.timeout_ns = (uint64_t)P.opt.wait_timeout_us * 1000ull;
     k.skip_signal_task = P.opt.debug_skip_signal_task;
+    k.tag = tag;
+    k.flagged = P.flagged;
     k.lookahead = (uint32_t)(P.opt.l2_prefetch_kb > 0 ? P.opt.l2_prefetch_kb : 0) * 1024u;
     k.inflight = amk_inflight_bytes(&P.opt);
     k.piece = amk_piece_bytes(&P.opt);

@@ -21,6 +21,7 @@ struct amk_plan {
     int n_arrive = 0;    // attention arrival counters, [L][nkv], after them
     int att_pg = 1;      // attention position groups per warp
     int ffn_fused = 0;   // 1: one FFN level per layer (gate/up + down column slice)
+    int flagged = 0;     // 1: tasks wait on the flagged words they read, not on counters
     int ffn_box_rows = 0;  // rows of a Wdown TMA box (divides hidden)
     int is_pos0 = 0;     // 1: the schedule of steps at position 0 (no attention level)
     amk_plan *pos0 = nullptr;  // owned: that schedule, for a plan of all other steps

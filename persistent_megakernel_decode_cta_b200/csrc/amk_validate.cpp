@@ -16,6 +16,11 @@
 //    subsequence, which is exactly the condition under which the per-SM
 //    loops cannot deadlock.
 //  * "happens before" is reachability in that union graph.
+//  * A flagged read (the task polls the words themselves, each carrying the
+//    epoch's tag once its one writer stored it or its accumulators finished)
+//    is a wait on every task with a WRITE or ACCUM overlapping the range: it
+//    adds those edges to the graph (rule V10 makes sure there is exactly one
+//    value to wait for).
 //  * The pages' reader/writer rule is extended with the other conflicts a
 //    single-assignment step can have (write/write, accumulate, the previous
 //    step's value, resets for the next step) and with a coverage rule for
@@ -153,7 +158,7 @@ extern "C" int amk_validate_graph(const amk_graph *g, amk_validation_report *rep
             const amk_graph_access &a = g->accesses[k.access_begin + i];
             if (!in(a.buffer, 0, B))
                 return fail(AMK_RULE_V7, t, -1, -1, a.buffer, "task %d names a missing buffer", t);
-            if (a.kind < AMK_ACC_READ || a.kind > AMK_ACC_RESET)
+            if (a.kind < AMK_ACC_READ || a.kind > AMK_ACC_READ_FLAGGED)
                 return fail(AMK_RULE_V7, t, -1, -1, a.buffer, "task %d: bad access kind", t);
             if (a.begin < 0 || a.end <= a.begin || a.end > g->buffers[a.buffer].size)
                 return fail(AMK_RULE_V7, t, -1, -1, a.buffer,
@@ -188,10 +193,59 @@ extern "C" int amk_validate_graph(const amk_graph *g, amk_validation_report *rep
         }
     }
 
+    // accesses per buffer (sorted by start, then task)
+    std::vector<std::vector<Acc>> per_buf(B);
+    for (int t = 0; t < T; ++t) {
+        const amk_graph_task &k = g->tasks[t];
+        for (int i = 0; i < k.access_count; ++i) {
+            const amk_graph_access &a = g->accesses[k.access_begin + i];
+            per_buf[a.buffer].push_back({t, a.kind, a.begin, a.end});
+        }
+    }
+    for (auto &v : per_buf)
+        std::sort(v.begin(), v.end(), [](const Acc &x, const Acc &y) {
+            return x.b != y.b ? x.b < y.b : x.task < y.task;
+        });
+    auto is_w = [](int k) { return k == AMK_ACC_WRITE || k == AMK_ACC_ACCUM; };
+
+    // ---- V10: flagged reads find exactly one value per element ---------------
+    for (int b = 0; b < B; ++b) {
+        const auto &v = per_buf[b];
+        bool any = false;
+        for (const Acc &a : v)
+            any |= a.kind == AMK_ACC_READ_FLAGGED;
+        if (!any)
+            continue;
+        const int64_t n = g->buffers[b].size;
+        std::vector<int64_t> dw(n + 1, 0), da(n + 1, 0);  // difference arrays
+        for (const Acc &a : v) {
+            if (a.kind == AMK_ACC_WRITE)
+                ++dw[a.b], --dw[a.e];
+            else if (a.kind == AMK_ACC_ACCUM)
+                ++da[a.b], --da[a.e];
+        }
+        std::vector<int64_t> bad(n + 1, 0);  // prefix count of elements without one value
+        int64_t cw = 0, ca = 0;
+        for (int64_t x = 0; x < n; ++x) {
+            cw += dw[x];
+            ca += da[x];
+            const bool ok = (cw == 1 && ca == 0) || (cw == 0 && ca >= 1);
+            bad[x + 1] = bad[x] + (ok ? 0 : 1);
+        }
+        for (const Acc &a : v)
+            if (a.kind == AMK_ACC_READ_FLAGGED && bad[a.e] != bad[a.b])
+                return fail(AMK_RULE_V10, a.task, -1, -1, b,
+                            "task %d reads flagged elements of buffer %d in [%lld,%lld) that "
+                            "are not written exactly once (or only accumulated)", a.task, b,
+                            (long long)a.b, (long long)a.e);
+    }
+
     // ---- V1 / V4: acyclicity -------------------------------------------------
-    // nodes: tasks [0, T) then counters [T, T+C)
-    const int N = T + C;
-    std::vector<std::vector<int>> succ(N);
+    // nodes: tasks [0, T), counters [T, T+C), then one join node per set of
+    // more than kDirect writers that a flagged read waits for (edges writer ->
+    // join -> reader, like a counter's); smaller sets get direct edges
+    constexpr size_t kDirect = 8;
+    std::vector<std::vector<int>> succ(T + C);
     for (int t = 0; t < T; ++t) {
         const amk_graph_task &k = g->tasks[t];
         for (int i = 0; i < k.signal_count; ++i)
@@ -199,19 +253,58 @@ extern "C" int amk_validate_graph(const amk_graph *g, amk_validation_report *rep
         for (int i = 0; i < k.wait_count; ++i)
             succ[T + g->waits[k.wait_begin + i].counter].push_back(t);
     }
+    {
+        std::vector<std::pair<std::vector<int>, int>> joins;  // writer set -> node
+        for (int b = 0; b < B; ++b) {
+            const auto &v = per_buf[b];
+            for (const Acc &r : v) {
+                if (r.kind != AMK_ACC_READ_FLAGGED)
+                    continue;
+                std::vector<int> ws;
+                for (const Acc &w : v)
+                    if (is_w(w.kind) && w.b < r.e && r.b < w.e)
+                        ws.push_back(w.task);
+                std::sort(ws.begin(), ws.end());
+                ws.erase(std::unique(ws.begin(), ws.end()), ws.end());
+                if (ws.size() <= kDirect) {
+                    for (int w : ws)
+                        succ[w].push_back(r.task);
+                    continue;
+                }
+                int node = -1;
+                for (const auto &j : joins)
+                    if (j.first == ws) {
+                        node = j.second;
+                        break;
+                    }
+                if (node < 0) {
+                    node = (int)succ.size();
+                    succ.emplace_back();
+                    for (int w : ws)
+                        succ[w].push_back(node);
+                    joins.push_back({ws, node});
+                }
+                succ[node].push_back(r.task);
+            }
+        }
+    }
+    const int N = (int)succ.size();
     std::vector<int> order;
     int stuck = -1;
     if (!topo_sort(N, succ, order, &stuck))
-        return fail(AMK_RULE_V1, stuck < T ? stuck : -1, -1, stuck >= T ? stuck - T : -1, -1,
+        return fail(AMK_RULE_V1, stuck < T ? stuck : -1, -1,
+                    stuck >= T && stuck < T + C ? stuck - T : -1, -1,
                     "producer/consumer graph has a cycle (through %s %d)",
-                    stuck < T ? "task" : "counter", stuck < T ? stuck : stuck - T);
+                    stuck < T ? "task" : stuck < T + C ? "counter" : "flagged join",
+                    stuck < T ? stuck : stuck < T + C ? stuck - T : stuck - T - C);
     for (int s = 0; s < S; ++s)
         for (int i = g->queue_offsets[s]; i + 1 < g->queue_offsets[s + 1]; ++i)
             succ[g->queue_tasks[i]].push_back(g->queue_tasks[i + 1]);
     if (!topo_sort(N, succ, order, &stuck))
         return fail(AMK_RULE_V4, stuck < T ? stuck : -1, -1, -1, -1,
                     "per-SM queue order contradicts the dependency graph (near %s %d)",
-                    stuck < T ? "task" : "counter", stuck < T ? stuck : stuck - T);
+                    stuck < T ? "task" : stuck < T + C ? "counter" : "flagged join",
+                    stuck < T ? stuck : stuck < T + C ? stuck - T : stuck - T - C);
 
     // ---- happens-before closure over tasks (bitsets in topological order) ---
     const size_t W = ((size_t)T + 63) / 64;
@@ -231,19 +324,8 @@ extern "C" int amk_validate_graph(const amk_graph *g, amk_validation_report *rep
     };
 
     // ---- V5 / V6: conflicting accesses ---------------------------------------
-    std::vector<std::vector<Acc>> per_buf(B);
-    for (int t = 0; t < T; ++t) {
-        const amk_graph_task &k = g->tasks[t];
-        for (int i = 0; i < k.access_count; ++i) {
-            const amk_graph_access &a = g->accesses[k.access_begin + i];
-            per_buf[a.buffer].push_back({t, a.kind, a.begin, a.end});
-        }
-    }
-    for (auto &v : per_buf)
-        std::sort(v.begin(), v.end(), [](const Acc &x, const Acc &y) {
-            return x.b != y.b ? x.b < y.b : x.task < y.task;
-        });
-    auto is_w = [](int k) { return k == AMK_ACC_WRITE || k == AMK_ACC_ACCUM; };
+    // (a READ_FLAGGED follows its writers by its own edges; it is checked as a
+    // READ below, which it always passes, and against RESETs as any access)
     for (int pass = 5; pass <= 6; ++pass) {
         for (int b = 0; b < B; ++b) {
             const auto &v = per_buf[b];
@@ -255,7 +337,8 @@ extern "C" int amk_validate_graph(const amk_graph *g, amk_validation_report *rep
                     if (pass == 5) {
                         // every READ after every overlapping WRITE/ACCUM
                         for (int r = 0; r < 2; ++r, std::swap(x, y))
-                            if (x->kind == AMK_ACC_READ && is_w(y->kind) && !hb(y->task, x->task))
+                            if ((x->kind == AMK_ACC_READ || x->kind == AMK_ACC_READ_FLAGGED) &&
+                                is_w(y->kind) && !hb(y->task, x->task))
                                 return fail(AMK_RULE_V5, y->task, x->task, -1, b,
                                             "task %d reads buffer %d before writer %d is "
                                             "ordered before it", x->task, b, y->task);

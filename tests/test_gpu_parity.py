@@ -154,7 +154,7 @@ def test_full_size_single_steps(name, ctxs):
 @pytest.mark.parametrize("name,ctx,fused", [
     ("tinyllama", 256, 2),     # the fused FFN level where the default keeps it split
     ("llama7b_w8", 0, 2),
-    ("smol135", 128, -1),      # split levels where the default fuses
+    ("smol135", 128, 2),       # the fused level (level counters) where the default splits
     ("llama1b_w8", 512, 2),    # the fused int8 level (dp2a column loop), split by default
 ])
 def test_ffn_level_variants(name, ctx, fused):
@@ -306,22 +306,31 @@ def test_bad_arguments():
     assert e.value.name == "AMK_ERR_INVALID_ARG"
 
 
-def test_wait_timeout_is_reported_and_recoverable():
-    """Fault injection on the host: one task never signals its counter, so a
-    downstream wait runs out after its (short) limit; the kernel returns, the
-    call reports AMK_ERR_TIMEOUT, the handle is poisoned until reset, and after
-    a reset a normal handle decodes correctly again."""
+@pytest.mark.parametrize("flagged", [1, -1])
+def test_wait_timeout_is_reported_and_recoverable(flagged):
+    """Fault injection on the host: one task never signals (level counters:
+    its counter add is skipped; flagged waits: its flagged words carry a wrong
+    tag), so a downstream wait runs out after its (short) limit; the kernel
+    returns, the call reports AMK_ERR_TIMEOUT, the handle is poisoned until
+    reset, and after a reset a normal handle decodes correctly again.  The
+    general schedule runs at position 0 too, so that the attention level
+    reads the victim's rows."""
     cfg = si.get_config("tiny")
     plan = amk.Plan(cfg, 4)
     kinds, _ = plan.task_info()
     victim = kinds.index(1)  # a QKV task
-    opts = amk.default_options(n_sms=4, wait_timeout_us=20000, debug_skip_signal_task=victim)
+    opts = amk.default_options(n_sms=4, wait_timeout_us=20000, debug_skip_signal_task=victim,
+                               flagged_waits=flagged, pos0_plan=-1)
     pair = Pair(cfg, options=opts)
     with pytest.raises(amk.AmkError) as e:
         pair.dec.step(3, 0)
     assert e.value.name == "AMK_ERR_TIMEOUT"
     info = pair.dec.error_info()
-    assert info.code == 1 and info.counter >= 0
+    assert info.code == 1 and info.task >= 0
+    if flagged > 0:
+        assert info.counter == -1  # a flagged read gave up: no counter
+    else:
+        assert info.counter >= 0
     with pytest.raises(amk.AmkError) as e:
         pair.dec.step(3, 0)
     assert e.value.name == "AMK_ERR_POISONED"
@@ -330,6 +339,28 @@ def test_wait_timeout_is_reported_and_recoverable():
     good = Pair(cfg, weights=pair.w, options=amk.default_options(n_sms=4))
     g, am, ref, ref_am = good.step(3, 0)
     compare(cfg, g, am, ref, ref_am, "after timeout")
+
+
+@pytest.mark.parametrize("name,ctx,steps", [
+    ("tiny", 0, 6),
+    ("tinyllama", 256, 2),
+    ("llama1b_w8", 512, 2),
+    ("llama7b", 0, 2),
+])
+def test_level_counters_match_the_oracle(name, ctx, steps):
+    """The level-counter protocol (flagged_waits = -1) on models whose FFN
+    levels are split, where flagged waits are the default: the same logits
+    within the tolerance, steps chained on the device."""
+    cfg = si.get_config(name)
+    pair = Pair(cfg, options=amk.default_options(flagged_waits=-1))
+    if ctx:
+        pair.fill_kv(ctx)
+    prompt = si.make_prompt(cfg, steps)
+    for i, t in enumerate(prompt):
+        g, am, ref, ref_am = pair.step(t, ctx + i)
+        compare(cfg, g, am, ref, ref_am, what=f"{name} counters pos {ctx + i}")
+    del pair
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("name,ctx,steps", [

@@ -241,3 +241,22 @@ def test_sm_rotation_moves_tiles_not_balance():
     assert sorted(ka) == sorted(kb)
     assert sa != sb
     assert a.stats().weight_bytes == b.stats().weight_bytes
+
+
+@pytest.mark.parametrize("name,fused_with_counters", [
+    ("tinyllama", 0), ("llama7b", 0), ("llama1b_w8", 0), ("llama7b_w8", 0),
+    ("smol135", 1),  # residual rows of 1152 B: fused when the counters are asked for
+])
+def test_flagged_waits_resolution(name, fused_with_counters):
+    """Flagged waits with separate FFN levels are the default everywhere; with
+    flagged_waits = -1 the level counters come back, and with them the fused
+    FFN level on narrow residuals; a fused level (forced) always runs on the
+    counters (its residual is a fixed-point sum)."""
+    cfg = si.get_config(name)
+    st = amk.Plan(cfg, 148).stats()
+    assert (st.flagged_waits, st.ffn_fused) == (1, 0)
+    off = amk.Plan(cfg, 148, amk.default_options(flagged_waits=-1)).stats()
+    assert (off.flagged_waits, off.ffn_fused) == (0, fused_with_counters)
+    fused = amk.Plan(cfg, 148, amk.default_options(ffn_fused=2)).stats()
+    if fused.ffn_fused:
+        assert fused.flagged_waits == 0

@@ -16,7 +16,7 @@ import persistent_megakernel_decode_cta_b200 as amk
 from persistent_megakernel_decode_cta_b200 import build
 from oracle import interleave as bf
 
-R, W, A, RP, RS = bf.READ, bf.WRITE, bf.ACCUM, bf.READ_PREV, bf.RESET
+R, W, A, RP, RS, RF = bf.READ, bf.WRITE, bf.ACCUM, bf.READ_PREV, bf.RESET, bf.READ_FLAGGED
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -93,6 +93,10 @@ def random_schedule(rng: random.Random):
         for t in range(T):
             if writer in anc[t] and rng.random() < 0.5:
                 acc[t].append((b, R, rng.randint(lo, hi - 1), hi))
+            elif t != writer and rng.random() < 0.25:
+                # a flagged read orders itself after the writer (a cycle or a
+                # queue contradiction when t comes first: a deadlock)
+                acc[t].append((b, RF, rng.randint(lo, hi - 1), hi))
     if rng.random() < 0.5:
         bufs[0]["output"] = True
     if rng.random() < 0.3:
@@ -145,7 +149,8 @@ def mutate(g, rng: random.Random):
         b = rng.randrange(len(g["buffers"]))
         size = g["buffers"][b]["size"]
         lo = rng.randrange(size)
-        tasks[t]["accesses"].append((b, rng.choice([R, W, A]), lo, rng.randint(lo + 1, size)))
+        tasks[t]["accesses"].append((b, rng.choice([R, W, A, RF]), lo,
+                                     rng.randint(lo + 1, size)))
     elif kind == 6:                                   # dangling references
         choice = rng.randrange(4)
         if choice == 0:
@@ -263,3 +268,56 @@ def test_rule_examples():
     bufs = [{"size": 2, "output": False, "pair": 1}, {"size": 2, "output": False, "pair": -1}]
     assert agree(_g([T_(0, acc=[(0, A, 0, 2), (1, RS, 0, 1)])], [[0]], 0, bufs))[1] == "V9"
     assert agree(_g([T_(0, acc=[(0, A, 0, 2), (1, RS, 0, 2)])], [[0]], 0, bufs))[0]
+
+
+def test_flagged_read_examples():
+    """READ_FLAGGED: the reader waits for the words themselves (no counter):
+    ordered after every writer or accumulator of its range; rule V10 wants
+    exactly one value per element to wait for."""
+    buf = [{"size": 4, "output": False, "pair": -1}]
+    # valid: no counter at all, the flagged read orders the reader
+    assert agree(_g([T_(0, acc=[(0, W, 0, 4)]), T_(1, acc=[(0, RF, 0, 4)])],
+                    [[0], [1]], 0, buf))[0]
+    # valid: two writers of disjoint halves, one reader of the whole
+    assert agree(_g([T_(0, acc=[(0, W, 0, 2)]), T_(1, acc=[(0, W, 2, 4)]),
+                     T_(2, acc=[(0, RF, 0, 4)])], [[0], [1], [2]], 0, buf))[0]
+    # valid: accumulated elements (the flag comes when the accumulation ends)
+    assert agree(_g([T_(0, acc=[(0, A, 0, 2)]), T_(1, acc=[(0, A, 0, 2)]),
+                     T_(2, acc=[(0, RF, 0, 2)])], [[0], [1], [2]], 0, buf))[0]
+    # V10: an element nobody writes (the reader would wait for ever)
+    assert agree(_g([T_(0, acc=[(0, W, 0, 2)]), T_(1, acc=[(0, RF, 0, 3)])],
+                    [[0], [1]], 0, buf))[1] == "V10"
+    # V10: an element written twice (the reader could take the first value)
+    assert agree(_g([T_(0, signals=[0], acc=[(0, W, 0, 2)]),
+                     T_(1, waits=[(0, 1)], acc=[(0, W, 1, 2)]),
+                     T_(2, acc=[(0, RF, 0, 2)])], [[0], [1], [2]], 1, buf))[1] == "V10"
+    # V10: written and accumulated
+    assert agree(_g([T_(0, acc=[(0, W, 0, 2)]), T_(1, acc=[(0, A, 0, 2)]),
+                     T_(2, acc=[(0, RF, 0, 2)])], [[0], [1], [2]], 0, buf))[1] == "V10"
+    # V1: a task that flag-reads its own output
+    assert agree(_g([T_(0, acc=[(0, W, 0, 2), (0, RF, 0, 2)])], [[0]], 0, buf))[1] == "V1"
+    # V1: two tasks flag-reading each other's output
+    bufs = [{"size": 2, "output": False, "pair": -1}, {"size": 2, "output": False, "pair": -1}]
+    assert agree(_g([T_(0, acc=[(0, W, 0, 2), (1, RF, 0, 2)]),
+                     T_(1, acc=[(1, W, 0, 2), (0, RF, 0, 2)])], [[0], [1]], 0,
+                    bufs))[1] == "V1"
+    # V4: the reader is queued before its writer on the same SM
+    assert agree(_g([T_(0, acc=[(0, W, 0, 2)]), T_(0, acc=[(0, RF, 0, 2)])], [[1, 0]], 0,
+                    buf))[1] == "V4"
+    # a flagged read does not order the reader against a later reset
+    bufs = [{"size": 2, "output": False, "pair": -1}]
+    assert agree(_g([T_(0, acc=[(0, W, 0, 2)]), T_(1, acc=[(0, RF, 0, 2)]),
+                     T_(2, acc=[(0, RS, 0, 2)])], [[0], [1], [2]], 0, bufs))[1] == "V6"
+
+
+def test_flagged_join_nodes_scale():
+    """A level of many writers and many full-width flagged readers (the
+    shape of a decode layer) validates quickly: the readers of one writer set
+    share a join node."""
+    n = 64
+    buf = [{"size": n, "output": False, "pair": -1}]
+    tasks = [T_(i, acc=[(0, W, i, i + 1)]) for i in range(n)]
+    tasks += [T_(i, acc=[(0, RF, 0, n)]) for i in range(n)]
+    queues = [[i, n + i] for i in range(n)]
+    ok, rule, msg = amk.validate_graph(_g(tasks, queues, 0, buf))
+    assert ok, (rule, msg)

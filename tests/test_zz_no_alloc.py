@@ -8,10 +8,12 @@ The tests call it through the C ABI several times in a row (positions 0, 1,
 ... so that each call reads the KV rows the earlier ones wrote) and check
 logits, greedy token and KV cache against the allocating entry point
 amk_decode_step, within the parity tolerance the other GPU tests use, and
-the logits against the fp64 oracle directly.  The SmolLM2 shapes run the
-fused FFN level, whose Wdown tiles come through tensor maps kept in the
-static array (bf16 and int8 maps); two such models with different weights
-alternate on it.  This file is collected last.
+the logits against the fp64 oracle directly.  The "_fused" SmolLM2 cases
+run the fused FFN level (options ffn_fused = 2, with the level counters),
+whose Wdown tiles come through tensor maps kept in the static array (bf16
+and int8 maps); the others run the default schedule (separate FFN levels,
+flagged waits).  Two fused models with different weights alternate on the
+array.  This file is collected last.
 """
 import ctypes
 
@@ -53,20 +55,27 @@ def _weights_struct(cfg, w):
 
 
 def _config(name):
+    """(config, options) of a test case name."""
+    opts = None
+    if name.endswith("_fused"):
+        name = name[:-len("_fused")]
+        opts = amk.default_options(ffn_fused=2)
     if name == "tiny_w8":
-        return si.get_config("tiny").with_(quant="w8a16", name="tiny_w8")
+        return si.get_config("tiny").with_(quant="w8a16", name="tiny_w8"), opts
     if name == "smol135_w8":
-        return si.get_config("smol135").with_(quant="w8a16", name="smol135_w8")
-    return si.get_config(name)
+        return si.get_config("smol135").with_(quant="w8a16", name="smol135_w8"), opts
+    return si.get_config(name), opts
 
 
 class NoAlloc:
     """A caller of amk_decode_step_noalloc: its own KV cache and logits."""
 
-    def __init__(self, cfg, w):
+    def __init__(self, cfg, w, options=None):
         self.cfg = cfg
         sms = torch.cuda.get_device_properties(0).multi_processor_count
-        self.plan = amk.Plan(cfg, sms)
+        self.plan = amk.Plan(cfg, sms, options)
+        if options is not None and options.ffn_fused == 2:
+            assert self.plan.stats().ffn_fused == 1
         self.ws, self.keep = _weights_struct(cfg, w)
         self.kv = torch.zeros((cfg.n_layers, 2, cfg.n_kv_heads, cfg.max_ctx, cfg.head_dim),
                               dtype=torch.bfloat16, device="cuda")
@@ -86,16 +95,17 @@ class NoAlloc:
         self.plan.close()
 
 
-@pytest.mark.parametrize("name", ["tiny", "tiny_w8", "smol135", "smol135_w8"])
+@pytest.mark.parametrize("name", ["tiny", "tiny_w8", "smol135", "smol135_fused",
+                                  "smol135_w8_fused"])
 def test_noalloc_matches_allocating_entry_point(name):
-    cfg = _config(name)
+    cfg, opts = _config(name)
     w = si.make_model(cfg, device="cuda")
     n = 4
     toks = si.make_prompt(cfg, n)
     tol = (2e-2 if cfg.quant == "w8a16" else 1e-2)
 
     # reference: the allocating entry point
-    dec = amk.Decoder(cfg, w)
+    dec = amk.Decoder(cfg, w, opts)
     ref_logits, ref_tok = [], []
     lg = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
     for pos, t in enumerate(toks):
@@ -105,7 +115,7 @@ def test_noalloc_matches_allocating_entry_point(name):
     dec.close()
 
     # the no-allocation entry point: caller-owned KV cache and logits
-    na = NoAlloc(cfg, w)
+    na = NoAlloc(cfg, w, opts)
     for pos, t in enumerate(toks):
         g, am = na.step(t, pos)
         r = ref_logits[pos].double().cpu().numpy()
@@ -117,15 +127,15 @@ def test_noalloc_matches_allocating_entry_point(name):
     na.close()
 
 
-@pytest.mark.parametrize("name", ["tiny", "smol135", "smol135_w8"])
+@pytest.mark.parametrize("name", ["tiny", "smol135", "smol135_fused", "smol135_w8_fused"])
 def test_noalloc_matches_oracle(name):
     """The no-allocation step against the fp64 oracle on the same bytes,
-    element by element, at positions 0..3 (the SmolLM2 shapes run the fused
-    FFN level through the tensor maps in the static array)."""
-    cfg = _config(name)
+    element by element, at positions 0..3 (the fused cases run the FFN level
+    through the tensor maps in the static array)."""
+    cfg, opts = _config(name)
     w = si.make_model(cfg, device="cuda")
     ref = orc.OracleModel(cfg, w)
-    na = NoAlloc(cfg, w)
+    na = NoAlloc(cfg, w, opts)
     for pos, t in enumerate(si.make_prompt(cfg, 4)):
         g, am = na.step(t, pos)
         r, r_am, _ = ref.step(t, pos)
@@ -138,10 +148,11 @@ def test_noalloc_two_models_alternate():
     one static array: every call re-writes the Wdown tensor maps there, and
     each model's logits must still be its own."""
     cfg = si.get_config("smol135")
+    opts = amk.default_options(ffn_fused=2)
     ws = [si.make_model(cfg, seed=s, device="cuda") for s in (0, 7)]
     refs = []
     for w in ws:
-        dec = amk.Decoder(cfg, w)
+        dec = amk.Decoder(cfg, w, opts)
         lg = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
         out = []
         for pos, t in enumerate(si.make_prompt(cfg, 3)):
@@ -149,7 +160,7 @@ def test_noalloc_two_models_alternate():
             out.append(lg.double().cpu().numpy())
         dec.close()
         refs.append(out)
-    nas = [NoAlloc(cfg, w) for w in ws]
+    nas = [NoAlloc(cfg, w, opts) for w in ws]
     for pos, t in enumerate(si.make_prompt(cfg, 3)):
         for i in (0, 1):
             g, _ = nas[i].step(t, pos)
