@@ -331,13 +331,14 @@ AMK_API int amk_plan_get_stats(const amk_plan *p, amk_plan_stats *out);
 
 /* Introspection for tests: device pointers (owned by the handle) to the
  * activations the last step left, per layer l, as flagged words (64 bits:
- * the fp32 value in the low half, the step's tag in the high half):
+ * the fp32 value in the low half, the step's tag in the high half; act: 32
+ * bits, the fp32 value with its 8 low mantissa bits replaced by an 8-bit tag):
  *   qkv  [n_layers][qkv_rows]  q | k | v before RoPE, qkv_rows = (n_heads + 2*n_kv_heads)*head_dim
  *   xmid [n_layers][hidden]    residual stream after attention
  *   xout [n_layers][hidden]    residual stream after the FFN (with a fused FFN level
  *                              the residual after it lives in a fixed-point buffer instead)
  *   act  [n_layers][ffn]       SwiGLU activations (unused with a fused FFN level) */
-typedef struct { uint64_t *qkv, *xmid, *xout, *act; int32_t qkv_rows; } amk_workspace;
+typedef struct { uint64_t *qkv, *xmid, *xout; uint32_t *act; int32_t qkv_rows; } amk_workspace;
 AMK_API int amk_get_workspace(amk_handle *h, amk_workspace *out);
 
 /* Phase timers of the last step, recorded when amk_options.profile was 1

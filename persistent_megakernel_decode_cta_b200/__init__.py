@@ -325,8 +325,8 @@ class Decoder:
 
     def workspace(self) -> Dict[str, object]:
         """fp32 views of the last step's activations: qkv [L, qkv_rows],
-        xmid / xout [L, hidden], act [L, ffn] (the value halves of the
-        flagged words)."""
+        xmid / xout [L, hidden], act [L, ffn] (the values of the flagged
+        words; act's with 15 mantissa bits)."""
         import torch
         ws = abi.Workspace()
         _check(abi.lib().amk_get_workspace(self._h, ctypes.byref(ws)), "amk_get_workspace")
@@ -336,8 +336,10 @@ class Decoder:
             w = torch.as_tensor(_DevArray(p, (L, n, 2), "<f4"), device="cuda")
             return w[:, :, 0]
 
+        act = torch.as_tensor(_DevArray(ws.act, (L, self.cfg.ffn), "<i4"), device="cuda")
+        act = (act & ~0xFF).view(torch.float32)  # drop the 8-bit tag
         return {"qkv": view(ws.qkv, ws.qkv_rows), "xmid": view(ws.xmid, self.cfg.hidden),
-                "xout": view(ws.xout, self.cfg.hidden), "act": view(ws.act, self.cfg.ffn)}
+                "xout": view(ws.xout, self.cfg.hidden), "act": act}
 
     def profile(self):
         """Phase timers of the last step (needs options.profile = 1): a uint64

@@ -175,8 +175,9 @@ struct amk_handle {
     uint32_t *d_ctr0 = nullptr;
     uint32_t epoch0 = 0;  // steps run with it since the last reset
     ErrorWord *d_err = nullptr;
-    uint64_t *d_qkv = nullptr, *d_attn = nullptr, *d_xmid = nullptr, *d_xout = nullptr,
-             *d_act = nullptr;  // flagged words
+    uint64_t *d_qkv = nullptr, *d_attn = nullptr, *d_xmid = nullptr,
+             *d_xout = nullptr;  // flagged words
+    uint32_t *d_act = nullptr;  // 32-bit flagged words
     float *d_part = nullptr, *d_logits = nullptr;
     uint32_t tag = 0;  // tag of the last step's flagged words (0: none yet)
     unsigned long long *d_argkey = nullptr;
@@ -440,11 +441,11 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     const size_t attn_f = (size_t)L * c.n_heads * hd;
     const size_t h_f = (size_t)L * c.hidden, act_f = (size_t)L * c.ffn;
     H->kv_bytes = (size_t)L * 2 * nkv * c.max_ctx * hd * sizeof(uint16_t);
-    // activations in one block: xacc (int64) | qkv | attn | xmid | xout | act
-    // (flagged words, 8 bytes each) | part (fp32)
+    // activations in one block: xacc (int64) | qkv | attn | xmid | xout
+    // (flagged words, 8 bytes each) | act (32-bit flagged words) | part (fp32)
     const size_t xacc_b = P->ffn_fused ? (size_t)L * c.hidden * sizeof(long long) : 0;
-    const size_t words = qkv_f + attn_f + 2 * h_f + act_f;
-    H->fw_bytes = words * sizeof(uint64_t);
+    const size_t words = qkv_f + attn_f + 2 * h_f;
+    H->fw_bytes = words * sizeof(uint64_t) + act_f * sizeof(uint32_t);
     H->act_bytes = xacc_b + H->fw_bytes + part_f * sizeof(float);
     float *act_block = nullptr;
     if ((rc = dalloc(H, &H->d_tasks, sizeof(TaskDesc) * P->tasks.size())) ||
@@ -473,7 +474,7 @@ extern "C" int amk_create(const amk_config *cfg, const amk_weights *w, const amk
     H->d_attn = H->d_qkv + qkv_f;
     H->d_xmid = H->d_attn + attn_f;
     H->d_xout = H->d_xmid + h_f;
-    H->d_act = H->d_xout + h_f;
+    H->d_act = reinterpret_cast<uint32_t *>(H->d_xout + h_f);
     H->d_part = reinterpret_cast<float *>(H->d_act + act_f);
     if ((e = cudaMallocHost(&H->h_err, sizeof(ErrorWord))) != cudaSuccess ||
         (e = cudaMallocHost(&H->h_key, 2 * sizeof(unsigned long long))) != cudaSuccess ||

@@ -142,7 +142,8 @@ struct KParams {
     uint64_t *attn;   // [L][nh * hd]: attention output, the chunks merged (flagged)
     uint64_t *xmid;   // [L][h]: residual after attention (flagged)
     uint64_t *xout;   // [L][h]: residual after the FFN (flagged)
-    uint64_t *act;    // [L][ffn]: SwiGLU activations (flagged)
+    uint32_t *act;    // [L][ffn]: SwiGLU activations, 32-bit flagged words (the fp32
+                      // value's low 8 bits replaced by the step's 8-bit tag)
     long long *xacc;  // [L][h]: residual after the FFN in fixed point (value * 2^32), when
                       // the FFN level is fused: OPROJ writes the residual, FFN slices add
     const void *dmaps;  // [L] 128-byte tensor maps of Wdown (fused FFN), 64-byte aligned

@@ -152,7 +152,6 @@ __device__ __forceinline__ void red_release_add(uint32_t *p, uint32_t v)
 {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
-constexpr int kFwRoundWords = 48;  // flagged words a GEMV lane loads in one round
 // Flagged words carry a value from one level to the next: the fp32 value in
 // the low half and the tag of the step that wrote it in the high half of one
 // aligned 64-bit word, stored and loaded as single relaxed accesses at GPU
@@ -180,6 +179,36 @@ __device__ __forceinline__ void fw_ld2(const uint64_t *a, uint64_t &x, uint64_t 
 }
 __device__ __forceinline__ float fw_val(uint64_t w) { return __uint_as_float((uint32_t)w); }
 __device__ __forceinline__ bool fw_ok(uint64_t w, uint32_t tag) { return (uint32_t)(w >> 32) == tag; }
+// The SwiGLU activations, read by every SM in full for the down projection,
+// are 32-bit flagged words instead (half the bytes to load and to poll): the
+// fp32 value with its 8 low mantissa bits replaced by an 8-bit step tag in
+// 1 .. 255 (consecutive steps differ; cleared memory never matches), so a
+// value keeps 15 mantissa bits, a relative step of 2^-15 -- finer than the
+// int16 steps the int8 / int4 GEMV takes its activations in, and than the
+// bf16 weights they multiply.
+__device__ __forceinline__ uint32_t fw8_tag(uint32_t tag) { return tag % 255u + 1u; }
+__device__ __forceinline__ void fw32_st(uint32_t *a, float v, uint32_t t8)
+{
+    const uint32_t w = (__float_as_uint(v) & ~0xffu) | t8;
+    asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(a), "r"(w) : "memory");
+}
+// four consecutive words (16-byte aligned), each loaded as its own access
+__device__ __forceinline__ void fw32_ld4(const uint32_t *a, uint32_t (&w)[4])
+{
+    asm volatile("ld.relaxed.gpu.global.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                 : "l"(a)
+                 : "memory");
+}
+__device__ __forceinline__ void fw32_ld2(const uint32_t *a, uint32_t (&w)[2])
+{
+    asm volatile("ld.relaxed.gpu.global.v2.b32 {%0, %1}, [%2];"
+                 : "=r"(w[0]), "=r"(w[1])
+                 : "l"(a)
+                 : "memory");
+}
+__device__ __forceinline__ float fw32_val(uint32_t w) { return __uint_as_float(w & ~0xffu); }
+__device__ __forceinline__ bool fw32_ok(uint32_t w, uint32_t t8) { return (w & 0xffu) == t8; }
 // The residual after a fused FFN level is held in fixed point (value * 2^32
 // in an int64): integer addition is associative, so the FFN slices' partial
 // down projections add up to the same bits in any order.  |value| < 2^31.
@@ -1031,74 +1060,92 @@ __device__ __forceinline__ bool fw_gather(const KParams &p, const SmemLayout &s,
     return true;
 }
 
-// A GEMV lane's activations from a flagged vector: vector v = vb + lane +
-// 32 i (i < ni; zeros for the others) holds the E elements at xg + v E, read
-// two words at a time.  The vectors go in rounds of RI (a round's raw words
-// take two registers each, so a lane with 64 activations reads them in two
-// rounds); every load of a round goes out before any word of it is looked at.
+// A GEMV lane's activations from the 32-bit flagged SwiGLU words: vector
+// v = vb + lane + 32 i (i < ni; zeros for the others) holds the E elements at
+// xg + v E, read G = min(E, 4) words at a time, in rounds of RI vectors (a
+// bf16 or int8 lane with more than 48 activations takes two, to bound the
+// registers a round holds; an int4 lane's 64 take one);
+// every load of a round goes out before any word of it is looked at, and
+// groups still without this step's tag are loaded again until all have it.
 template <int NI, int E, int RI>
 __device__ __forceinline__ bool fw_lane_round(const KParams &p, const SmemLayout &s,
-                                              const uint64_t *xg, int vb, int ni, int lane,
+                                              const uint32_t *xg, int vb, int ni, int lane,
                                               int i0, float (&xf)[NI][E])
 {
-    constexpr int H = E / 2;
-    static_assert(RI * H <= 32, "pending bits");
-    const uint32_t tag = p.tag;
-    uint64_t wa[RI][H], wb[RI][H];
-    const uint64_t none = (uint64_t)tag << 32;  // a zero with this step's tag
+    constexpr int G = E < 4 ? E : 4;
+    constexpr int H = E / G;  // groups per vector
+    static_assert(E % G == 0 && (G == 2 || G == 4) && RI * H <= 32, "pending bits");
+    const uint32_t t8 = fw8_tag(p.tag);
+    uint32_t w[RI][H][G];
 #pragma unroll
     for (int r = 0; r < RI; ++r) {
-        const int i = i0 + r;
-        const uint64_t *vp = xg + (size_t)(vb + lane + 32 * i) * E;
+        const uint32_t *vp = xg + (size_t)(vb + lane + 32 * (i0 + r)) * E;
 #pragma unroll
-        for (int e = 0; e < H; ++e) {
-            wa[r][e] = wb[r][e] = none;
-            if (i < ni)
-                fw_ld2(vp + 2 * e, wa[r][e], wb[r][e]);
+        for (int h = 0; h < H; ++h) {
+#pragma unroll
+            for (int q = 0; q < G; ++q)
+                w[r][h][q] = t8;  // a zero with this step's tag
+            if (i0 + r < ni) {
+                if constexpr (G == 4)
+                    fw32_ld4(vp + 4 * h, w[r][h]);
+                else
+                    fw32_ld2(vp + 2 * h, w[r][h]);
+            }
         }
     }
     uint32_t pend = 0u;
 #pragma unroll
     for (int r = 0; r < RI; ++r)
 #pragma unroll
-        for (int e = 0; e < H; ++e) {
-            xf[i0 + r][2 * e] = fw_val(wa[r][e]);
-            xf[i0 + r][2 * e + 1] = fw_val(wb[r][e]);
-            if (!fw_ok(wa[r][e], tag) || !fw_ok(wb[r][e], tag))
-                pend |= 1u << (r * H + e);
+        for (int h = 0; h < H; ++h) {
+            bool ok = true;
+#pragma unroll
+            for (int q = 0; q < G; ++q) {
+                xf[i0 + r][G * h + q] = fw32_val(w[r][h][q]);
+                ok = ok && fw32_ok(w[r][h][q], t8);
+            }
+            if (!ok)
+                pend |= 1u << (r * H + h);
         }
     uint64_t t0 = 0;
-    // (the words are usually there by the first load once the task's inputs
-    // are complete; the compiler is told so, to keep this loop out of the
-    // straight-line code)
     for (uint32_t it = 0; __builtin_expect(pend != 0u, 0); ++it) {
         if (it == 0)
             t0 = gtimer();
 #pragma unroll
         for (int r = 0; r < RI; ++r) {
-            const uint64_t *vp = xg + (size_t)(vb + lane + 32 * (i0 + r)) * E;
+            const uint32_t *vp = xg + (size_t)(vb + lane + 32 * (i0 + r)) * E;
 #pragma unroll
-            for (int e = 0; e < H; ++e)
-                if (pend & (1u << (r * H + e)))
-                    fw_ld2(vp + 2 * e, wa[r][e], wb[r][e]);
+            for (int h = 0; h < H; ++h)
+                if (pend & (1u << (r * H + h))) {
+                    if constexpr (G == 4)
+                        fw32_ld4(vp + 4 * h, w[r][h]);
+                    else
+                        fw32_ld2(vp + 2 * h, w[r][h]);
+                }
         }
-        uint64_t last = 0;
+        uint32_t last = 0;
 #pragma unroll
         for (int r = 0; r < RI; ++r)
 #pragma unroll
-            for (int e = 0; e < H; ++e) {
-                const uint32_t bit = 1u << (r * H + e);
+            for (int h = 0; h < H; ++h) {
+                const uint32_t bit = 1u << (r * H + h);
                 if (pend & bit) {
-                    if (fw_ok(wa[r][e], tag) && fw_ok(wb[r][e], tag)) {
-                        xf[i0 + r][2 * e] = fw_val(wa[r][e]);
-                        xf[i0 + r][2 * e + 1] = fw_val(wb[r][e]);
+                    bool ok = true;
+#pragma unroll
+                    for (int q = 0; q < G; ++q)
+                        ok = ok && fw32_ok(w[r][h][q], t8);
+                    if (ok) {
+#pragma unroll
+                        for (int q = 0; q < G; ++q)
+                            xf[i0 + r][G * h + q] = fw32_val(w[r][h][q]);
                         pend &= ~bit;
                     } else {
-                        last = fw_ok(wa[r][e], tag) ? wb[r][e] : wa[r][e];
+                        last = w[r][h][0];
                     }
                 }
             }
-        if (pend && (it & 15) == 15 && fw_give_up(p, s, t0, last, it))
+        if (pend && (it & 15) == 15 &&
+            fw_give_up(p, s, t0, (uint64_t)(last & 0xffu) << 32, it))
             return false;
     }
     if (t0)
@@ -1106,18 +1153,16 @@ __device__ __forceinline__ bool fw_lane_round(const KParams &p, const SmemLayout
     return true;
 }
 
-template <int NI, int E, int W = kFwRoundWords>
+template <int NI, int E>
 __device__ __forceinline__ bool fw_lane_vectors(const KParams &p, const SmemLayout &s,
-                                                const uint64_t *xg, int vb, int ni, int lane,
+                                                const uint32_t *xg, int vb, int ni, int lane,
                                                 float (&xf)[NI][E])
 {
-    // one round up to W words, else rounds of at most min(W, 32)
-    constexpr int WR = W < 32 ? W : 32;
-    constexpr int RI = NI * E <= W ? NI : (WR / E > 0 ? WR / E : 1);
-#pragma unroll
-    for (int i0 = 0; i0 < NI; i0 += RI)
-        if (!fw_lane_round<NI, E, (RI < NI ? RI : NI)>(p, s, xg, vb, ni, lane, i0, xf))
-            return false;
+    constexpr int RI = NI * E > 48 && E < 32 && NI > 1 ? (NI + 1) / 2 : NI;
+    if (!fw_lane_round<NI, E, RI>(p, s, xg, vb, ni, lane, 0, xf))
+        return false;
+    if constexpr (RI < NI)
+        return fw_lane_round<NI, E, NI - RI>(p, s, xg, vb, ni, lane, RI, xf);
     return true;
 }
 
@@ -1212,7 +1257,7 @@ __device__ void rmsnorm_prologue(const KParams &p, const SmemLayout &s, const ui
 // shared vector (prologue output) or, when xg is set, straight from L2.
 template <int ESZ, int VB>
 __device__ __forceinline__ bool gemv_task(const KParams &p, const SmemLayout &s, const Geom g,
-                                          RingPos &kc, int warp, int lane, const uint64_t *xg,
+                                          RingPos &kc, int warp, int lane, const uint32_t *xg,
                                           uint64_t *wt)
 {
     constexpr int E = VB / ESZ;   // elements per vector (even)
@@ -1231,7 +1276,7 @@ __device__ __forceinline__ bool gemv_task(const KParams &p, const SmemLayout &s,
     f2_t xp[NI][EP];
     if (xg) {
         float xf[NI][E];
-        if (!fw_lane_vectors<NI, E, 16>(p, s, xg, vb, ni, lane, xf))
+        if (!fw_lane_vectors<NI, E>(p, s, xg, vb, ni, lane, xf))
             return false;
 #pragma unroll
         for (int i = 0; i < NI; ++i)
@@ -1537,9 +1582,9 @@ __device__ __forceinline__ void gemv_rows(const LaneX<ESZ, NI> &x, uint32_t stag
 // transposed shuffle reduction serves the four rows.  NI (vectors a lane
 // holds) is a template parameter so that the activation registers are sized
 // to the shape, not to the largest one.
-template <int ESZ, int NI, int W = kFwRoundWords>
+template <int ESZ, int NI>
 __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &s, const Geom g,
-                                            RingPos &kc, int warp, int lane, const uint64_t *xg,
+                                            RingPos &kc, int warp, int lane, const uint32_t *xg,
                                             uint64_t *wt)
 {
     using LX = LaneX<ESZ, NI>;
@@ -1555,7 +1600,7 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
     {
         float xf[NI][E];
         if (xg) {
-            if (!fw_lane_vectors<NI, E, W>(p, s, xg, vb, ni, lane, xf))
+            if (!fw_lane_vectors<NI, E>(p, s, xg, vb, ni, lane, xf))
                 return false;
         } else {
 #pragma unroll
@@ -1683,33 +1728,33 @@ __device__ __forceinline__ bool gemv16_task(const KParams &p, const SmemLayout &
 }
 
 // Dispatch on the vectors a lane holds for this task's K-slice.
-template <int ESZ, int W = kFwRoundWords>
+template <int ESZ>
 __device__ __forceinline__ bool gemv16(const KParams &p, const SmemLayout &s, const Geom &g,
-                                       RingPos &kc, int warp, int lane, const uint64_t *xg,
+                                       RingPos &kc, int warp, int lane, const uint32_t *xg,
                                        uint64_t *wt)
 {
     const int vps = ((ESZ ? g.RB >> 4 : g.K >> 5) + g.KS - 1) >> g.ks_log2;
     const int nimax = (vps + 31) >> 5;
     if constexpr (ESZ == 0) {
         if (nimax <= 1)
-            return gemv16_task<0, 1, W>(p, s, g, kc, warp, lane, xg, wt);
-        return gemv16_task<0, 2, W>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<0, 1>(p, s, g, kc, warp, lane, xg, wt);
+        return gemv16_task<0, 2>(p, s, g, kc, warp, lane, xg, wt);
     } else if constexpr (ESZ == 2) {
         if (nimax <= 2)
-            return gemv16_task<2, 2, W>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<2, 2>(p, s, g, kc, warp, lane, xg, wt);
         if (nimax <= 4)
-            return gemv16_task<2, 4, W>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<2, 4>(p, s, g, kc, warp, lane, xg, wt);
         if (nimax <= 6)
-            return gemv16_task<2, 6, W>(p, s, g, kc, warp, lane, xg, wt);
-        return gemv16_task<2, 8, W>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<2, 6>(p, s, g, kc, warp, lane, xg, wt);
+        return gemv16_task<2, 8>(p, s, g, kc, warp, lane, xg, wt);
     } else {
         if (nimax <= 1)
-            return gemv16_task<1, 1, W>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<1, 1>(p, s, g, kc, warp, lane, xg, wt);
         if (nimax <= 2)
-            return gemv16_task<1, 2, W>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<1, 2>(p, s, g, kc, warp, lane, xg, wt);
         if (nimax <= 3)
-            return gemv16_task<1, 3, W>(p, s, g, kc, warp, lane, xg, wt);
-        return gemv16_task<1, 4, W>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16_task<1, 3>(p, s, g, kc, warp, lane, xg, wt);
+        return gemv16_task<1, 4>(p, s, g, kc, warp, lane, xg, wt);
     }
 }
 
@@ -1718,7 +1763,7 @@ __device__ __forceinline__ bool gemv16(const KParams &p, const SmemLayout &s, co
 // time (models with odd row widths, or a bf16 tied head on int8 layers).
 template <int Q8, int GENERIC>
 __device__ __forceinline__ bool run_gemv(const KParams &p, const SmemLayout &s, const Geom &g,
-                                         RingPos &kc, int warp, int lane, const uint64_t *xg,
+                                         RingPos &kc, int warp, int lane, const uint32_t *xg,
                                          uint64_t *wt)
 {
     if constexpr (!GENERIC) {
@@ -1732,17 +1777,15 @@ __device__ __forceinline__ bool run_gemv(const KParams &p, const SmemLayout &s, 
             return gemv16<2>(p, s, g, kc, warp, lane, xg, wt);
         }
     } else {
-        // (smaller rounds of flagged activation loads: this instance holds
-        // every path, and the registers are shared by all of them)
         if (g.esz == 2) {
             if (g.VB == 16)
-                return gemv16<2, 16>(p, s, g, kc, warp, lane, xg, wt);
+                return gemv16<2>(p, s, g, kc, warp, lane, xg, wt);
             if (g.VB == 8)
                 return gemv_task<2, 8>(p, s, g, kc, warp, lane, xg, wt);
             return gemv_task<2, 4>(p, s, g, kc, warp, lane, xg, wt);
         }
         if (g.VB == 16)
-            return gemv16<1, 16>(p, s, g, kc, warp, lane, xg, wt);
+            return gemv16<1>(p, s, g, kc, warp, lane, xg, wt);
         if (g.VB == 8)
             return gemv_task<1, 8>(p, s, g, kc, warp, lane, xg, wt);
         return gemv_task<1, 4>(p, s, g, kc, warp, lane, xg, wt);
@@ -2679,7 +2722,7 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
                         const float gt = row_total(s, g, t) * sc0;
                         const float up = row_total(s, g, g.R + t) * sc1;
                         const float silu = gt / (1.f + __expf(-gt));
-                        fw_st(p.act + (size_t)l * p.ffn + d.r0 + t, silu * up, otag);
+                        fw32_st(p.act + (size_t)l * p.ffn + d.r0 + t, silu * up, fw8_tag(otag));
                     }
                 } else if (d.kind == TK_DOWN) {
                     if (ct < g.R)

@@ -62,7 +62,7 @@ Layout layout_of(const amk_plan &P)
     o.attn = take(sizeof(uint64_t) * L * c.n_heads * c.head_dim);
     o.xmid = take(sizeof(uint64_t) * L * c.hidden);
     o.xout = take(sizeof(uint64_t) * L * c.hidden);
-    o.act = take(sizeof(uint64_t) * L * c.ffn);
+    o.act = take(sizeof(uint32_t) * L * c.ffn);
     o.part = take(sizeof(float) * L * part);
     o.xacc = take(P.ffn_fused ? sizeof(long long) * L * c.hidden : 0);
     o.dmaps = take(P.ffn_fused ? 128 * L : 0);
@@ -326,7 +326,7 @@ extern "C" int amk_decode_step_noalloc(const amk_plan *plan, const amk_weights *
     k.arrive = reinterpret_cast<uint32_t *>(base + lay.ctr) + P.n_counters;
     k.xmid = reinterpret_cast<uint64_t *>(base + lay.xmid);
     k.xout = reinterpret_cast<uint64_t *>(base + lay.xout);
-    k.act = reinterpret_cast<uint64_t *>(base + lay.act);
+    k.act = reinterpret_cast<uint32_t *>(base + lay.act);
     k.xacc = reinterpret_cast<long long *>(base + lay.xacc);
     k.dmaps = base + lay.dmaps;
     k.dpack = nullptr;  // no room for a packed copy: the tensor maps read the caller's Wdown

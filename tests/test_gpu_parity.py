@@ -341,24 +341,25 @@ def test_wait_timeout_is_reported_and_recoverable(flagged):
     compare(cfg, g, am, ref, ref_am, "after timeout")
 
 
-@pytest.mark.parametrize("name,ctx,steps", [
-    ("tiny", 0, 6),
-    ("tinyllama", 256, 2),
-    ("llama1b_w8", 512, 2),
-    ("llama7b", 0, 2),
+@pytest.mark.parametrize("name,ctx,steps,mode", [
+    ("tiny", 0, 6, -1),
+    ("tinyllama", 256, 2, -1),
+    ("llama1b_w8", 512, 2, -1),
+    ("llama7b", 0, 2, -1),
+    ("smol135_w4", 0, 2, -1),
 ])
-def test_level_counters_match_the_oracle(name, ctx, steps):
+def test_wait_protocols_match_the_oracle(name, ctx, steps, mode):
     """The level-counter protocol (flagged_waits = -1) on models whose FFN
     levels are split, where flagged waits are the default: the same logits
     within the tolerance, steps chained on the device."""
     cfg = si.get_config(name)
-    pair = Pair(cfg, options=amk.default_options(flagged_waits=-1))
+    pair = Pair(cfg, options=amk.default_options(flagged_waits=mode))
     if ctx:
         pair.fill_kv(ctx)
     prompt = si.make_prompt(cfg, steps)
     for i, t in enumerate(prompt):
         g, am, ref, ref_am = pair.step(t, ctx + i)
-        compare(cfg, g, am, ref, ref_am, what=f"{name} counters pos {ctx + i}")
+        compare(cfg, g, am, ref, ref_am, what=f"{name} waits {mode} pos {ctx + i}")
     del pair
     torch.cuda.empty_cache()
 
