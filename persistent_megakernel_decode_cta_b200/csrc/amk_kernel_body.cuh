@@ -189,7 +189,11 @@ __device__ __forceinline__ bool fw_ok(uint64_t w, uint32_t tag) { return (uint32
 __device__ __forceinline__ uint32_t fw8_tag(uint32_t tag) { return tag % 255u + 1u; }
 __device__ __forceinline__ void fw32_st(uint32_t *a, float v, uint32_t t8)
 {
-    const uint32_t w = (__float_as_uint(v) & ~0xffu) | t8;
+    // round to the nearest 15-bit mantissa (half away from zero: the add
+    // carries into the exponent when the mantissa overflows), then the tag;
+    // truncating instead biased every value toward zero, and the down
+    // projection's long sums added that bias up
+    const uint32_t w = ((__float_as_uint(v) + 0x80u) & ~0xffu) | t8;
     asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(a), "r"(w) : "memory");
 }
 // four consecutive words (16-byte aligned), each loaded as its own access
