@@ -536,7 +536,9 @@ def run_noalloc(args):
     w = si.make_model(cfg, seed=0, device="cuda")
     kv_fill = si.make_kv_fill(cfg, ctx, device="cuda") if ctx else None
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    plan = amk.Plan(cfg, sms)
+    owner = amk.Plan(cfg, sms)
+    # at position 0 the caller runs the position-0 schedule, as amk_decode_step does
+    plan = (owner.pos0() or owner) if ctx == 0 else owner
     ws, keep = amk.weights_struct(cfg, w)
     kv = torch.zeros((cfg.n_layers, 2, cfg.n_kv_heads, cfg.max_ctx, cfg.head_dim),
                      dtype=torch.bfloat16, device="cuda")
@@ -586,9 +588,10 @@ def run_noalloc(args):
         "host_us_per_call": {"p50": float(np.percentile(host, 50) * 1e6),
                              "p90": float(np.percentile(host, 90) * 1e6)},
         "amk_decode_step_us_per_call": alloc_us,
-        "schedule_upload_bytes_per_call": table, "tasks": st.n_tasks,
+        "schedule_table_bytes": table,  # uploaded when the plan, weights or KV change "tasks": st.n_tasks,
     }), flush=True)
     plan.close()
+    owner.close()
 
 
 def main():
