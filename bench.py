@@ -26,6 +26,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -74,10 +75,16 @@ def algorithmic_bytes(cfg, ctx: int) -> int:
     return si.streamed_weight_bytes(cfg) + kv_row * ctx + kv_row + cfg.vocab * 4
 
 
-def kernel_hash() -> str:
+def kernel_hash(sources=None) -> str:
+    """Hash of the kernel's code: the sources with their comments and blank
+    space removed, so that a profile stays attached to the code it measured
+    when only the commentary changes."""
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
-        h.update(open(os.path.join(ROOT, p), "rb").read())
+    for p in (sources or [os.path.join(ROOT, q) for q in KERNEL_SOURCES]):
+        text = open(p, encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -115,7 +115,9 @@ typedef struct {
     int32_t tasks_per_sm;     /* GEMV row tiles per SM per level; 0 = auto */
     int32_t n_sms;            /* persistent CTAs; 0 = all SMs of the device */
     uint32_t wait_timeout_us; /* limit of every device-side wait */
-    int32_t debug_skip_signal_task; /* test hook: this task id never signals; -1 = off */
+    int32_t debug_skip_signal_task; /* test hook: this task id never signals (level
+                                 counters: no add; flagged waits: its flagged words carry
+                                 a wrong tag), so a later wait runs out; -1 = off */
     int32_t profile;          /* 1: record per-CTA phase timers (amk_get_profile) */
     int32_t l2_prefetch_kb;   /* while its ring is full, each SM prefetches this many KiB
                                  of its coming weight stream into L2; 0 = off */
@@ -372,7 +374,8 @@ AMK_API int amk_get_profile(amk_handle *h, uint64_t *out, int64_t n_u64);
 AMK_API int amk_check_guards(amk_handle *h, int32_t *n_bad);
 
 /* After AMK_ERR_TIMEOUT: the task that gave up, the counter it waited on,
- * the value it saw and the value it needed. */
+ * the value it saw and the value it needed (a flagged read that gave up:
+ * counter -1, the tag it last saw and the step's tag). */
 typedef struct { int32_t code, task, counter, sm; uint32_t seen, target; } amk_error_info;
 AMK_API int amk_get_error_info(amk_handle *h, amk_error_info *out);
 

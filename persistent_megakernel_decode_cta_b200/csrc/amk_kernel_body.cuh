@@ -6,12 +6,16 @@
 //
 // One launch = one forward pass = one token ("RightNow-AI/AutoMegaKernel"
 // README, opening summary).  One CTA per SM walks its own queue of tasks in a
-// global topological order: wait on a counter -> run the task -> signal a
-// counter (gist.science technical summary, "Methodologie", layer 0; paperfeed
-// review, "How it works").  Producers only increment counters and consumers
-// only wait for statically known thresholds (README, "Deadlock-free by
-// construction").  Weights of upcoming tasks are prefetched while the current
-// one computes (README, "Why a megakernel").
+// global topological order: wait for the inputs -> run the task -> hand the
+// outputs on (gist.science technical summary, "Methodologie", layer 0;
+// paperfeed review, "How it works").  The pages wait on counters with
+// statically known thresholds (README, "Deadlock-free by construction"); by
+// default this kernel waits on the data itself instead: every vector a level
+// hands to the next is made of flagged words (value + step tag in one word,
+// see fw_st / fw32_st), and a task's poll of the words it reads is its wait.
+// The counter protocol remains for the fused FFN level and on request.
+// Weights of upcoming tasks are prefetched while the current one computes
+// (README, "Why a megakernel").
 //
 // B200 design (not the pages' sm_80..sm_120 design):
 //  * 384 threads per CTA in three warpgroups.  The producer warpgroup gives
@@ -20,14 +24,15 @@
 //    ring of shared-memory stages with cp.async.bulk (TMA bulk copies) that
 //    complete on per-stage mbarriers.  Weights never depend on activations,
 //    so the copies run ahead across counter waits.
-//  * Two consumer warpgroups (8 warps) take the freed registers.  They wait
-//    on the task's counter (ld.acquire.gpu spin with a time limit), build
-//    the task's input vector in shared memory (RMSNorm / split-K combine
-//    prologues, from L2 with .cg loads), run the GEMV from the ring -- each
-//    warp owns a K-slice whose activations sit in registers -- reduce with
-//    warp shuffles, apply the fused epilogue (RoPE + KV append, SwiGLU,
-//    residual add, argmax), then release their stores with red.release.gpu
-//    on the task's counter.
+//  * Two consumer warpgroups (8 warps) take the freed registers.  They poll
+//    the flagged words of the task's inputs (or, with level counters, spin
+//    on the task's counter with ld.acquire.gpu; both with a time limit),
+//    build the task's input vector in shared memory (RMSNorm / attention
+//    output prologues), run the GEMV from the ring -- each warp owns a
+//    K-slice whose activations sit in registers -- reduce with warp
+//    shuffles, and apply the fused epilogue (RoPE + KV append, SwiGLU,
+//    residual add, argmax), whose flagged stores are the task's signal (with
+//    level counters: a red.release.gpu on the task's counter).
 //  * Task records carry host-resolved pointers and are prefetched one task
 //    ahead, so no task boundary waits on a dependent global load.
 //  * Every wait is bounded (globaltimer + iteration cap); on expiry the CTA
@@ -2567,7 +2572,7 @@ __device__ __forceinline__ void consumer_loop(const KParams &p, const SmemLayout
         if (wprof)
             wt_store[0] = wt_store[1] = 0;
         // loads that do not depend on this step's activations go out before
-        // the counter wait: the RMSNorm gains and the int8 row scales of the
+        // the task's wait: the RMSNorm gains and the int8 row scales of the
         // epilogue (thread t finalises row r0 + t; R <= 256)
         const Geom g = task_geom(p, d);
         // (kept as raw bits until first use: a conversion here would wait for
