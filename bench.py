@@ -486,7 +486,8 @@ def run_ours(args):
             "dtype": {"w8a16": "int8 weights x int16 activations, i32 then f32 accumulate",
                       "w4a16": "int4 weights (fp16 group scales) x int16 activations, "
                                "i32 then f32 accumulate"}.get(
-                          cfg.quant, "bf16 weights x f32 activations, f32 accumulate"),
+                          cfg.quant, "bf16 weights x f32 activations (the SwiGLU vector "
+                          "handed over at 15 mantissa bits), f32 accumulate"),
             "data": "synthetic (seeded random-init weights and KV cache)",
             "config": dict(workload_config(name, cfg, ctx),
                            parallelism=f"replicas{world}" if world > 1 else "single"),
