@@ -422,11 +422,10 @@ AMK_API int amk_read_ceiling(const void *buf, int64_t bytes, int32_t n_sms, int3
  * scratch would exceed AMK_NOALLOC_SCRATCH_BYTES (amk_last_error says how
  * much it needs), and when cuda_stream is capturing (the schedule uploads
  * read host stack memory).  AMK_ERR_INVALID_ARG for the position-0 schedule
- * (amk_plan_pos0) at any pos other than 0.  The first call on each device is
- * the set-up: it looks up the static array's device address
- * (cudaGetSymbolAddress, which may load the library's device code), so make
- * that first call before any stream capture; later calls look the address
- * up again, so it stays right after a cudaDeviceReset.  A call uploads the
+ * (amk_plan_pos0) at any pos other than 0.  Every call looks up the static
+ * array's device address (cudaGetSymbolAddress; the first lookup on a device
+ * may load the library's device code), so the address stays right after a
+ * cudaDeviceReset.  A call uploads the
  * schedule (the task table resolved against w and kv_cache) into the shared
  * array unless the previous call on the device left the same plan's table
  * there, resolved against the same pointers in the same CUDA context; every
