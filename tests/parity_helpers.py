@@ -5,6 +5,12 @@ Tolerances are the ones the workload states for this path: max |logit
 difference| <= 1e-2 * max |logit| for bf16 weights and 2e-2 * max |logit| for
 W8A16; greedy tokens must match wherever the oracle's top-2 margin exceeds
 that bound (elsewhere both candidates are correct).
+
+Every comparison is also held to DRIFT_GUARD of that bound. Over the whole GPU
+suite the largest error measured on B200 is 0.25 of it (SmolLM2 bf16 at
+position 0; W8A16 at most 0.21, W4A16 0.17), and the kernel's sums run in a
+fixed order, so a change that doubles an error fails here even while it is
+still inside the workload's tolerance.
 """
 from __future__ import annotations
 
@@ -14,6 +20,9 @@ import torch
 import oracle as orc
 import persistent_megakernel_decode_cta_b200 as amk
 import synth_inputs as si
+
+
+DRIFT_GUARD = 0.5
 
 
 def tol_frac(cfg) -> float:
@@ -57,6 +66,9 @@ def compare(cfg, g, am, ref, ref_am, what=""):
     err = np.abs(g - ref).max()
     tol = tol_frac(cfg) * scale
     assert err <= tol, f"{what}: max|dlogit| {err:.4g} > {tol:.4g} (max|logit| {scale:.4g})"
+    assert err <= DRIFT_GUARD * tol, (
+        f"{what}: max|dlogit| {err:.4g} is {err / tol:.3f} of the tolerance {tol:.4g}: inside "
+        f"the workload's bound but above the drift guard of {DRIFT_GUARD} of it")
     top2 = np.sort(ref)[-2:]
     margin = top2[1] - top2[0]
     if margin > tol:
