@@ -14,3 +14,16 @@ def test_kernel_hash_ignores_comments_not_code(tmp_path):
     assert bench.kernel_hash([str(a)]) == bench.kernel_hash([str(b)])
     assert bench.kernel_hash([str(a)]) != bench.kernel_hash([str(c)])
 
+
+
+def test_traffic_is_reported_only_for_the_code_it_was_taken_on(tmp_path, monkeypatch):
+    import json
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"w": {"kernel_hash": "aaaa", "dram_bytes_per_launch": 123}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_hash", lambda sources=None: "aaaa")
+    assert bench.load_traffic("w") == 123
+    assert bench.load_traffic("other") is None
+    monkeypatch.setattr(bench, "kernel_hash", lambda sources=None: "bbbb")
+    assert bench.load_traffic("w") is None
