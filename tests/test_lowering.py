@@ -117,10 +117,17 @@ def test_fused_ffn_slices_cover_ffn():
         assert n == -(-cfg.ffn // w) and n <= 148, (name, n)
 
 
-def test_small_real_lowering_passes_brute_force():
+@pytest.mark.parametrize("flagged", [1, -1])
+@pytest.mark.parametrize("pos0", [False, True])
+def test_small_real_lowering_passes_brute_force(flagged, pos0):
+    """Every interleaving of a one-layer lowering is safe, with the waits on
+    the flagged words (default) or on the level counters, and for the
+    general schedule as for the position-0 one (no attention level)."""
     cfg = si.get_config("tiny").with_(n_layers=1, name="tiny1")
-    opts = amk.default_options(attn_splits=1)
-    g = amk.Plan(cfg, 2, opts).graph()
+    opts = amk.default_options(attn_splits=1, flagged_waits=flagged)
+    plan = amk.Plan(cfg, 2, opts)
+    assert plan.stats().flagged_waits == (1 if flagged > 0 else 0)
+    g = (plan.pos0() if pos0 else plan).graph()
     assert len(g["tasks"]) <= 14
     assert bf.check(g) == (True, "ok")
 
