@@ -189,9 +189,10 @@ __device__ __forceinline__ bool fw_ok(uint64_t w, uint32_t tag) { return (uint32
 // fp32 value with its 8 low mantissa bits replaced by an 8-bit step tag in
 // 1 .. 255 (consecutive steps differ; cleared memory never matches, and
 // every such word is rewritten every step, so a stale one is one step old
-// and never passes), so a value keeps 15 mantissa bits, a relative step of
-// 2^-15 -- finer than the int16 steps the int8 / int4 GEMV takes its
-// activations in, and than the bf16 weights they multiply.
+// and never passes), so a value keeps 15 mantissa bits, rounded to nearest
+// (a relative error of at most 2^-16) -- finer than the int16 steps the
+// int8 / int4 GEMV takes its activations in, and than the bf16 weights they
+// multiply.
 __device__ __forceinline__ uint32_t fw8_tag(uint32_t tag) { return tag % 255u + 1u; }
 __device__ __forceinline__ void fw32_st(uint32_t *a, float v, uint32_t t8)
 {
