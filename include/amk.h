@@ -161,7 +161,11 @@ typedef struct {
                                  (B200: 4% faster on Llama-7B at context 2048, 7% on
                                  TinyLlama at 0, 8% on SmolLM2 at 128).  -1, or a fused
                                  FFN level: the level counters (release-add by each task,
-                                 acquire-poll by the next level's) */
+                                 acquire-poll by the next level's).  With the FFN level
+                                 split (either protocol), the SwiGLU vector goes to the
+                                 down projection as 32-bit words: the fp32 value rounded to 15 mantissa bits (a
+                                 relative error of at most 2^-16), an 8-bit tag in its
+                                 low byte */
 } amk_options;
 
 typedef struct amk_handle amk_handle;
